@@ -1,0 +1,336 @@
+/*
+ * LatentMoE forward oracle -- TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.
+ *
+ * A plain, slow, double-precision CPU restatement of what the LatentMoE
+ * feed-forward layer computes.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file's library.  It shares no
+ * code, header, table or helper with the CUDA library; the two meet only
+ * through the seeded inputs of the `synth` module.
+ *
+ * Sources (the K3 repository pages):
+ *   [sec07]  notes/sections/sec-07.tex, chapter "SiTU-GLU 与 Stable LatentMoE":
+ *            the SiTU-GLU formula and its property table, the five-step compute
+ *            flow (latent compression, K3 eq.13 routing, routed experts, shared
+ *            experts, merge), the routing notes, and the sparse-dispatch
+ *            subsection.
+ *   [diff]   compare view 584f7e9..main, kda/layers/latent_moe.py:
+ *            SiTU.forward, LatentMoE._route, LatentMoE._routed_u,
+ *            LatentMoE.forward.
+ *   [tests]  same compare view, tests/integration/test_k3_arch.py:
+ *            _dense_moe_forward and test_moe_router_activates_topk_only.
+ *
+ * Precision: every input arrives as float (bf16 inputs are the exact bf16
+ * values widened to float); every product and sum is formed in double and
+ * the outputs are double.  No blocking, fusion or reordering beyond the
+ * formulas: each token is computed on its own, slots in order i = 0..k-1.
+ *
+ * Readings where the pages leave a step open:
+ *   - TopK order: keys sorted descending, a tie goes to the lower expert index
+ *     ([diff] uses torch.topk, which returns values sorted descending).
+ *   - RMSNorm (its file is not on the pages): u * (1/sqrt(mean(u^2) + eps)) * w.
+ *   - The clamp of the routing denominator at 1e-9 is kept ([diff] _route).
+ *   - Routed and shared experts may have different hidden widths (F and G).
+ *
+ * Parity pins for every function are in tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+  int64_t n_tokens;  /* N = B*T                                   */
+  int32_t d;         /* model width                               */
+  int32_t latent;    /* l = d/2                                   */
+  int32_t n_routed;  /* R                                         */
+  int32_t top_k;     /* k                                         */
+  int32_t n_shared;  /* S                                         */
+  int32_t ff_routed; /* F: routed expert hidden width             */
+  int32_t ff_shared; /* G: shared expert hidden width             */
+  double beta1;      /* SiTU gate soft cap (4)                    */
+  double beta2;      /* SiTU up soft cap (25)                     */
+  double rms_eps;    /* RMSNorm epsilon                           */
+} orc_dims;
+
+/* Logistic function.  The two branches are the same function; the second
+ * avoids overflow of exp(-v) for very negative v. */
+static double orc_sigmoid(double v) {
+  if (v >= 0.0) return 1.0 / (1.0 + exp(-v));
+  double e = exp(v);
+  return e / (1.0 + e);
+}
+
+/* nn.Linear without bias: y[o] = sum_i W[o, i] * v[i], W stored [out, in]. */
+static void orc_linear(const float* W, int64_t out, int64_t in, const double* v, double* y) {
+  for (int64_t o = 0; o < out; ++o) {
+    const float* row = W + o * in;
+    double acc = 0.0;
+    for (int64_t i = 0; i < in; ++i) acc += (double)row[i] * v[i];
+    y[o] = acc;
+  }
+}
+
+/* SiTU-GLU expert ([sec07] SiTU formula; [diff] SiTU.forward):
+ *   a = W_g v,  c = W_u v,
+ *   gate = beta1 * tanh(a / beta1) * sigmoid(a)      (sigmoid of a, not a/beta1)
+ *   up   = beta2 * tanh(c / beta2)
+ *   out  = W_o (gate * up)
+ * w_g, w_u: [ff, dim_in]; w_o: [dim_in, ff].  `hidden` (optional) receives
+ * gate*up, the quantity whose magnitude the property table bounds by beta1*beta2. */
+void orc_situ(int32_t dim_in, int32_t ff, double beta1, double beta2,
+              const float* w_g, const float* w_u, const float* w_o,
+              const double* v, double* out, double* hidden) {
+  double* a = (double*)malloc(sizeof(double) * (size_t)ff);
+  double* c = (double*)malloc(sizeof(double) * (size_t)ff);
+  double* h = (double*)malloc(sizeof(double) * (size_t)ff);
+  orc_linear(w_g, ff, dim_in, v, a);
+  orc_linear(w_u, ff, dim_in, v, c);
+  for (int32_t j = 0; j < ff; ++j) {
+    double gate = beta1 * tanh(a[j] / beta1) * orc_sigmoid(a[j]);
+    double up = beta2 * tanh(c[j] / beta2);
+    h[j] = gate * up;
+  }
+  orc_linear(w_o, dim_in, ff, h, out);
+  if (hidden) memcpy(hidden, h, sizeof(double) * (size_t)ff);
+  free(a);
+  free(c);
+  free(h);
+}
+
+/* Router for one token ([sec07] compute flow step 2, K3 eq.13; [diff] _route):
+ *   l = W_r x,  s = sigmoid(l),  T = TopK(s + b, k),
+ *   p_i = s_i / max(sum_{j in T} s_j, 1e-9).
+ * The bias b enters the selection only; p uses the raw scores s.
+ * ids/probs: [k] in slot order (key descending, ties to the lower index).
+ * keys (optional): [R] receives s + b. */
+static void orc_route_token(int32_t d, int32_t R, int32_t k, const float* x, const float* w_r,
+                            const float* bias, int32_t* ids, double* probs, double* keys_out,
+                            double* scores_out) {
+  double* l = (double*)malloc(sizeof(double) * (size_t)R);
+  double* s = (double*)malloc(sizeof(double) * (size_t)R);
+  double* key = (double*)malloc(sizeof(double) * (size_t)R);
+  char* taken = (char*)calloc((size_t)R, 1);
+  double* xv = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int32_t i = 0; i < d; ++i) xv[i] = (double)x[i];
+  orc_linear(w_r, R, d, xv, l);
+  for (int32_t e = 0; e < R; ++e) {
+    s[e] = orc_sigmoid(l[e]);
+    key[e] = s[e] + (bias ? (double)bias[e] : 0.0);
+  }
+  /* k rounds of "largest remaining key"; strict '>' keeps the lower index on a tie. */
+  for (int32_t slot = 0; slot < k; ++slot) {
+    int32_t best = -1;
+    for (int32_t e = 0; e < R; ++e) {
+      if (taken[e]) continue;
+      if (best < 0 || key[e] > key[best]) best = e;
+    }
+    taken[best] = 1;
+    ids[slot] = best;
+  }
+  double den = 0.0;
+  for (int32_t slot = 0; slot < k; ++slot) den += s[ids[slot]];
+  if (den < 1e-9) den = 1e-9;
+  for (int32_t slot = 0; slot < k; ++slot) probs[slot] = s[ids[slot]] / den;
+  if (keys_out) memcpy(keys_out, key, sizeof(double) * (size_t)R);
+  if (scores_out) memcpy(scores_out, s, sizeof(double) * (size_t)R);
+  free(l);
+  free(s);
+  free(key);
+  free(taken);
+  free(xv);
+}
+
+/* Routing for all N tokens.  keys (optional): [N, R] = s + b.  scores
+ * (optional): [N, R] = s. */
+void orc_route(const orc_dims* dm, const float* x, const float* w_r, const float* bias,
+               int32_t* ids, double* probs, double* keys, double* scores) {
+  const int64_t N = dm->n_tokens;
+  const int32_t d = dm->d, R = dm->n_routed, k = dm->top_k;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t t = 0; t < N; ++t) {
+    orc_route_token(d, R, k, x + t * d, w_r, bias, ids + t * k, probs + t * k,
+                    keys ? keys + t * R : NULL, scores ? scores + t * R : NULL);
+  }
+}
+
+/* Token-expert pair permutation ([diff] _routed_u; [sec07] sparse dispatch,
+ * step 1): the N*k pairs (t, ids[t, i]) are flattened token-major and sorted
+ * by expert id with a stable sort, so that the pairs of one expert are
+ * contiguous and, inside an expert, in ascending token order.
+ *   counts[e]   = number of pairs with expert e          (bincount)
+ *   offsets[e]  = sum_{e' < e} counts[e'], offsets[R] = N*k (cumsum - counts)
+ *   perm_token[r] = token of the r-th pair in sorted order
+ *   inv_pair[t*k + i] = sorted position r of the pair (t, ids[t, i])
+ * Written as the textbook counting sort, which is a stable sort. */
+void orc_permute(int64_t N, int32_t k, int32_t R, const int32_t* ids, int32_t* counts,
+                 int32_t* offsets, int32_t* perm_token, int32_t* inv_pair) {
+  for (int32_t e = 0; e < R; ++e) counts[e] = 0;
+  for (int64_t p = 0; p < N * k; ++p) counts[ids[p]] += 1;
+  offsets[0] = 0;
+  for (int32_t e = 0; e < R; ++e) offsets[e + 1] = offsets[e] + counts[e];
+  int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)R);
+  for (int32_t e = 0; e < R; ++e) cursor[e] = offsets[e];
+  for (int64_t p = 0; p < N * k; ++p) { /* token-major order: p = t*k + i */
+    int32_t e = ids[p];
+    int32_t r = cursor[e]++;
+    perm_token[r] = (int32_t)(p / k);
+    inv_pair[p] = r;
+  }
+  free(cursor);
+}
+
+/* RMSNorm over one vector: out = u * (1/sqrt(mean(u^2) + eps)) * w. */
+static void orc_rmsnorm(int32_t n, const double* u, const float* w, double eps, double* out) {
+  double ms = 0.0;
+  for (int32_t j = 0; j < n; ++j) ms += u[j] * u[j];
+  ms /= (double)n;
+  double inv = 1.0 / sqrt(ms + eps);
+  for (int32_t j = 0; j < n; ++j) out[j] = u[j] * inv * (double)w[j];
+}
+
+/* Weights in the pages' nn.Linear layout ([out, in], K contiguous). */
+typedef struct {
+  const float* w_down;     /* [l, d]      W_down: d -> l                    */
+  const float* w_router;   /* [R, d]      W_r                               */
+  const float* w_up;       /* [d, l]      W_up: l -> d                      */
+  const float* rms_weight; /* [l]                                           */
+  const float* expert_bias;/* [R] or NULL (= 0)                             */
+  const float* w_g;        /* [R, F, l]   routed gate projections           */
+  const float* w_u;        /* [R, F, l]   routed up projections             */
+  const float* w_o;        /* [R, l, F]   routed output projections         */
+  const float* ws_g;       /* [S, G, d]   shared gate projections           */
+  const float* ws_u;       /* [S, G, d]   shared up projections             */
+  const float* ws_o;       /* [S, d, G]   shared output projections         */
+} orc_weights;
+
+/* Per-token forward ([sec07] compute flow, five steps; [diff] LatentMoE.forward):
+ *   1. z = W_down x
+ *   2. routing (K3 eq.13), see orc_route_token
+ *   3. u = sum_{i in T} p_i * E_i(z)           (routed SiTU experts in l)
+ *   4. s_sh = sum_j E^sh_j(x)                  (shared SiTU experts in d)
+ *   5. y = s_sh + W_up RMSNorm(u)
+ * Optional outputs (NULL to skip): z [N,l], u [N,l], uhat [N,l], shared [N,d],
+ * routed_out [N,k,l] (E_{ids[t,i]}(z_t) before weighting). */
+static void orc_forward_token(const orc_dims* dm, const orc_weights* w, const float* x_t,
+                              double* y_t, int32_t* ids_t, double* probs_t, double* z_t_out,
+                              double* u_t_out, double* uhat_t_out, double* sh_t_out,
+                              double* routed_t_out) {
+  const int32_t d = dm->d, L = dm->latent, R = dm->n_routed, k = dm->top_k;
+  const int32_t F = dm->ff_routed, S = dm->n_shared, G = dm->ff_shared;
+  double* xv = (double*)malloc(sizeof(double) * (size_t)d);
+  double* z = (double*)malloc(sizeof(double) * (size_t)L);
+  double* u = (double*)calloc((size_t)L, sizeof(double));
+  double* e_out = (double*)malloc(sizeof(double) * (size_t)L);
+  double* uhat = (double*)malloc(sizeof(double) * (size_t)L);
+  double* sh = (double*)calloc((size_t)d, sizeof(double));
+  double* sh_j = (double*)malloc(sizeof(double) * (size_t)d);
+  double* up = (double*)malloc(sizeof(double) * (size_t)d);
+
+  for (int32_t i = 0; i < d; ++i) xv[i] = (double)x_t[i];
+  /* step 1: latent compression */
+  orc_linear(w->w_down, L, d, xv, z);
+  /* step 2: routing on the full-width x (not z) */
+  orc_route_token(d, R, k, x_t, w->w_router, w->expert_bias, ids_t, probs_t, NULL, NULL);
+  /* step 3: routed experts, slots in order */
+  for (int32_t slot = 0; slot < k; ++slot) {
+    const int64_t e = ids_t[slot];
+    orc_situ(L, F, dm->beta1, dm->beta2, w->w_g + e * F * L, w->w_u + e * F * L,
+             w->w_o + e * L * F, z, e_out, NULL);
+    for (int32_t j = 0; j < L; ++j) u[j] += probs_t[slot] * e_out[j];
+    if (routed_t_out) memcpy(routed_t_out + (int64_t)slot * L, e_out, sizeof(double) * (size_t)L);
+  }
+  /* step 4: shared experts on x */
+  for (int32_t j = 0; j < S; ++j) {
+    orc_situ(d, G, dm->beta1, dm->beta2, w->ws_g + (int64_t)j * G * d,
+             w->ws_u + (int64_t)j * G * d, w->ws_o + (int64_t)j * d * G, xv, sh_j, NULL);
+    for (int32_t i = 0; i < d; ++i) sh[i] += sh_j[i];
+  }
+  /* step 5: merge */
+  orc_rmsnorm(L, u, w->rms_weight, dm->rms_eps, uhat);
+  orc_linear(w->w_up, d, L, uhat, up);
+  for (int32_t i = 0; i < d; ++i) y_t[i] = sh[i] + up[i];
+
+  if (z_t_out) memcpy(z_t_out, z, sizeof(double) * (size_t)L);
+  if (u_t_out) memcpy(u_t_out, u, sizeof(double) * (size_t)L);
+  if (uhat_t_out) memcpy(uhat_t_out, uhat, sizeof(double) * (size_t)L);
+  if (sh_t_out) memcpy(sh_t_out, sh, sizeof(double) * (size_t)d);
+  free(xv);
+  free(z);
+  free(u);
+  free(e_out);
+  free(uhat);
+  free(sh);
+  free(sh_j);
+  free(up);
+}
+
+void orc_forward(const orc_dims* dm, const orc_weights* w, const float* x, double* y,
+                 int32_t* ids, double* probs, double* z_out, double* u_out, double* uhat_out,
+                 double* shared_out, double* routed_out) {
+  const int64_t N = dm->n_tokens;
+  const int32_t d = dm->d, L = dm->latent, k = dm->top_k;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t t = 0; t < N; ++t) {
+    orc_forward_token(dm, w, x + t * d, y + t * d, ids + t * k, probs + t * k,
+                      z_out ? z_out + t * L : NULL, u_out ? u_out + t * L : NULL,
+                      uhat_out ? uhat_out + t * L : NULL, shared_out ? shared_out + t * d : NULL,
+                      routed_out ? routed_out + t * (int64_t)k * L : NULL);
+  }
+}
+
+/* Dense evaluation ([tests] _dense_moe_forward; the removed forward in
+ * [diff]): every routed expert runs on every token, all_out[t, e] = E_e(z_t),
+ * then u_t = sum_i p_i * all_out[t, ids[t, i]].  The pages test that it
+ * equals the sparse dispatch.  ids/probs come from the same router. */
+void orc_forward_dense(const orc_dims* dm, const orc_weights* w, const float* x, double* y,
+                       double* u_out) {
+  const int64_t N = dm->n_tokens;
+  const int32_t d = dm->d, L = dm->latent, R = dm->n_routed, k = dm->top_k;
+  const int32_t F = dm->ff_routed, S = dm->n_shared, G = dm->ff_shared;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t t = 0; t < N; ++t) {
+    const float* x_t = x + t * d;
+    double* xv = (double*)malloc(sizeof(double) * (size_t)d);
+    double* z = (double*)malloc(sizeof(double) * (size_t)L);
+    double* all_out = (double*)malloc(sizeof(double) * (size_t)R * (size_t)L);
+    double* u = (double*)calloc((size_t)L, sizeof(double));
+    double* uhat = (double*)malloc(sizeof(double) * (size_t)L);
+    double* sh = (double*)calloc((size_t)d, sizeof(double));
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)d);
+    int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* probs = (double*)malloc(sizeof(double) * (size_t)k);
+    for (int32_t i = 0; i < d; ++i) xv[i] = (double)x_t[i];
+    orc_linear(w->w_down, L, d, xv, z);
+    orc_route_token(d, R, k, x_t, w->w_router, w->expert_bias, ids, probs, NULL, NULL);
+    for (int32_t e = 0; e < R; ++e)
+      orc_situ(L, F, dm->beta1, dm->beta2, w->w_g + (int64_t)e * F * L,
+               w->w_u + (int64_t)e * F * L, w->w_o + (int64_t)e * L * F, z,
+               all_out + (int64_t)e * L, NULL);
+    for (int32_t slot = 0; slot < k; ++slot)
+      for (int32_t j = 0; j < L; ++j) u[j] += probs[slot] * all_out[(int64_t)ids[slot] * L + j];
+    for (int32_t j = 0; j < S; ++j) {
+      orc_situ(d, G, dm->beta1, dm->beta2, w->ws_g + (int64_t)j * G * d,
+               w->ws_u + (int64_t)j * G * d, w->ws_o + (int64_t)j * d * G, xv, tmp, NULL);
+      for (int32_t i = 0; i < d; ++i) sh[i] += tmp[i];
+    }
+    orc_rmsnorm(L, u, w->rms_weight, dm->rms_eps, uhat);
+    orc_linear(w->w_up, d, L, uhat, tmp);
+    for (int32_t i = 0; i < d; ++i) y[t * d + i] = sh[i] + tmp[i];
+    if (u_out) memcpy(u_out + t * L, u, sizeof(double) * (size_t)L);
+    free(xv);
+    free(z);
+    free(all_out);
+    free(u);
+    free(uhat);
+    free(sh);
+    free(tmp);
+    free(ids);
+    free(probs);
+  }
+}
+
+/* Standalone RMSNorm over N rows of width n (for pins). */
+void orc_rmsnorm_rows(int64_t N, int32_t n, const double* u, const float* w, double eps,
+                      double* out) {
+  for (int64_t t = 0; t < N; ++t) orc_rmsnorm(n, u + t * n, w, eps, out + t * n);
+}
