@@ -1,0 +1,359 @@
+#!/usr/bin/env python
+"""LatentMoE layer forward throughput on B200 (tokens/s) and roofline fraction.
+
+One step = one latent_moe_forward over the workload's N tokens (every kernel of
+the layer).  Default workload: the 0.5b-preset layer (halfb_uniform: N=4096,
+d=768, l=384, 16 routed experts top-2, 2 shared, F=768, G=1536, bf16).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the CPU oracle, timed on host cores)
+
+Multi-GPU (torchrun): token-sharded replicas, no data-path collective; each
+rank runs its own N tokens, the time is the max over ranks ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "LatentMoE layer fwd tokens/s on 1 B200; % of bf16 roofline (FLOPs vs HBM)"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# Algorithmic work of each kernel (per launch, full workload): FLOPs or bytes.
+def kernel_work(wl: synth.Workload, tag: str):
+    N, d, L, R, k, F, S, G = (wl.n_tokens, wl.d, wl.latent, wl.n_routed, wl.top_k, wl.ff_routed,
+                              wl.n_shared, wl.ff_shared)
+    es = 2 if wl.dtype == "bf16" else 4
+    P = N * k
+    if tag == "xpass":      # z = W_down x, router logits, shared gate/up + SiTU
+        return "tensor", 2.0 * N * d * (L + R + 2 * S * G)
+    if tag == "expert_gemm1":
+        return "tensor", 2.0 * P * L * 2 * F
+    if tag == "expert_gemm2":
+        return "tensor", 2.0 * P * F * L
+    if tag == "final":
+        return "tensor", 2.0 * N * (S * G + L) * d
+    if tag == "combine":    # read k expert rows + ids/probs, write uhat
+        return "hbm", float(P * L * es + P * 8 + N * L * es)
+    if tag == "dispatch":
+        return "hbm", float(P * 4 + P * 8)
+    if tag == "route":
+        return "hbm", float(N * d * es + R * d * es + P * 8)
+    raise KeyError(tag)
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+               "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+               "display_clock_setting": 0x100}
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_baseline(wl: synth.Workload, seed: int, budget_s: float = 12.0) -> dict:
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    workload's tokens: first a small probe, then a sample sized to ~budget_s."""
+    import oracle
+    inp = synth.make_inputs(wl.with_tokens(0), seed, with_x=False)
+    w = {k: synth.to_f32(inp[k]) for k in synth.WEIGHT_NAMES}
+    cores = os.cpu_count() or 1
+
+    def run(n):
+        x = synth.to_f32(synth.make_x_rows(wl, seed, np.arange(n)))
+        dims = oracle.Dims(n, wl.d, wl.latent, wl.n_routed, wl.top_k, wl.n_shared, wl.ff_routed,
+                           wl.ff_shared, wl.beta1, wl.beta2, wl.rms_eps)
+        t0 = time.perf_counter()
+        oracle.forward(dims, w, x)
+        return time.perf_counter() - t0
+
+    probe_n = max(1, min(wl.n_tokens, cores * 2))
+    t_probe = run(probe_n)
+    n = int(min(wl.n_tokens, max(probe_n, probe_n * budget_s / max(t_probe, 1e-6))))
+    t = run(n)
+    return {"value": n / t, "unit": "tokens/s", "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
+            "kind": "oracle",
+            "sample": f"{n} of {wl.n_tokens} tokens of {wl.name}, fp64 C oracle, OpenMP over tokens, "
+                      f"{t:.1f} s"}
+
+
+def run_reference(args, wl):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import oracle
+    inp = synth.make_inputs(wl.with_tokens(0), args.seed, with_x=False)
+    w = {k: synth.to_f32(inp[k]) for k in synth.WEIGHT_NAMES}
+    cores = os.cpu_count() or 1
+    # each step: a bounded sample of the workload's tokens
+    probe = max(1, min(wl.n_tokens, cores))
+    dims = lambda n: oracle.Dims(n, wl.d, wl.latent, wl.n_routed, wl.top_k, wl.n_shared,
+                                 wl.ff_routed, wl.ff_shared, wl.beta1, wl.beta2, wl.rms_eps)
+    xp = synth.to_f32(synth.make_x_rows(wl, args.seed, np.arange(probe)))
+    t0 = time.perf_counter()
+    oracle.forward(dims(probe), w, xp)
+    per_tok = (time.perf_counter() - t0) / probe
+    total_budget = 60.0
+    n_step = int(max(1, min(wl.n_tokens, total_budget / (args.steps + args.warmup) / per_tok)))
+    x = synth.to_f32(synth.make_x_rows(wl, args.seed, np.arange(n_step)))
+    for _ in range(args.warmup):
+        oracle.forward(dims(n_step), w, x)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.forward(dims(n_step), w, x)
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = n_step / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens_per_step": n_step, "n_tokens": wl.n_tokens},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{n_step} of {wl.n_tokens} tokens per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="halfb_uniform", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--profile-kernel", default=None,
+                    help="kernel tag for the roofline line (default: the largest GEMM)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    import torch
+    import torch.distributed as dist
+
+    import sigmoid_top_routing_latentmoe_b200 as lm
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    # inputs: weights shared by all ranks (seed), x drawn per rank (its own tokens)
+    inp = synth.make_inputs(wl, args.seed, with_x=False)
+    x_np = synth.make_x_rows(wl, args.seed, np.arange(wl.n_tokens) + rank * wl.n_tokens)
+
+    def todev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    w = {k: todev(inp[k]) for k in synth.WEIGHT_NAMES}
+    x = todev(x_np)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    dims = lm.make_dims(wl.n_tokens, wl.d, wl.latent, wl.n_routed, wl.top_k, wl.n_shared,
+                        wl.ff_routed, wl.ff_shared, wl.beta1, wl.beta2, wl.rms_eps, dt)
+    ws = lm.alloc_workspace(dims, device=dev)
+    y = torch.empty(wl.n_tokens, wl.d, dtype=dt, device=dev)
+    wstruct = lm.weights_struct(w)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        lm.latent_moe_forward(dims, wstruct, x, y, ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if lm.get_device_status(ws) != lm.OK:
+        raise SystemExit("device status not OK after warm-up")
+
+    prof_tag = args.profile_kernel or "xpass"
+    bound, work = kernel_work(wl, prof_tag)
+    lm.profile_read()                       # drop anything recorded so far
+    lm.profile_enable(prof_tag)
+    clocks = ClockSampler(local)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    lm.launch_count(reset=True)
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()                        # L2 flushed between timed steps (outside the events)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    launches = lm.launch_count()
+    lm.profile_enable(None)
+    k_ms, k_n = lm.profile_read()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * wl.n_tokens / (ms_per_step / 1e3)
+    if lm.get_device_status(ws) != lm.OK:
+        raise SystemExit("device status not OK after the timed region")
+
+    # end to end through the host entry point: pinned x in, y out, copies timed
+    ws_h = lm.alloc_workspace(dims, device=dev, host=True)
+    x_h = x.cpu().pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    for _ in range(3):
+        lm.latent_moe_forward_host(dims, wstruct, x_h, y_h, ws_h)
+    e2e_steps = max(3, min(args.steps, 50))
+    if world > 1:
+        dist.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        lm.latent_moe_forward_host(dims, wstruct, x_h, y_h, ws_h)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    io_bytes = wl.n_tokens * wl.d * (2 if wl.dtype == "bf16" else 4)
+
+    peaks = _peaks()
+    if k_n > 0:
+        k_avg_s = k_ms / k_n / 1e3
+        if bound == "tensor":
+            achieved = work / k_avg_s / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            unit = "TFLOP/s"
+        else:
+            achieved = work / k_avg_s / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        roof = {"kernel": prof_tag, "bound": bound, "achieved": achieved, "peak": peak,
+                "unit": unit, "frac": achieved / peak, "traffic": None,
+                "launch_us": k_avg_s * 1e6, "launches": k_n,
+                "peak_source": peaks["source"] + (" sustained" if bound == "tensor" else "")}
+    else:
+        roof = None
+    roof_s = max(wl.flops() / (peaks["bf16_tflops"] * 1e12), wl.compulsory_bytes() / (peaks["hbm_gbs"] * 1e9))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "n_tokens": wl.n_tokens, "d": wl.d, "latent": wl.latent,
+                   "n_routed": wl.n_routed, "top_k": wl.top_k, "ff_routed": wl.ff_routed,
+                   "n_shared": wl.n_shared, "ff_shared": wl.ff_shared,
+                   "parallelism": f"replicas{world}", "l2": "flushed (256 MiB write) between steps"},
+        "layer_roofline": {"flops": wl.flops(), "compulsory_bytes": wl.compulsory_bytes(),
+                           "roof_us": roof_s * 1e6, "frac": roof_s / (ms_per_step / 1e3),
+                           "peak_source": peaks["source"] + " burst"},
+        "roofline": roof,
+        "clocks": clk,
+        "e2e": {"value": world * wl.n_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
+        "gpu_launches": launches,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.seed)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,206 @@
+/*
+ * latent_moe.h -- C ABI of the B200 (sm_100a) LatentMoE forward library.
+ *
+ * The library computes the forward pass of the LatentMoE feed-forward layer of
+ * the K3 notes (sec-07, "SiTU-GLU 与 Stable LatentMoE", compute flow in five
+ * steps; kda/layers/latent_moe.py in the K3 compare view 584f7e9..main):
+ *
+ *   z = W_down x                                   (latent compression, l = d/2)
+ *   s = sigmoid(W_r x), T = TopK(s + b, k),
+ *   p_i = s_i / max(sum_{j in T} s_j, 1e-9)        (K3 eq.13; b selects only)
+ *   u = sum_{i in T} p_i E_i(z)                    (routed SiTU-GLU experts in l)
+ *   s_sh = sum_j E^sh_j(x)                         (shared SiTU-GLU experts in d)
+ *   y = s_sh + W_up RMSNorm(u)
+ *   E(v) = W_o [beta1 tanh(W_g v / beta1) sigmoid(W_g v) * beta2 tanh(W_u v / beta2)]
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller, except
+ *     where a function says "host".  The library never allocates, frees or
+ *     keeps device memory; scratch lives in a caller-provided workspace.
+ *   - Row-major, contiguous, 16-byte-aligned buffers.  Weights follow
+ *     nn.Linear: [out, in], the reduction dimension contiguous.
+ *   - Activations and weights have the dtype in lmoe_dims.dtype (bf16 or
+ *     fp32); accumulation is always fp32.  expert_bias, rms_weight and probs
+ *     are always fp32; ids and permutation arrays are int32.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) unless stated.  Argument errors are returned before any
+ *     launch; launch failures return LMOE_ECUDA.  Anomalies found on the device
+ *     (a capped wait that ran out, a failed consistency check) are recorded in
+ *     the workspace status word, read by lmoe_get_device_status.
+ *   - Calls that share one workspace must not overlap on the device.
+ *   - Requires an sm_100a device (B200).  Otherwise LMOE_EUNSUPPORTED.
+ */
+#ifndef LATENT_MOE_H
+#define LATENT_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LMOE_API __attribute__((visibility("default")))
+#else
+#define LMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LMOE_OK = 0,
+  LMOE_EINVAL = 1,       /* bad dims, null or misaligned pointer              */
+  LMOE_EUNSUPPORTED = 2, /* not an sm_100a device, or a size out of range     */
+  LMOE_EWORKSPACE = 3,   /* workspace too small                               */
+  LMOE_ECUDA = 4,        /* a CUDA runtime/driver call or a launch failed     */
+  LMOE_EDEVICE = 5,      /* the device status word holds a failed check       */
+  LMOE_ETIMEOUT = 6      /* a capped device-side wait ran out                 */
+} lmoe_status;
+
+typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
+
+typedef void* lmoe_stream; /* cudaStream_t */
+
+/* Layer sizes (the pages' LatentMoE(hidden_size, latent_size, n_routed, top_k,
+ * n_shared, d_ff, beta1, beta2) with B*T flattened to n_tokens and separate
+ * routed/shared hidden widths).  Limits: 1 <= top_k <= n_routed <= 4096;
+ * d, latent, ff_routed, ff_shared multiples of 64 (bf16) or 8 (fp32);
+ * 0 <= n_shared <= 7; n_tokens * top_k < 2^31. */
+typedef struct {
+  int64_t n_tokens; /* N                                    */
+  int32_t d;        /* model width                          */
+  int32_t latent;   /* l (d/2 in the pages)                 */
+  int32_t n_routed; /* R                                    */
+  int32_t top_k;    /* k                                    */
+  int32_t n_shared; /* S                                    */
+  int32_t ff_routed;/* F, routed expert hidden width        */
+  int32_t ff_shared;/* G, shared expert hidden width        */
+  float beta1;      /* SiTU gate cap (pages: 4)             */
+  float beta2;      /* SiTU up cap (pages: 25)              */
+  float rms_eps;    /* RMSNorm epsilon (1e-6)               */
+  int32_t dtype;    /* lmoe_dtype                           */
+} lmoe_dims;
+
+/* Layer weights, device pointers in nn.Linear layout. */
+typedef struct {
+  const void* w_down;       /* [l, d]      W_down                               */
+  const void* w_router;     /* [R, d]      W_r                                  */
+  const void* w_up;         /* [d, l]      W_up                                 */
+  const float* rms_weight;  /* [l] fp32    RMSNorm weight                       */
+  const float* expert_bias; /* [R] fp32    selection bias b; NULL means b = 0   */
+  const void* w_g;          /* [R, F, l]   routed gate projections              */
+  const void* w_u;          /* [R, F, l]   routed up projections                */
+  const void* w_o;          /* [R, l, F]   routed output projections            */
+  const void* ws_g;         /* [S, G, d]   shared gate projections (S > 0)      */
+  const void* ws_u;         /* [S, G, d]   shared up projections                */
+  const void* ws_o;         /* [S, d, G]   shared output projections            */
+} lmoe_weights;
+
+/* Bytes of device workspace that every entry point below accepts for these
+ * dims (one size serves all of them).  0 on invalid dims. */
+LMOE_API size_t lmoe_workspace_size(const lmoe_dims* dims);
+
+/* Router (sec-07 compute flow step 2, K3 eq.13; latent_moe.py LatentMoE._route):
+ * l = W_r x (fp32 accumulation), s = sigmoid(l), T = TopK(s + b, k) with the
+ * slots in descending s + b (a tie goes to the lower expert index),
+ * p_i = s_i / max(sum_T s, 1e-9).
+ *   x        [N, d]      input rows
+ *   w_router [R, d]
+ *   expert_bias [R] fp32 or NULL
+ *   ids      [N, k] int32 out;  probs [N, k] fp32 out.
+ * Workspace: lmoe_workspace_size(dims) bytes. */
+LMOE_API lmoe_status moe_route(const lmoe_dims* dims, const void* x, const void* w_router,
+                      const float* expert_bias, int32_t* ids, float* probs, void* ws,
+                      size_t ws_bytes, lmoe_stream stream);
+
+/* Pair permutation (latent_moe.py LatentMoE._routed_u; sec-07 sparse dispatch,
+ * step 1): the N*k (token, expert) pairs, flattened token-major, stably sorted
+ * by expert id.  Bit-exact and deterministic.
+ *   ids        [N, k] int32 in, each row k distinct ids in [0, R)
+ *   counts     [R]    int32 out: pairs per expert (bincount)
+ *   offsets    [R+1]  int32 out: exclusive prefix sum, offsets[R] = N*k
+ *   perm_token [N*k]  int32 out: token of each sorted pair (expert-major,
+ *                     tokens ascending inside an expert)
+ *   inv_pair   [N, k] int32 out: sorted position of pair (t, slot)
+ * Out-of-range ids set LMOE_EDEVICE in the status word (the pair is dropped). */
+LMOE_API lmoe_status moe_dispatch(const lmoe_dims* dims, const int32_t* ids, int32_t* counts,
+                         int32_t* offsets, int32_t* perm_token, int32_t* inv_pair, void* ws,
+                         size_t ws_bytes, lmoe_stream stream);
+
+/* Routed experts on the sorted pairs (sec-07 compute flow step 3 and the
+ * sparse-dispatch subsection; latent_moe.py _routed_u, without padding to
+ * the capacity C): for each expert e and sorted row r in
+ * [offsets[e], offsets[e+1]):
+ *   expert_out[r] = W_o,e [beta1 tanh(a/beta1) sigmoid(a) * beta2 tanh(c/beta2)],
+ *   a = W_g,e z[perm_token[r]],  c = W_u,e z[perm_token[r]].
+ *   z          [N, l]
+ *   perm_token [N*k], offsets [R+1]   from moe_dispatch
+ *   w_g, w_u   [R, F, l];  w_o [R, l, F]
+ *   expert_out [N*k, l]   out, in sorted-pair order (not yet weighted by p). */
+LMOE_API lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const int32_t* perm_token,
+                           const int32_t* offsets, const void* w_g, const void* w_u,
+                           const void* w_o, void* expert_out, void* ws, size_t ws_bytes,
+                           lmoe_stream stream);
+
+/* Weighted combine + RMSNorm (latent_moe.py index_add and self.norm; sec-07
+ * step 3 sum and step 5 RMSNorm): for each token t, in slot order,
+ *   u_t = sum_i probs[t, i] * expert_out[inv_pair[t, i]]   (fp32, no atomics)
+ *   u_normed_t = u_t / sqrt(mean(u_t^2) + eps) * rms_weight
+ *   u_normed [N, l] out. */
+LMOE_API lmoe_status moe_combine(const lmoe_dims* dims, const void* expert_out, const int32_t* inv_pair,
+                        const float* probs, const float* rms_weight, void* u_normed,
+                        lmoe_stream stream);
+
+/* The whole layer: y [N, d] = s_sh + W_up RMSNorm(u).  Optional outputs (NULL
+ * to skip): ids_out [N, k], probs_out [N, k], counts_out [R].  All work is on
+ * `stream`; no host synchronisation. */
+LMOE_API lmoe_status latent_moe_forward(const lmoe_dims* dims, const lmoe_weights* weights, const void* x,
+                               void* y, int32_t* ids_out, float* probs_out, int32_t* counts_out,
+                               void* ws, size_t ws_bytes, lmoe_stream stream);
+
+/* The whole layer from HOST memory: copies x_host [N, d] (pinned or pageable)
+ * to the device, runs latent_moe_forward, copies y back to y_host [N, d] and
+ * waits for the stream.  Weights and workspace are device memory.  The
+ * workspace must be lmoe_workspace_size_host(dims) bytes (it also holds the
+ * device copies of x and y). */
+LMOE_API size_t lmoe_workspace_size_host(const lmoe_dims* dims);
+LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_weights* weights,
+                                    const void* x_host, void* y_host, void* ws, size_t ws_bytes,
+                                    lmoe_stream stream);
+
+/* Zeroes the workspace header (status word and scheduling counters).  Call
+ * once on a new workspace before its first use. */
+LMOE_API lmoe_status lmoe_workspace_init(void* ws, size_t ws_bytes, lmoe_stream stream);
+
+/* Waits for `stream`, then reads and clears the workspace status word.
+ * Returns LMOE_OK, LMOE_EDEVICE or LMOE_ETIMEOUT (or LMOE_ECUDA). */
+LMOE_API lmoe_status lmoe_get_device_status(void* ws, lmoe_stream stream);
+
+/* Launches one kernel that waits on a device flag nothing sets, with a cap of
+ * about `cap_ms` milliseconds, then records LMOE_ETIMEOUT in the status word and
+ * returns.  Exists to test the capped-wait path; the GPU stays usable. */
+LMOE_API lmoe_status lmoe_selftest_capped_wait(void* ws, size_t ws_bytes, int32_t cap_ms,
+                                      lmoe_stream stream);
+
+/* Human-readable name of a status code. */
+LMOE_API const char* lmoe_status_string(lmoe_status status);
+
+/* Last error message of this thread (empty string if none). */
+LMOE_API const char* lmoe_last_error(void);
+
+/* Brackets every launch of the kernel named `tag` (NULL or "" turns it off)
+ * with CUDA events on its stream.  Tags: "xpass", "route", "dispatch",
+ * "gather", "expert_gemm1", "expert_gemm2", "combine", "final". */
+LMOE_API lmoe_status lmoe_profile_enable(const char* tag);
+/* Waits for the recorded events; returns the summed device time (ms) and the
+ * number of bracketed launches since the last read, then clears them. */
+LMOE_API lmoe_status lmoe_profile_read(double* total_ms, int64_t* launches);
+
+/* Number of kernel launches the library issued on this thread since the last
+ * reset (instrumentation for benchmarks). */
+LMOE_API uint64_t lmoe_launch_count(int32_t reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LATENT_MOE_H */

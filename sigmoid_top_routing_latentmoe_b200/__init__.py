@@ -1,0 +1,200 @@
+"""Python binding of liblatent_moe.so, the B200 LatentMoE forward library.
+
+Argument marshalling only: every function here passes torch tensors' device
+pointers to the C ABI of the same name (include/latent_moe.h) and raises
+:class:`LmoeError` on a non-OK status.  All work runs in the library's CUDA
+kernels; there is no Python or CPU fallback.  If the shared library is
+missing, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblatent_moe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python sigmoid_top_routing_latentmoe_b200/build.py` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, EINVAL, EUNSUPPORTED, EWORKSPACE, ECUDA, EDEVICE, ETIMEOUT = range(7)
+F32, BF16 = 0, 1
+
+
+class LmoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = _lib.lmoe_status_string(status).decode()
+        msg = _lib.lmoe_last_error().decode()
+        super().__init__(f"{where}: {name}: {msg}")
+
+
+class Dims(ctypes.Structure):
+    """lmoe_dims."""
+    _fields_ = [("n_tokens", ctypes.c_int64), ("d", ctypes.c_int32), ("latent", ctypes.c_int32),
+                ("n_routed", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32), ("ff_routed", ctypes.c_int32),
+                ("ff_shared", ctypes.c_int32), ("beta1", ctypes.c_float),
+                ("beta2", ctypes.c_float), ("rms_eps", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+WEIGHT_NAMES = ("w_down", "w_router", "w_up", "rms_weight", "expert_bias",
+                "w_g", "w_u", "w_o", "ws_g", "ws_u", "ws_o")
+
+
+class Weights(ctypes.Structure):
+    """lmoe_weights."""
+    _fields_ = [(n, _P) for n in WEIGHT_NAMES]
+
+
+_S = ctypes.c_int
+_DP = ctypes.POINTER(Dims)
+_sigs = {
+    "lmoe_workspace_size": (ctypes.c_size_t, [_DP]),
+    "lmoe_workspace_size_host": (ctypes.c_size_t, [_DP]),
+    "moe_route": (_S, [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_dispatch": (_S, [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_expert_ffn": (_S, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_combine": (_S, [_DP, _P, _P, _P, _P, _P, _P]),
+    "latent_moe_forward": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, _P, _P, _P, _P,
+                                ctypes.c_size_t, _P]),
+    "latent_moe_forward_host": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, _P, ctypes.c_size_t,
+                                     _P]),
+    "lmoe_workspace_init": (_S, [_P, ctypes.c_size_t, _P]),
+    "lmoe_get_device_status": (_S, [_P, _P]),
+    "lmoe_selftest_capped_wait": (_S, [_P, ctypes.c_size_t, ctypes.c_int32, _P]),
+    "lmoe_status_string": (ctypes.c_char_p, [_S]),
+    "lmoe_last_error": (ctypes.c_char_p, []),
+    "lmoe_launch_count": (ctypes.c_uint64, [ctypes.c_int32]),
+    "lmoe_profile_enable": (_S, [ctypes.c_char_p]),
+    "lmoe_profile_read": (_S, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
+}
+for _name, (_res, _args) in _sigs.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def make_dims(n_tokens, d, latent, n_routed, top_k, n_shared, ff_routed, ff_shared,
+              beta1=4.0, beta2=25.0, rms_eps=1e-6, dtype=torch.bfloat16) -> Dims:
+    code = {torch.bfloat16: BF16, torch.float32: F32}[dtype]
+    return Dims(n_tokens, d, latent, n_routed, top_k, n_shared, ff_routed, ff_shared,
+                beta1, beta2, rms_eps, code)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return _P(torch.cuda.current_stream().cuda_stream)
+    return _P(stream.cuda_stream if hasattr(stream, "cuda_stream") else stream)
+
+
+def _check(status, where):
+    if status != OK:
+        raise LmoeError(status, where)
+
+
+def workspace_size(dims: Dims, host: bool = False) -> int:
+    n = (_lib.lmoe_workspace_size_host if host else _lib.lmoe_workspace_size)(ctypes.byref(dims))
+    if n == 0:
+        raise LmoeError(EINVAL, "workspace_size")
+    return n
+
+
+def alloc_workspace(dims: Dims, device="cuda", host: bool = False, stream=None) -> torch.Tensor:
+    """A byte tensor of the required size (256-byte aligned), header zeroed."""
+    n = workspace_size(dims, host)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + n]
+    workspace_init(ws, stream)
+    return ws
+
+
+def workspace_init(ws: torch.Tensor, stream=None):
+    _check(_lib.lmoe_workspace_init(_ptr(ws), ws.numel(), _stream(stream)), "lmoe_workspace_init")
+
+
+def weights_struct(w: dict) -> Weights:
+    return Weights(*[_ptr(w.get(n)) for n in WEIGHT_NAMES])
+
+
+def moe_route(dims, x, w_router, expert_bias, ids, probs, ws, stream=None):
+    _check(_lib.moe_route(ctypes.byref(dims), _ptr(x), _ptr(w_router), _ptr(expert_bias),
+                          _ptr(ids), _ptr(probs), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_route")
+
+
+def moe_dispatch(dims, ids, counts, offsets, perm_token, inv_pair, ws, stream=None):
+    _check(_lib.moe_dispatch(ctypes.byref(dims), _ptr(ids), _ptr(counts), _ptr(offsets),
+                             _ptr(perm_token), _ptr(inv_pair), _ptr(ws), ws.numel(),
+                             _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_ffn(dims, z, perm_token, offsets, w_g, w_u, w_o, expert_out, ws, stream=None):
+    _check(_lib.moe_expert_ffn(ctypes.byref(dims), _ptr(z), _ptr(perm_token), _ptr(offsets),
+                               _ptr(w_g), _ptr(w_u), _ptr(w_o), _ptr(expert_out), _ptr(ws),
+                               ws.numel(), _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(dims, expert_out, inv_pair, probs, rms_weight, u_normed, stream=None):
+    _check(_lib.moe_combine(ctypes.byref(dims), _ptr(expert_out), _ptr(inv_pair), _ptr(probs),
+                            _ptr(rms_weight), _ptr(u_normed), _stream(stream)), "moe_combine")
+
+
+def latent_moe_forward(dims, weights, x, y, ws, ids_out=None, probs_out=None, counts_out=None,
+                       stream=None):
+    ws_struct = weights if isinstance(weights, Weights) else weights_struct(weights)
+    _check(_lib.latent_moe_forward(ctypes.byref(dims), ctypes.byref(ws_struct), _ptr(x), _ptr(y),
+                                   _ptr(ids_out), _ptr(probs_out), _ptr(counts_out), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "latent_moe_forward")
+
+
+def latent_moe_forward_host(dims, weights, x_host, y_host, ws, stream=None):
+    ws_struct = weights if isinstance(weights, Weights) else weights_struct(weights)
+    _check(_lib.latent_moe_forward_host(ctypes.byref(dims), ctypes.byref(ws_struct),
+                                        _ptr(x_host), _ptr(y_host), _ptr(ws), ws.numel(),
+                                        _stream(stream)), "latent_moe_forward_host")
+
+
+def get_device_status(ws, stream=None) -> int:
+    """Waits for the stream; returns (and clears) the workspace status code."""
+    return _lib.lmoe_get_device_status(_ptr(ws), _stream(stream))
+
+
+def selftest_capped_wait(ws, cap_ms: int, stream=None):
+    _check(_lib.lmoe_selftest_capped_wait(_ptr(ws), ws.numel(), cap_ms, _stream(stream)),
+           "lmoe_selftest_capped_wait")
+
+
+def launch_count(reset: bool = False) -> int:
+    return _lib.lmoe_launch_count(1 if reset else 0)
+
+
+def profile_enable(tag):
+    """Brackets every launch of kernel ``tag`` with CUDA events (None: off)."""
+    _check(_lib.lmoe_profile_enable(None if tag is None else tag.encode()), "lmoe_profile_enable")
+
+
+def profile_read():
+    """(summed device ms, launches) of the bracketed kernel since the last read."""
+    ms, n = ctypes.c_double(), ctypes.c_int64()
+    _check(_lib.lmoe_profile_read(ctypes.byref(ms), ctypes.byref(n)), "lmoe_profile_read")
+    return ms.value, n.value
+
+
+def status_string(code: int) -> str:
+    return _lib.lmoe_status_string(code).decode()

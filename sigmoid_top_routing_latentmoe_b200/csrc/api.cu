@@ -1,0 +1,574 @@
+// C ABI of the LatentMoE forward library: argument checks, workspace layout
+// and the launch sequence of each entry point.  See include/latent_moe.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lmoe {
+
+static thread_local std::string g_last_error;
+static thread_local uint64_t g_launches = 0;
+
+void count_launch(int n) { g_launches += (uint64_t)n; }
+
+// --------------------------------------------------------------- profiling
+// Optional CUDA-event brackets around the launches of one named kernel, on the
+// stream they are launched on.  Off unless lmoe_profile_enable names a tag.
+struct ProfRec {
+  cudaEvent_t a, b;
+};
+static thread_local std::string g_prof_tag;
+static thread_local std::vector<ProfRec> g_prof;
+
+struct ProfScope {
+  bool on = false;
+  cudaStream_t st;
+  ProfRec r{};
+  ProfScope(const char* tag, cudaStream_t s) : st(s) {
+    if (g_prof_tag.empty() || g_prof_tag != tag) return;
+    if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) return;
+    on = cudaEventRecord(r.a, st) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(r.b, st);
+    g_prof.push_back(r);
+  }
+};
+
+static lmoe_status fail(lmoe_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+static lmoe_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(LMOE_ECUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define LMOE_CUDA(call, where)                      \
+  do {                                              \
+    cudaError_t _e = (call);                        \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+// ------------------------------------------------------------- device check
+static lmoe_status check_device() {
+  static std::mutex mu;
+  static int verdict[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  LMOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LMOE_EUNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (verdict[dev] == 0) {
+    int major = 0, minor = 0;
+    LMOE_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "attr");
+    LMOE_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "attr");
+    verdict[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  if (verdict[dev] != 1) return fail(LMOE_EUNSUPPORTED, "device %d is not sm_100 (B200)", dev);
+  return LMOE_OK;
+}
+
+// ------------------------------------------------------------- validation
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static lmoe_status check_dims(const lmoe_dims* d) {
+  if (d == nullptr) return fail(LMOE_EINVAL, "dims is NULL");
+  if (d->dtype != LMOE_F32 && d->dtype != LMOE_BF16) return fail(LMOE_EINVAL, "dtype %d", d->dtype);
+  if (d->n_tokens < 0) return fail(LMOE_EINVAL, "n_tokens < 0");
+  if (d->d <= 0 || d->latent <= 0 || d->ff_routed <= 0)
+    return fail(LMOE_EINVAL, "d, latent and ff_routed must be positive");
+  if (d->n_routed < 1 || d->n_routed > 4096) return fail(LMOE_EUNSUPPORTED, "n_routed out of [1, 4096]");
+  if (d->top_k < 1 || d->top_k > d->n_routed) return fail(LMOE_EINVAL, "top_k out of [1, n_routed]");
+  if (d->n_shared < 0 || d->n_shared > kMaxSeg - 1) return fail(LMOE_EUNSUPPORTED, "n_shared out of [0, 7]");
+  if (d->n_shared > 0 && d->ff_shared <= 0) return fail(LMOE_EINVAL, "ff_shared must be positive");
+  if (d->d % 8 || d->latent % 8 || d->ff_routed % 8 || (d->n_shared > 0 && d->ff_shared % 8))
+    return fail(LMOE_EINVAL, "d, latent, ff_routed and ff_shared must be multiples of 8");
+  if (d->latent > 4096) return fail(LMOE_EUNSUPPORTED, "latent > 4096");
+  if (d->d > 65536) return fail(LMOE_EUNSUPPORTED, "d > 65536");
+  if (d->n_tokens * (int64_t)d->top_k >= ((int64_t)1 << 31) - kTileM * 8)
+    return fail(LMOE_EUNSUPPORTED, "n_tokens * top_k too large");
+  if (!(d->beta1 > 0.0f) || !(d->beta2 > 0.0f) || !(d->rms_eps >= 0.0f))
+    return fail(LMOE_EINVAL, "beta1, beta2 must be > 0 and rms_eps >= 0");
+  return LMOE_OK;
+}
+
+#define LMOE_PTR(p, name)                                                          \
+  do {                                                                             \
+    if ((p) == nullptr) return fail(LMOE_EINVAL, "%s is NULL", name);              \
+    if (!aligned16(p)) return fail(LMOE_EINVAL, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+// ------------------------------------------------------------ workspace
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct Layout {
+  size_t header, z, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, zp, h, eo,
+      hsh, uhat, x, y, total;
+  int64_t logits_ld;
+  int max_tiles;
+};
+
+static Layout layout(const lmoe_dims* d, bool host_copies) {
+  Layout L{};
+  const int64_t N = d->n_tokens, P = N * d->top_k;
+  const size_t es = d->dtype == LMOE_BF16 ? 2 : 4;
+  const int R = d->n_routed;
+  L.logits_ld = (R + 15) / 16 * 16;
+  L.max_tiles = (int)(P / kTileM + R + 1);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t at = off; off += align256(bytes); return at; };
+  L.header = take(sizeof(WsHeader));
+  L.z = take((size_t)N * d->latent * es);
+  L.logits = take((size_t)N * L.logits_ld * 4);
+  L.ids = take((size_t)P * 4);
+  L.probs = take((size_t)P * 4);
+  L.counts = take((size_t)R * 4);
+  L.offsets = take((size_t)(R + 1) * 4);
+  L.perm = take((size_t)P * 4);
+  L.inv = take((size_t)P * 4);
+  L.block_counts = take((size_t)dispatch_blocks(P) * R * 4);
+  L.tiles = take((size_t)L.max_tiles * sizeof(int4));
+  L.zp = take((size_t)P * d->latent * es);
+  L.h = take((size_t)P * d->ff_routed * es);
+  L.eo = take((size_t)P * d->latent * es);
+  L.hsh = take((size_t)N * d->n_shared * (size_t)d->ff_shared * es);
+  L.uhat = take((size_t)N * d->latent * es);
+  if (host_copies) {
+    L.x = take((size_t)N * d->d * es);
+    L.y = take((size_t)N * d->d * es);
+  }
+  L.total = off;
+  return L;
+}
+
+template <typename P>
+static P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<char*>(ws) + off);
+}
+
+static lmoe_status check_ws(const lmoe_dims* d, void* ws, size_t ws_bytes, bool host) {
+  LMOE_PTR(ws, "ws");
+  if (((uintptr_t)ws & 255u) != 0) return fail(LMOE_EINVAL, "ws must be 256-byte aligned");
+  size_t need = layout(d, host).total;
+  if (ws_bytes < need)
+    return fail(LMOE_EWORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+  return LMOE_OK;
+}
+
+#define LMOE_TRY(expr)                  \
+  do {                                  \
+    lmoe_status _s = (expr);            \
+    if (_s != LMOE_OK) return _s;       \
+  } while (0)
+
+// ------------------------------------------------------------- launchers
+template <typename T>
+static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r, const float* bias,
+                             int32_t* ids, float* probs, void* ws, cudaStream_t st) {
+  const Layout L = layout(d, false);
+  const int64_t N = d->n_tokens;
+  if (N == 0) return LMOE_OK;
+  if (d->n_routed <= 32) {
+    ProfScope ps("route", st);
+    LMOE_CUDA(launch_route_gemv<T>((const T*)x, (const T*)w_r, bias, N, d->d, d->n_routed,
+                                   d->top_k, ids, probs, st),
+              "route_gemv");
+    return LMOE_OK;
+  }
+  float* logits = at<float>(ws, L.logits);
+  ProfScope ps("route", st);
+  SimtGemm g{};
+  g.A[0] = x; g.lda[0] = d->d; g.B[0] = w_r; g.ldb[0] = d->d; g.K[0] = d->d; g.nseg = 1;
+  g.C = logits; g.ldc = L.logits_ld; g.M = (int)N; g.N = d->n_routed; g.out_f32 = 1;
+  g.mode = kStore;
+  LMOE_CUDA(launch_simt_gemm<T>(g, st), "router logits");
+  LMOE_CUDA(launch_route_topk(logits, L.logits_ld, bias, N, d->n_routed, d->top_k, ids, probs, st),
+            "route_topk");
+  return LMOE_OK;
+}
+
+static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t* counts,
+                                int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
+                                cudaStream_t st) {
+  const Layout L = layout(d, false);
+  DispatchScratch s;
+  s.block_counts = at<int32_t>(ws, L.block_counts);
+  s.status = &at<WsHeader>(ws, L.header)->status;
+  s.n_mtiles = &at<WsHeader>(ws, L.header)->n_mtiles;
+  s.tiles = at<int4>(ws, L.tiles);
+  ProfScope ps("dispatch", st);
+  LMOE_CUDA(launch_dispatch(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm, inv, s,
+                            st),
+            "dispatch");
+  return LMOE_OK;
+}
+
+// Routed experts on sorted pairs; the tile list must already be in the workspace.
+template <typename T>
+static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32_t* perm,
+                                  const void* w_g, const void* w_u, const void* w_o, void* eo,
+                                  void* ws, cudaStream_t st) {
+  const Layout L = layout(d, false);
+  const int64_t P = d->n_tokens * d->top_k;
+  if (P == 0) return LMOE_OK;
+  const int Lt = d->latent, F = d->ff_routed;
+  T* zp = at<T>(ws, L.zp);
+  T* h = at<T>(ws, L.h);
+  const int4* tiles = at<int4>(ws, L.tiles);
+  const int32_t* n_tiles = &at<WsHeader>(ws, L.header)->n_mtiles;
+  {
+    ProfScope ps("gather", st);
+    LMOE_CUDA(launch_gather_rows<T>((const T*)z, perm, P, Lt, zp, st), "gather");
+  }
+  SimtGemm g1{};
+  g1.A[0] = zp; g1.lda[0] = Lt; g1.B[0] = w_g; g1.ldb[0] = Lt; g1.K[0] = Lt; g1.nseg = 1;
+  g1.B_up = w_u; g1.b_expert_stride = (int64_t)F * Lt;
+  g1.C = h; g1.ldc = F; g1.N = F; g1.tiles = tiles; g1.n_tiles = n_tiles;
+  g1.max_tiles = L.max_tiles; g1.beta1 = d->beta1; g1.beta2 = d->beta2; g1.mode = kSitu;
+  {
+    ProfScope ps("expert_gemm1", st);
+    LMOE_CUDA(launch_simt_gemm<T>(g1, st), "routed gemm1");
+  }
+  SimtGemm g2{};
+  g2.A[0] = h; g2.lda[0] = F; g2.B[0] = w_o; g2.ldb[0] = F; g2.K[0] = F; g2.nseg = 1;
+  g2.b_expert_stride = (int64_t)Lt * F;
+  g2.C = eo; g2.ldc = Lt; g2.N = Lt; g2.tiles = tiles; g2.n_tiles = n_tiles;
+  g2.max_tiles = L.max_tiles; g2.mode = kStore;
+  {
+    ProfScope ps("expert_gemm2", st);
+    LMOE_CUDA(launch_simt_gemm<T>(g2, st), "routed gemm2");
+  }
+  return LMOE_OK;
+}
+
+template <typename T>
+static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const void* x, void* y,
+                               int32_t* ids_out, float* probs_out, int32_t* counts_out, void* ws,
+                               cudaStream_t st) {
+  const Layout L = layout(d, false);
+  const int64_t N = d->n_tokens;
+  const int Lt = d->latent, S = d->n_shared, G = d->ff_shared, D = d->d;
+  int32_t* ids = ids_out ? ids_out : at<int32_t>(ws, L.ids);
+  float* probs = probs_out ? probs_out : at<float>(ws, L.probs);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  T* z = at<T>(ws, L.z);
+  T* hsh = at<T>(ws, L.hsh);
+  T* eo = at<T>(ws, L.eo);
+  T* uhat = at<T>(ws, L.uhat);
+  if (N == 0) {
+    // still produce zero counts
+    LMOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * d->n_routed, st), "memset");
+    return LMOE_OK;
+  }
+  // step 1: z = W_down x
+  {
+    SimtGemm g{};
+    g.A[0] = x; g.lda[0] = D; g.B[0] = w->w_down; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
+    g.C = z; g.ldc = Lt; g.M = (int)N; g.N = Lt; g.mode = kStore;
+    ProfScope ps("xpass", st);
+    LMOE_CUDA(launch_simt_gemm<T>(g, st), "down");
+  }
+  // step 4 (independent of routing): h_sh = SiTU hidden of the shared experts
+  if (S > 0) {
+    SimtGemm g{};
+    g.A[0] = x; g.lda[0] = D; g.B[0] = w->ws_g; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
+    g.B_up = w->ws_u; g.C = hsh; g.ldc = (int64_t)S * G; g.M = (int)N; g.N = S * G;
+    g.beta1 = d->beta1; g.beta2 = d->beta2; g.mode = kSitu;
+    ProfScope ps("xpass", st);
+    LMOE_CUDA(launch_simt_gemm<T>(g, st), "shared gemm1");
+  }
+  // step 2: routing
+  LMOE_TRY(run_route<T>(d, x, w->w_router, w->expert_bias, ids, probs, ws, st));
+  // step 3: dispatch, routed experts, combine + RMSNorm
+  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st));
+  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st));
+  {
+    ProfScope ps("combine", st);
+    LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, d->top_k, Lt, d->rms_eps, uhat,
+                                st),
+              "combine");
+  }
+  // step 5: y = sum_j W_o,sh_j h_sh_j + W_up uhat
+  {
+    SimtGemm g{};
+    int s = 0;
+    for (int j = 0; j < S; ++j, ++s) {
+      g.A[s] = hsh + (int64_t)j * G; g.lda[s] = (int64_t)S * G;
+      g.B[s] = static_cast<const T*>(w->ws_o) + (int64_t)j * D * G; g.ldb[s] = G; g.K[s] = G;
+    }
+    g.A[s] = uhat; g.lda[s] = Lt; g.B[s] = w->w_up; g.ldb[s] = Lt; g.K[s] = Lt; ++s;
+    g.nseg = s; g.C = y; g.ldc = D; g.M = (int)N; g.N = D; g.mode = kStore;
+    ProfScope ps("final", st);
+    LMOE_CUDA(launch_simt_gemm<T>(g, st), "final");
+  }
+  return LMOE_OK;
+}
+
+static lmoe_status check_weights(const lmoe_dims* d, const lmoe_weights* w) {
+  if (w == nullptr) return fail(LMOE_EINVAL, "weights is NULL");
+  LMOE_PTR(w->w_down, "w_down");
+  LMOE_PTR(w->w_router, "w_router");
+  LMOE_PTR(w->w_up, "w_up");
+  LMOE_PTR(w->rms_weight, "rms_weight");
+  if (w->expert_bias != nullptr && !aligned16(w->expert_bias))
+    return fail(LMOE_EINVAL, "expert_bias is not 16-byte aligned");
+  LMOE_PTR(w->w_g, "w_g");
+  LMOE_PTR(w->w_u, "w_u");
+  LMOE_PTR(w->w_o, "w_o");
+  if (d->n_shared > 0) {
+    LMOE_PTR(w->ws_g, "ws_g");
+    LMOE_PTR(w->ws_u, "ws_u");
+    LMOE_PTR(w->ws_o, "ws_o");
+  }
+  return LMOE_OK;
+}
+
+}  // namespace lmoe
+
+using namespace lmoe;
+
+extern "C" {
+
+size_t lmoe_workspace_size(const lmoe_dims* dims) {
+  if (check_dims(dims) != LMOE_OK) return 0;
+  return layout(dims, false).total;
+}
+
+size_t lmoe_workspace_size_host(const lmoe_dims* dims) {
+  if (check_dims(dims) != LMOE_OK) return 0;
+  return layout(dims, true).total;
+}
+
+lmoe_status moe_route(const lmoe_dims* dims, const void* x, const void* w_router,
+                      const float* expert_bias, int32_t* ids, float* probs, void* ws,
+                      size_t ws_bytes, lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  if (dims->n_tokens > 0) {
+    LMOE_PTR(x, "x");
+    LMOE_PTR(ids, "ids");
+    LMOE_PTR(probs, "probs");
+  }
+  LMOE_PTR(w_router, "w_router");
+  if (expert_bias != nullptr && !aligned16(expert_bias))
+    return fail(LMOE_EINVAL, "expert_bias is not 16-byte aligned");
+  LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
+  LMOE_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dims->dtype == LMOE_BF16)
+    return run_route<__nv_bfloat16>(dims, x, w_router, expert_bias, ids, probs, ws, st);
+  return run_route<float>(dims, x, w_router, expert_bias, ids, probs, ws, st);
+}
+
+lmoe_status moe_dispatch(const lmoe_dims* dims, const int32_t* ids, int32_t* counts,
+                         int32_t* offsets, int32_t* perm_token, int32_t* inv_pair, void* ws,
+                         size_t ws_bytes, lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  if (dims->n_tokens > 0) {
+    LMOE_PTR(ids, "ids");
+    LMOE_PTR(perm_token, "perm_token");
+    LMOE_PTR(inv_pair, "inv_pair");
+  }
+  LMOE_PTR(counts, "counts");
+  LMOE_PTR(offsets, "offsets");
+  LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
+  LMOE_TRY(check_device());
+  return run_dispatch(dims, ids, counts, offsets, perm_token, inv_pair, ws, (cudaStream_t)stream);
+}
+
+lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const int32_t* perm_token,
+                           const int32_t* offsets, const void* w_g, const void* w_u,
+                           const void* w_o, void* expert_out, void* ws, size_t ws_bytes,
+                           lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  if (dims->n_tokens > 0) {
+    LMOE_PTR(z, "z");
+    LMOE_PTR(perm_token, "perm_token");
+    LMOE_PTR(expert_out, "expert_out");
+  }
+  LMOE_PTR(offsets, "offsets");
+  LMOE_PTR(w_g, "w_g");
+  LMOE_PTR(w_u, "w_u");
+  LMOE_PTR(w_o, "w_o");
+  LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
+  LMOE_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  const Layout L = layout(dims, false);
+  LMOE_CUDA(launch_build_tiles(offsets, dims->n_routed, &at<WsHeader>(ws, L.header)->n_mtiles,
+                               at<int4>(ws, L.tiles), st),
+            "build_tiles");
+  if (dims->dtype == LMOE_BF16)
+    return run_expert_ffn<__nv_bfloat16>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
+  return run_expert_ffn<float>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
+}
+
+lmoe_status moe_combine(const lmoe_dims* dims, const void* expert_out, const int32_t* inv_pair,
+                        const float* probs, const float* rms_weight, void* u_normed,
+                        lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  if (dims->n_tokens > 0) {
+    LMOE_PTR(expert_out, "expert_out");
+    LMOE_PTR(inv_pair, "inv_pair");
+    LMOE_PTR(probs, "probs");
+    LMOE_PTR(u_normed, "u_normed");
+  }
+  LMOE_PTR(rms_weight, "rms_weight");
+  LMOE_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dims->dtype == LMOE_BF16) {
+    LMOE_CUDA(launch_combine<__nv_bfloat16>((const __nv_bfloat16*)expert_out, inv_pair, probs,
+                                            rms_weight, dims->n_tokens, dims->top_k, dims->latent,
+                                            dims->rms_eps, (__nv_bfloat16*)u_normed, st),
+              "combine");
+  } else {
+    LMOE_CUDA(launch_combine<float>((const float*)expert_out, inv_pair, probs, rms_weight,
+                                    dims->n_tokens, dims->top_k, dims->latent, dims->rms_eps,
+                                    (float*)u_normed, st),
+              "combine");
+  }
+  return LMOE_OK;
+}
+
+lmoe_status latent_moe_forward(const lmoe_dims* dims, const lmoe_weights* weights, const void* x,
+                               void* y, int32_t* ids_out, float* probs_out, int32_t* counts_out,
+                               void* ws, size_t ws_bytes, lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  LMOE_TRY(check_weights(dims, weights));
+  if (dims->n_tokens > 0) {
+    LMOE_PTR(x, "x");
+    LMOE_PTR(y, "y");
+  }
+  if (ids_out && !aligned16(ids_out)) return fail(LMOE_EINVAL, "ids_out is not 16-byte aligned");
+  if (probs_out && !aligned16(probs_out)) return fail(LMOE_EINVAL, "probs_out is not 16-byte aligned");
+  if (counts_out && !aligned16(counts_out)) return fail(LMOE_EINVAL, "counts_out is not 16-byte aligned");
+  LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
+  LMOE_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dims->dtype == LMOE_BF16)
+    return run_forward<__nv_bfloat16>(dims, weights, x, y, ids_out, probs_out, counts_out, ws, st);
+  return run_forward<float>(dims, weights, x, y, ids_out, probs_out, counts_out, ws, st);
+}
+
+lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_weights* weights,
+                                    const void* x_host, void* y_host, void* ws, size_t ws_bytes,
+                                    lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  LMOE_TRY(check_weights(dims, weights));
+  if (dims->n_tokens > 0 && (x_host == nullptr || y_host == nullptr))
+    return fail(LMOE_EINVAL, "x_host / y_host is NULL");
+  LMOE_TRY(check_ws(dims, ws, ws_bytes, true));
+  LMOE_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  const Layout L = layout(dims, true);
+  const size_t bytes = (size_t)dims->n_tokens * dims->d * (dims->dtype == LMOE_BF16 ? 2 : 4);
+  void* xd = at<char>(ws, L.x);
+  void* yd = at<char>(ws, L.y);
+  if (bytes) LMOE_CUDA(cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st), "H2D x");
+  lmoe_status s;
+  if (dims->dtype == LMOE_BF16)
+    s = run_forward<__nv_bfloat16>(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st);
+  else
+    s = run_forward<float>(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st);
+  if (s != LMOE_OK) return s;
+  if (bytes) LMOE_CUDA(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st), "D2H y");
+  LMOE_CUDA(cudaStreamSynchronize(st), "sync");
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_workspace_init(void* ws, size_t ws_bytes, lmoe_stream stream) {
+  LMOE_PTR(ws, "ws");
+  if (ws_bytes < sizeof(WsHeader)) return fail(LMOE_EWORKSPACE, "workspace smaller than its header");
+  LMOE_CUDA(cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream), "memset header");
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_get_device_status(void* ws, lmoe_stream stream) {
+  LMOE_PTR(ws, "ws");
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t v = 0;
+  LMOE_CUDA(cudaMemcpyAsync(&v, &static_cast<WsHeader*>(ws)->status, sizeof(v),
+                            cudaMemcpyDeviceToHost, st),
+            "read status");
+  LMOE_CUDA(cudaStreamSynchronize(st), "sync");
+  if (v != 0) {
+    LMOE_CUDA(cudaMemsetAsync(&static_cast<WsHeader*>(ws)->status, 0, sizeof(int32_t), st),
+              "clear status");
+    LMOE_CUDA(cudaStreamSynchronize(st), "sync");
+    return v == LMOE_ETIMEOUT ? LMOE_ETIMEOUT : LMOE_EDEVICE;
+  }
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_selftest_capped_wait(void* ws, size_t ws_bytes, int32_t cap_ms,
+                                      lmoe_stream stream) {
+  LMOE_PTR(ws, "ws");
+  if (ws_bytes < sizeof(WsHeader)) return fail(LMOE_EWORKSPACE, "workspace smaller than its header");
+  if (cap_ms < 1 || cap_ms > 10000) return fail(LMOE_EINVAL, "cap_ms out of [1, 10000]");
+  LMOE_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  WsHeader* h = static_cast<WsHeader*>(ws);
+  // the flag nothing sets: a zeroed word of the header padding
+  LMOE_CUDA(cudaMemsetAsync(&h->pad[0], 0, sizeof(int32_t), st), "memset flag");
+  LMOE_CUDA(launch_capped_wait(&h->pad[0], &h->status, cap_ms, st), "capped wait");
+  return LMOE_OK;
+}
+
+const char* lmoe_status_string(lmoe_status s) {
+  switch (s) {
+    case LMOE_OK: return "LMOE_OK";
+    case LMOE_EINVAL: return "LMOE_EINVAL";
+    case LMOE_EUNSUPPORTED: return "LMOE_EUNSUPPORTED";
+    case LMOE_EWORKSPACE: return "LMOE_EWORKSPACE";
+    case LMOE_ECUDA: return "LMOE_ECUDA";
+    case LMOE_EDEVICE: return "LMOE_EDEVICE";
+    case LMOE_ETIMEOUT: return "LMOE_ETIMEOUT";
+  }
+  return "LMOE_UNKNOWN";
+}
+
+const char* lmoe_last_error(void) { return g_last_error.c_str(); }
+
+lmoe_status lmoe_profile_enable(const char* tag) {
+  g_prof_tag = tag ? tag : "";
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_profile_read(double* total_ms, int64_t* launches) {
+  double tot = 0.0;
+  int64_t n = 0;
+  for (auto& r : g_prof) {
+    float ms = 0.0f;
+    LMOE_CUDA(cudaEventSynchronize(r.b), "event sync");
+    LMOE_CUDA(cudaEventElapsedTime(&ms, r.a, r.b), "elapsed");
+    tot += ms;
+    ++n;
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof.clear();
+  if (total_ms) *total_ms = tot;
+  if (launches) *launches = n;
+  return LMOE_OK;
+}
+
+uint64_t lmoe_launch_count(int32_t reset) {
+  uint64_t v = g_launches;
+  if (reset) g_launches = 0;
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,100 @@
+// Weighted combine + RMSNorm (kda/layers/latent_moe.py: the index_add of
+// p-weighted expert outputs back to their tokens, then self.norm; sec-07
+// compute flow steps 3 and 5):
+//   u_t = sum_{i < k} p[t, i] * expert_out[inv_pair[t, i]]     (slot order, fp32)
+//   u_normed_t = u_t * (1 / sqrt(mean(u_t^2) + eps)) * w
+// Each token is reduced by one warp in a fixed order: no float atomics, so
+// the result is deterministic.  Rows are read with 16-byte vectors.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lmoe {
+namespace {
+
+template <typename T, int VPL>  // VPL: 16-byte vectors per lane
+__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ eo,
+                                                      const int32_t* __restrict__ inv_pair,
+                                                      const float* __restrict__ probs,
+                                                      const float* __restrict__ rms_w, int64_t n,
+                                                      int k, int L, float eps, T* __restrict__ out) {
+  constexpr int E = 16 / sizeof(T);  // elements per vector
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= n) return;
+  const int nvec = L / E;
+  float u[VPL][E];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v)
+#pragma unroll
+    for (int e = 0; e < E; ++e) u[v][e] = 0.0f;
+  for (int i = 0; i < k; ++i) {
+    const int64_t r = inv_pair[t * k + i];
+    const float p = probs[t * k + i];
+    const uint4* row = reinterpret_cast<const uint4*>(eo + r * L);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      int vi = v * 32 + lane;
+      if (vi < nvec) {
+        uint4 raw = row[vi];
+        const T* el = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+        for (int e = 0; e < E; ++e) u[v][e] = fmaf(p, to_f(el[e]), u[v][e]);
+      }
+    }
+  }
+  float ss = 0.0f;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v)
+#pragma unroll
+    for (int e = 0; e < E; ++e) ss = fmaf(u[v][e], u[v][e], ss);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float inv = rsqrtf(ss / (float)L + eps);
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    int vi = v * 32 + lane;
+    if (vi < nvec) {
+      uint4 raw;
+      T* el = reinterpret_cast<T*>(&raw);
+#pragma unroll
+      for (int e = 0; e < E; ++e) el[e] = from_f<T>(u[v][e] * inv * rms_w[vi * E + e]);
+      reinterpret_cast<uint4*>(out + t * L)[vi] = raw;
+    }
+  }
+}
+
+}  // namespace
+
+template <typename T>
+cudaError_t launch_combine(const T* eo, const int32_t* inv_pair, const float* probs,
+                           const float* rms_w, int64_t n, int k, int L, float eps, T* out,
+                           cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  constexpr int E = 16 / sizeof(T);
+  const int nvec = L / E;
+  const int vpl = (nvec + 31) / 32;
+  const int warps = 8;
+  unsigned blocks = (unsigned)((n + warps - 1) / warps);
+#define LMOE_COMBINE_CASE(V)                                                              \
+  if (vpl <= V) {                                                                         \
+    combine_kernel<T, V><<<blocks, warps * 32, 0, st>>>(eo, inv_pair, probs, rms_w, n, k, L, \
+                                                        eps, out);                        \
+    count_launch();                                                                       \
+    return cudaGetLastError();                                                            \
+  }
+  LMOE_COMBINE_CASE(1)
+  LMOE_COMBINE_CASE(2)
+  LMOE_COMBINE_CASE(4)
+  LMOE_COMBINE_CASE(8)
+  LMOE_COMBINE_CASE(16)
+#undef LMOE_COMBINE_CASE
+  return cudaErrorInvalidValue;
+}
+template cudaError_t launch_combine<float>(const float*, const int32_t*, const float*,
+                                           const float*, int64_t, int, int, float, float*,
+                                           cudaStream_t);
+template cudaError_t launch_combine<__nv_bfloat16>(const __nv_bfloat16*, const int32_t*,
+                                                   const float*, const float*, int64_t, int, int,
+                                                   float, __nv_bfloat16*, cudaStream_t);
+
+}  // namespace lmoe

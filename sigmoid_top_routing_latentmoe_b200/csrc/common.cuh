@@ -1,0 +1,46 @@
+// Shared device helpers of the LatentMoE CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/latent_moe.h"
+
+namespace lmoe {
+
+// Status word values written on the device (same codes as lmoe_status).
+constexpr int kStatusDevice = LMOE_EDEVICE;
+constexpr int kStatusTimeout = LMOE_ETIMEOUT;
+
+// Routed GEMMs are scheduled in row tiles of this many sorted pairs.
+constexpr int kTileM = 128;
+
+// Header at the start of every workspace.
+struct WsHeader {
+  int32_t status;        // 0, or the first failure code recorded on the device
+  int32_t n_mtiles;      // number of routed row tiles (written by dispatch)
+  int32_t pad[62];
+};
+
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ void record_status(int32_t* status, int code) {
+  atomicCAS(status, 0, code);
+}
+
+// Exact fp32 SiTU-GLU hidden unit: beta1 tanh(a/beta1) sigmoid(a) * beta2 tanh(c/beta2).
+__device__ __forceinline__ float situ_exact(float a, float c, float beta1, float beta2) {
+  float gate = beta1 * tanhf(a / beta1) * (1.0f / (1.0f + expf(-a)));
+  float up = beta2 * tanhf(c / beta2);
+  return gate * up;
+}
+
+}  // namespace lmoe

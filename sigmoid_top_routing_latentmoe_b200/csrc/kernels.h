@@ -1,0 +1,78 @@
+// Internal launch interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lmoe {
+
+// ---------------------------------------------------------------- routing
+// Warp-per-token router for small R (<= 32): fp32 GEMV over W_r, sigmoid,
+// biased top-k in registers, L1 normalisation.  T = float or bf16.
+template <typename T>
+cudaError_t launch_route_gemv(const T* x, const T* w_r, const float* bias, int64_t n, int d, int R,
+                              int k, int32_t* ids, float* probs, cudaStream_t st);
+// Top-k + normalisation from precomputed fp32 logits [n, ld] (R valid columns).
+cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias, int64_t n, int R,
+                              int k, int32_t* ids, float* probs, cudaStream_t st);
+
+// ----------------------------------------------------------- permutation
+struct DispatchScratch {
+  int32_t* block_counts;  // [n_blocks, R]
+  int32_t* status;        // workspace status word
+  int32_t* n_mtiles;      // out: number of routed row tiles
+  int4* tiles;            // out: [max_tiles] (expert, row0, rows, 0)
+};
+int dispatch_blocks(int64_t n_pairs);
+cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
+                            int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
+                            const DispatchScratch& s, cudaStream_t st);
+cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
+                               cudaStream_t st);
+// zp[r, :] = z[perm_token[r], :]
+template <typename T>
+cudaError_t launch_gather_rows(const T* z, const int32_t* perm_token, int64_t n_rows, int width,
+                               T* zp, cudaStream_t st);
+
+// ------------------------------------------------------------ SIMT GEMM
+// C[m, n] = sum_s A_s[m, :K_s] . B_s[n, :K_s]  (all operands K-contiguous).
+// mode kStore: C = acc (T or fp32 out);  kSitu: two accumulators against B and
+// B_up, C = SiTU(acc_g, acc_u).  Ragged: rows come from the tile list and B
+// pointers advance by b_expert_stride elements per expert.
+constexpr int kMaxSeg = 8;
+enum SimtMode { kStore = 0, kSitu = 1 };
+struct SimtGemm {
+  const void* A[kMaxSeg];
+  int64_t lda[kMaxSeg];
+  const void* B[kMaxSeg];
+  int64_t ldb[kMaxSeg];
+  int K[kMaxSeg];
+  int nseg;
+  const void* B_up;        // SiTU mode: up-projection rows (same ldb as B[0])
+  int64_t b_expert_stride; // ragged mode: elements between experts' weights
+  void* C;
+  int64_t ldc;
+  int M, N;                // dense mode rows; output columns
+  int out_f32;             // 1: C is fp32 regardless of T
+  const int4* tiles;       // ragged mode tile list or nullptr
+  const int32_t* n_tiles;
+  int max_tiles;
+  float beta1, beta2;
+  int mode;
+};
+template <typename T>
+cudaError_t launch_simt_gemm(const SimtGemm& g, cudaStream_t st);
+
+// -------------------------------------------------------------- combine
+template <typename T>
+cudaError_t launch_combine(const T* expert_out, const int32_t* inv_pair, const float* probs,
+                           const float* rms_w, int64_t n, int k, int L, float eps, T* out,
+                           cudaStream_t st);
+
+// ------------------------------------------------------------ self-test
+cudaError_t launch_capped_wait(int32_t* flag, int32_t* status, int cap_ms, cudaStream_t st);
+
+// Launch counter (api.cu)
+void count_launch(int n = 1);
+
+}  // namespace lmoe

@@ -1,0 +1,181 @@
+// Router kernels: K3 sigmoid routing (sec-07 compute flow step 2, K3 eq.13;
+// kda/layers/latent_moe.py LatentMoE._route):
+//   l = W_r x,  s = sigmoid(l),  T = TopK(s + b, k),  p_i = s_i / max(sum_T s, 1e-9).
+// The bias enters the selection only.  Slots are written in descending key
+// order; equal keys go to the lower expert index.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lmoe {
+namespace {
+
+__device__ __forceinline__ float sigmoid_f(float l) { return 1.0f / (1.0f + expf(-l)); }
+
+// Warp-wide selection of the largest key (ties: lower expert index).
+__device__ __forceinline__ void warp_argmax(float& key, int& idx) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    float ok = __shfl_xor_sync(0xffffffffu, key, off);
+    int oi = __shfl_xor_sync(0xffffffffu, idx, off);
+    if (ok > key || (ok == key && oi < idx)) {
+      key = ok;
+      idx = oi;
+    }
+  }
+}
+
+// Top-k over R <= 32 * VPL experts held VPL per lane (expert e = j*32 + lane),
+// then p = s / max(sum s, 1e-9).  Called by all 32 lanes of a warp.
+template <int VPL>
+__device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (&key_in)[VPL], int R,
+                                            int k, int32_t* ids_row, float* probs_row) {
+  const int lane = threadIdx.x & 31;
+  float key[VPL];
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) key[j] = (j * 32 + lane < R) ? key_in[j] : -INFINITY;
+  float den = 0.0f;
+  float sel_s = 0.0f;  // score of the slot this lane will write (lane == slot)
+  int sel_id = 0;
+  for (int slot = 0; slot < k; ++slot) {
+    float bk = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      int e = j * 32 + lane;
+      if (e < R && (key[j] > bk || (key[j] == bk && e < bi))) {
+        bk = key[j];
+        bi = e;
+      }
+    }
+    warp_argmax(bk, bi);
+    // owner lane retires the winner and broadcasts its raw score
+    float sc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      if (j * 32 + lane == bi) {
+        key[j] = -INFINITY;
+        sc = s[j];
+      }
+    }
+    sc = __shfl_sync(0xffffffffu, sc, bi & 31);
+    den += sc;
+    if ((slot & 31) == lane) {
+      sel_s = sc;
+      sel_id = bi;
+    }
+    if ((slot & 31) == 31 || slot == k - 1) {
+      // flush a group of up to 32 slots
+      int base = slot & ~31;
+      if (lane <= (slot & 31)) ids_row[base + lane] = sel_id;
+      // probs need the full sum: stash scores in probs_row for now
+      if (lane <= (slot & 31)) probs_row[base + lane] = sel_s;
+    }
+  }
+  den = fmaxf(den, 1e-9f);
+  __syncwarp();
+  for (int slot = lane; slot < k; slot += 32) probs_row[slot] = probs_row[slot] / den;
+}
+
+// One warp per token.  W_r rows are read through L1/L2 (R <= 32 rows).
+// Each lane accumulates its share of d for every expert, then a butterfly
+// reduction leaves lane e holding expert e's logit.
+template <typename T>
+__global__ void __launch_bounds__(256) route_gemv_kernel(const T* __restrict__ x,
+                                                         const T* __restrict__ w_r,
+                                                         const float* __restrict__ bias, int64_t n,
+                                                         int d, int R, int k,
+                                                         int32_t* __restrict__ ids,
+                                                         float* __restrict__ probs) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= n) return;
+  const T* xr = x + t * d;
+  float acc[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
+  for (int i = lane; i < d; i += 32) {
+    float xv = to_f(xr[i]);
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (e < R) acc[e] = fmaf(to_f(w_r[(int64_t)e * d + i]), xv, acc[e]);
+  }
+  // transpose-reduce: after the loop lane e holds sum over lanes of acc[e]
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  }
+  float logit = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 32; ++e)
+    if (e == lane) logit = acc[e];
+  float s[1], key[1];
+  s[0] = sigmoid_f(logit);
+  key[0] = s[0] + ((bias != nullptr && lane < R) ? bias[lane] : 0.0f);
+  select_topk<1>(s, key, R, k, ids + t * k, probs + t * k);
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
+                                                         int64_t ld, const float* __restrict__ bias,
+                                                         int64_t n, int R, int k,
+                                                         int32_t* __restrict__ ids,
+                                                         float* __restrict__ probs) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= n) return;
+  const float* lr = logits + t * ld;
+  float s[VPL], key[VPL];
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    int e = j * 32 + lane;
+    float l = (e < R) ? lr[e] : 0.0f;
+    s[j] = sigmoid_f(l);
+    key[j] = s[j] + ((bias != nullptr && e < R) ? bias[e] : 0.0f);
+  }
+  select_topk<VPL>(s, key, R, k, ids + t * k, probs + t * k);
+}
+
+}  // namespace
+
+template <typename T>
+cudaError_t launch_route_gemv(const T* x, const T* w_r, const float* bias, int64_t n, int d, int R,
+                              int k, int32_t* ids, float* probs, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int warps = 8;
+  int64_t blocks = (n + warps - 1) / warps;
+  route_gemv_kernel<T><<<(unsigned)blocks, warps * 32, 0, st>>>(x, w_r, bias, n, d, R, k, ids, probs);
+  count_launch();
+  return cudaGetLastError();
+}
+template cudaError_t launch_route_gemv<float>(const float*, const float*, const float*, int64_t,
+                                              int, int, int, int32_t*, float*, cudaStream_t);
+template cudaError_t launch_route_gemv<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                                      const float*, int64_t, int, int, int,
+                                                      int32_t*, float*, cudaStream_t);
+
+cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias, int64_t n, int R,
+                              int k, int32_t* ids, float* probs, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int warps = 8;
+  unsigned blocks = (unsigned)((n + warps - 1) / warps);
+  int vpl = (R + 31) / 32;
+#define LMOE_TOPK_CASE(V)                                                                  \
+  if (vpl <= V) {                                                                          \
+    route_topk_kernel<V><<<blocks, warps * 32, 0, st>>>(logits, ld, bias, n, R, k, ids, probs); \
+    count_launch();                                                                        \
+    return cudaGetLastError();                                                             \
+  }
+  LMOE_TOPK_CASE(1)
+  LMOE_TOPK_CASE(2)
+  LMOE_TOPK_CASE(4)
+  LMOE_TOPK_CASE(8)
+  LMOE_TOPK_CASE(16)
+  LMOE_TOPK_CASE(32)
+  LMOE_TOPK_CASE(64)
+  LMOE_TOPK_CASE(128)
+#undef LMOE_TOPK_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lmoe
