@@ -124,6 +124,22 @@ def _dist():
     return world, rank, local
 
 
+def rank_token_rows(wl: synth.Workload, rank: int) -> np.ndarray:
+    """Token rows of one replica: rank r draws x rows [r*N, (r+1)*N) of the stream."""
+    return np.arange(wl.n_tokens, dtype=np.int64) + rank * wl.n_tokens
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank number over the process group (the value itself at N = 1)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def cpu_baseline(wl: synth.Workload, seed: int, budget_s: float = 12.0) -> dict:
     """The oracle as it stands on the host cores, on a bounded sample of the
     workload's tokens: first a small probe, then a sample sized to ~budget_s."""
@@ -225,7 +241,7 @@ def main():
 
     # inputs: weights shared by all ranks (seed), x drawn per rank (its own tokens)
     inp = synth.make_inputs(wl, args.seed, with_x=False)
-    x_np = synth.make_x_rows(wl, args.seed, np.arange(wl.n_tokens) + rank * wl.n_tokens)
+    x_np = synth.make_x_rows(wl, args.seed, rank_token_rows(wl, rank))
 
     def todev(a):
         if a.dtype == np.uint16:
@@ -278,11 +294,7 @@ def main():
     lm.profile_enable(None)
     k_ms, k_n = lm.profile_read()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
     value = world * wl.n_tokens / (ms_per_step / 1e3)
     if lm.get_device_status(ws) != lm.OK:
@@ -303,11 +315,7 @@ def main():
         lm.latent_moe_forward_host(dims, wstruct, x_h, y_h, ws_h)
     ev1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, dev)
     io_bytes = wl.n_tokens * wl.d * (2 if wl.dtype == "bf16" else 4)
 
     peaks = _peaks()

@@ -167,6 +167,13 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
                                     const void* x_host, void* y_host, void* ws, size_t ws_bytes,
                                     lmoe_stream stream);
 
+/* Byte offsets of the forward's intermediates inside the workspace, for
+ * inspection after latent_moe_forward: offsets[0..6] = z [N,l], router logits
+ * [N, ld] fp32, shared hidden units [N, S*G], RMSNorm(u) [N,l], routed expert
+ * outputs [N*k, l], routed hidden units [N*k, F], sorted z rows [N*k, l];
+ * offsets[7] = ld, the row stride (elements) of the logits. */
+LMOE_API lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offsets, int32_t n);
+
 /* Zeroes the workspace header (status word and scheduling counters).  Call
  * once on a new workspace before its first use. */
 LMOE_API lmoe_status lmoe_workspace_init(void* ws, size_t ws_bytes, lmoe_stream stream);

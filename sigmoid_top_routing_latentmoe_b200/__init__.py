@@ -73,6 +73,7 @@ _sigs = {
     "lmoe_last_error": (ctypes.c_char_p, []),
     "lmoe_launch_count": (ctypes.c_uint64, [ctypes.c_int32]),
     "lmoe_profile_enable": (_S, [ctypes.c_char_p]),
+    "lmoe_workspace_layout": (_S, [_DP, ctypes.POINTER(ctypes.c_size_t), ctypes.c_int32]),
     "lmoe_profile_read": (_S, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
 }
 for _name, (_res, _args) in _sigs.items():
@@ -122,6 +123,25 @@ def alloc_workspace(dims: Dims, device="cuda", host: bool = False, stream=None) 
     ws = ws[off:off + n]
     workspace_init(ws, stream)
     return ws
+
+
+def workspace_views(dims: Dims, ws: torch.Tensor) -> dict:
+    """Views of the forward's intermediates inside ``ws`` (for inspection)."""
+    off = (ctypes.c_size_t * 8)()
+    _check(_lib.lmoe_workspace_layout(ctypes.byref(dims), off, 8), "lmoe_workspace_layout")
+    act = torch.bfloat16 if dims.dtype == BF16 else torch.float32
+    es = 2 if dims.dtype == BF16 else 4
+    N, L, k, F = dims.n_tokens, dims.latent, dims.top_k, dims.ff_routed
+    SG = dims.n_shared * dims.ff_shared
+
+    def view(o, rows, cols, dt, size):
+        return ws[o:o + rows * cols * size].view(dt).view(rows, cols)
+
+    return {"z": view(off[0], N, L, act, es),
+            "logits": view(off[1], N, off[7], torch.float32, 4)[:, :dims.n_routed],
+            "hsh": view(off[2], N, SG, act, es), "uhat": view(off[3], N, L, act, es),
+            "eo": view(off[4], N * k, L, act, es), "h": view(off[5], N * k, F, act, es),
+            "zp": view(off[6], N * k, L, act, es)}
 
 
 def workspace_init(ws: torch.Tensor, stream=None):

@@ -5,10 +5,12 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 #include <vector>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "umma_gemm.h"
 
 namespace lmoe {
 
@@ -189,11 +191,19 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
   }
   float* logits = at<float>(ws, L.logits);
   ProfScope ps("route", st);
-  SimtGemm g{};
-  g.A[0] = x; g.lda[0] = d->d; g.B[0] = w_r; g.ldb[0] = d->d; g.K[0] = d->d; g.nseg = 1;
-  g.C = logits; g.ldc = L.logits_ld; g.M = (int)N; g.N = d->n_routed; g.out_f32 = 1;
-  g.mode = kStore;
-  LMOE_CUDA(launch_simt_gemm<T>(g, st), "router logits");
+  if (std::is_same<T, __nv_bfloat16>::value) {
+    XpassArgs a{};
+    a.x = (const __nv_bfloat16*)x; a.N = N; a.d = d->d; a.L = 0; a.w_router = (const __nv_bfloat16*)w_r;
+    a.R = d->n_routed; a.S = 0; a.logits = logits; a.logits_ld = L.logits_ld;
+    a.beta1 = d->beta1; a.beta2 = d->beta2;
+    LMOE_CUDA(umma_xpass(a, &at<WsHeader>(ws, L.header)->status, st), "router logits (tcgen05)");
+  } else {
+    SimtGemm g{};
+    g.A[0] = x; g.lda[0] = d->d; g.B[0] = w_r; g.ldb[0] = d->d; g.K[0] = d->d; g.nseg = 1;
+    g.C = logits; g.ldc = L.logits_ld; g.M = (int)N; g.N = d->n_routed; g.out_f32 = 1;
+    g.mode = kStore;
+    LMOE_CUDA(launch_simt_gemm<T>(g, st), "router logits");
+  }
   LMOE_CUDA(launch_route_topk(logits, L.logits_ld, bias, N, d->n_routed, d->top_k, ids, probs, st),
             "route_topk");
   return LMOE_OK;
@@ -237,9 +247,20 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   g1.B_up = w_u; g1.b_expert_stride = (int64_t)F * Lt;
   g1.C = h; g1.ldc = F; g1.N = F; g1.tiles = tiles; g1.n_tiles = n_tiles;
   g1.max_tiles = L.max_tiles; g1.beta1 = d->beta1; g1.beta2 = d->beta2; g1.mode = kSitu;
+  const bool tc = std::is_same<T, __nv_bfloat16>::value;
+  int32_t* status = &at<WsHeader>(ws, L.header)->status;
+  RoutedArgs ra{};
+  ra.P = P; ra.L = Lt; ra.F = F; ra.R = d->n_routed; ra.tiles = tiles; ra.n_mtiles = n_tiles;
+  ra.max_tiles = L.max_tiles; ra.beta1 = d->beta1; ra.beta2 = d->beta2;
   {
     ProfScope ps("expert_gemm1", st);
-    LMOE_CUDA(launch_simt_gemm<T>(g1, st), "routed gemm1");
+    if (tc) {
+      ra.a = (const __nv_bfloat16*)zp; ra.w0 = (const __nv_bfloat16*)w_g;
+      ra.w1 = (const __nv_bfloat16*)w_u; ra.out = (__nv_bfloat16*)h;
+      LMOE_CUDA(umma_routed1(ra, status, st), "routed gemm1 (tcgen05)");
+    } else {
+      LMOE_CUDA(launch_simt_gemm<T>(g1, st), "routed gemm1");
+    }
   }
   SimtGemm g2{};
   g2.A[0] = h; g2.lda[0] = F; g2.B[0] = w_o; g2.ldb[0] = F; g2.K[0] = F; g2.nseg = 1;
@@ -248,7 +269,13 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   g2.max_tiles = L.max_tiles; g2.mode = kStore;
   {
     ProfScope ps("expert_gemm2", st);
-    LMOE_CUDA(launch_simt_gemm<T>(g2, st), "routed gemm2");
+    if (tc) {
+      ra.a = (const __nv_bfloat16*)h; ra.w0 = (const __nv_bfloat16*)w_o; ra.w1 = nullptr;
+      ra.out = (__nv_bfloat16*)eo;
+      LMOE_CUDA(umma_routed2(ra, status, st), "routed gemm2 (tcgen05)");
+    } else {
+      LMOE_CUDA(launch_simt_gemm<T>(g2, st), "routed gemm2");
+    }
   }
   return LMOE_OK;
 }
@@ -275,25 +302,48 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
     LMOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * d->n_routed, st), "memset");
     return LMOE_OK;
   }
-  // step 1: z = W_down x
-  {
-    SimtGemm g{};
-    g.A[0] = x; g.lda[0] = D; g.B[0] = w->w_down; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
-    g.C = z; g.ldc = Lt; g.M = (int)N; g.N = Lt; g.mode = kStore;
+  const bool tc = std::is_same<T, __nv_bfloat16>::value;
+  int32_t* status = &at<WsHeader>(ws, L.header)->status;
+  float* logits = at<float>(ws, L.logits);
+  if (tc) {
+    // steps 1, 2 (logits) and 4 (shared hidden units) in one tcgen05 pass over x
+    XpassArgs a{};
+    a.x = (const __nv_bfloat16*)x; a.N = N; a.d = D;
+    a.w_down = (const __nv_bfloat16*)w->w_down; a.L = Lt;
+    a.w_router = (const __nv_bfloat16*)w->w_router; a.R = d->n_routed;
+    a.ws_g = (const __nv_bfloat16*)w->ws_g; a.ws_u = (const __nv_bfloat16*)w->ws_u; a.S = S; a.G = G;
+    a.z = (__nv_bfloat16*)z; a.logits = logits; a.logits_ld = L.logits_ld;
+    a.hsh = (__nv_bfloat16*)hsh; a.beta1 = d->beta1; a.beta2 = d->beta2;
     ProfScope ps("xpass", st);
-    LMOE_CUDA(launch_simt_gemm<T>(g, st), "down");
+    LMOE_CUDA(umma_xpass(a, status, st), "x-pass (tcgen05)");
+  } else {
+    // step 1: z = W_down x
+    {
+      SimtGemm g{};
+      g.A[0] = x; g.lda[0] = D; g.B[0] = w->w_down; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
+      g.C = z; g.ldc = Lt; g.M = (int)N; g.N = Lt; g.mode = kStore;
+      ProfScope ps("xpass", st);
+      LMOE_CUDA(launch_simt_gemm<T>(g, st), "down");
+    }
+    // step 4 (independent of routing): h_sh = SiTU hidden of the shared experts
+    if (S > 0) {
+      SimtGemm g{};
+      g.A[0] = x; g.lda[0] = D; g.B[0] = w->ws_g; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
+      g.B_up = w->ws_u; g.C = hsh; g.ldc = (int64_t)S * G; g.M = (int)N; g.N = S * G;
+      g.beta1 = d->beta1; g.beta2 = d->beta2; g.mode = kSitu;
+      ProfScope ps("xpass", st);
+      LMOE_CUDA(launch_simt_gemm<T>(g, st), "shared gemm1");
+    }
   }
-  // step 4 (independent of routing): h_sh = SiTU hidden of the shared experts
-  if (S > 0) {
-    SimtGemm g{};
-    g.A[0] = x; g.lda[0] = D; g.B[0] = w->ws_g; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
-    g.B_up = w->ws_u; g.C = hsh; g.ldc = (int64_t)S * G; g.M = (int)N; g.N = S * G;
-    g.beta1 = d->beta1; g.beta2 = d->beta2; g.mode = kSitu;
-    ProfScope ps("xpass", st);
-    LMOE_CUDA(launch_simt_gemm<T>(g, st), "shared gemm1");
+  // step 2: routing (top-k + normalisation from the x-pass logits on the tcgen05 path)
+  if (tc) {
+    ProfScope ps("route", st);
+    LMOE_CUDA(launch_route_topk(logits, L.logits_ld, w->expert_bias, N, d->n_routed, d->top_k, ids,
+                                probs, st),
+              "route_topk");
+  } else {
+    LMOE_TRY(run_route<T>(d, x, w->w_router, w->expert_bias, ids, probs, ws, st));
   }
-  // step 2: routing
-  LMOE_TRY(run_route<T>(d, x, w->w_router, w->expert_bias, ids, probs, ws, st));
   // step 3: dispatch, routed experts, combine + RMSNorm
   LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st));
   LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st));
@@ -304,7 +354,14 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
               "combine");
   }
   // step 5: y = sum_j W_o,sh_j h_sh_j + W_up uhat
-  {
+  if (tc) {
+    FinalArgs a{};
+    a.hsh = (const __nv_bfloat16*)hsh; a.N = N; a.S = S; a.G = G;
+    a.ws_o = (const __nv_bfloat16*)w->ws_o; a.d = D; a.uhat = (const __nv_bfloat16*)uhat; a.L = Lt;
+    a.w_up = (const __nv_bfloat16*)w->w_up; a.y = (__nv_bfloat16*)y;
+    ProfScope ps("final", st);
+    LMOE_CUDA(umma_final(a, status, st), "final (tcgen05)");
+  } else {
     SimtGemm g{};
     int s = 0;
     for (int j = 0; j < S; ++j, ++s) {
@@ -486,6 +543,15 @@ lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_weights* w
   if (s != LMOE_OK) return s;
   if (bytes) LMOE_CUDA(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st), "D2H y");
   LMOE_CUDA(cudaStreamSynchronize(st), "sync");
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offsets, int32_t n) {
+  LMOE_TRY(check_dims(dims));
+  if (offsets == nullptr || n < 8) return fail(LMOE_EINVAL, "offsets needs 8 entries");
+  const Layout L = layout(dims, false);
+  const size_t v[8] = {L.z, L.logits, L.hsh, L.uhat, L.eo, L.h, L.zp, (size_t)L.logits_ld};
+  for (int i = 0; i < 8; ++i) offsets[i] = v[i];
   return LMOE_OK;
 }
 

@@ -1,0 +1,738 @@
+// tcgen05 GEMM engine for the bf16 LatentMoE forward (sm_100a).
+//
+// One persistent, warp-specialised kernel template serves the four GEMMs of
+// the layer.  Every tile is 128 rows x (128 or 256) columns, K in blocks of 64
+// bf16 (one 128-byte swizzle atom):
+//   warp 0   TMA producer: cp.async.bulk.tensor loads of the A tile and of
+//            one or two 128-row B sub-tiles into a 4-stage smem ring,
+//   warp 1   MMA issuer: tcgen05.mma.kind::f16 (bf16 x bf16 -> fp32) into a
+//            double-buffered TMEM accumulator (2 x 256 columns), and the
+//            TMEM allocator,
+//   warps 2-5 epilogue: tcgen05.ld of the accumulator, the fused epilogue of
+//            the GEMM (bf16/fp32 store, or the SiTU-GLU hidden unit of a
+//            gate/up column pair), 16-byte global stores.
+// The four GEMMs (sec-07 compute flow; kda/layers/latent_moe.py):
+//   XPASS   x [N, d] against [W_down | W_r | (W_g,sh, W_u,sh) pairs]: z, the
+//           router logits (step 2) and the shared experts' SiTU hidden units
+//           (step 4) in one pass over x.
+//   ROUTED1 sorted pairs z[perm] against (W_g,e, W_u,e) pairs: SiTU hidden
+//           units of the routed experts (step 3), row tiles from the device
+//           tile list (no padding to a capacity).
+//   ROUTED2 routed hidden units against W_o,e.
+//   FINAL   [h_sh | RMSNorm(u)] against [W_o,sh | W_up]: the shared experts'
+//           output projection and the latent restore summed in one
+//           accumulator (step 5, y = s_sh + W_up RMSNorm(u)).
+// Every mbarrier wait is capped: after ~2 s the kernel records LMOE_ETIMEOUT,
+// stops issuing work, drains what it issued, frees its TMEM and returns.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "umma_gemm.h"
+
+namespace lmoe {
+namespace {
+
+constexpr int BM = 128;          // tile rows (TMEM lanes)
+constexpr int BK = 64;           // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int SUB = 128;         // rows of one B sub-tile
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int SUB_BYTES = SUB * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + 2 * SUB_BYTES;  // 48 KB
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int THREADS = 192;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+constexpr uint64_t WAIT_CAP_NS = 2000000000ull;
+
+enum Mode { XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3 };
+enum Epi { EPI_Z = 1, EPI_LOGIT = 2, EPI_SITU = 3, EPI_STORE = 4 };
+
+struct Params {
+  CUtensorMap tmA0, tmA1;              // A operands (FINAL: h_sh, uhat)
+  CUtensorMap tmB0, tmB1, tmB2, tmB3;  // B operands (see decode_tile)
+  int M;                               // dense rows
+  int n_tiles;                         // tiles along the output columns
+  int kb0, kb1;                        // K blocks (FINAL: per shared expert, then uhat)
+  int S, G, L, R, F, d;
+  int nz_sub, nr_sub, n_zr_tiles, g_blocks;
+  void* out0;
+  void* out1;
+  void* out2;
+  int64_t ld0, ld1, ld2;
+  const int4* tiles;
+  const int32_t* n_mtiles;
+  int32_t* status;
+  float beta1, beta2, inv_beta1, inv_beta2;
+};
+
+struct Tile {
+  int m0, rows, expert, n_sub;
+  int bmap[2], brow[2], bz[2], epi, ocol;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Capped wait: false if the cap ran out (status recorded) or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  uint32_t it = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > WAIT_CAP_NS) {
+        *abort_flag = 1;
+        record_status(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 lanes x 32 columns of fp32: thread i of the warp gets row (lane base + i).
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
+// core groups 1024 bytes apart (SBO), descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = n.
+__device__ __forceinline__ uint32_t instr_desc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ float tanh_fast(float v) {
+  float r;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+// SiTU-GLU hidden unit: beta1 tanh(a/beta1) sigmoid(a) * beta2 tanh(c/beta2).
+__device__ __forceinline__ float situ_fast(float a, float c, const Params& p) {
+  float gate = p.beta1 * tanh_fast(a * p.inv_beta1) * __fdividef(1.0f, 1.0f + __expf(-a));
+  float up = p.beta2 * tanh_fast(c * p.inv_beta2);
+  return gate * up;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ---------------------------------------------------------- tile decoding
+template <int MODE>
+__device__ __forceinline__ int total_tiles(const Params& p) {
+  if (MODE == XPASS || MODE == FINAL) return ((p.M + BM - 1) / BM) * p.n_tiles;
+  return (*p.n_mtiles) * p.n_tiles;
+}
+
+template <int MODE>
+__device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
+  Tile tl;
+  tl.bz[0] = tl.bz[1] = 0;
+  if (MODE == XPASS || MODE == FINAL) {
+    const int m_tiles = (p.M + BM - 1) / BM;
+    const int mt = t % m_tiles, n = t / m_tiles;
+    tl.m0 = mt * BM;
+    tl.rows = min(BM, p.M - tl.m0);
+    tl.expert = 0;
+    if (MODE == FINAL) {
+      tl.n_sub = (n * 2 * SUB + SUB < p.d) ? 2 : 1;
+      tl.bmap[0] = tl.bmap[1] = 0;
+      tl.brow[0] = n * 2 * SUB;
+      tl.brow[1] = n * 2 * SUB + SUB;
+      tl.epi = EPI_STORE;
+      tl.ocol = n * 2 * SUB;
+    } else if (n < p.n_zr_tiles) {
+      tl.n_sub = 0;
+      for (int s = 0; s < 2; ++s) {
+        const int idx = 2 * n + s;
+        if (idx < p.nz_sub) {
+          tl.bmap[s] = 0;
+          tl.brow[s] = idx * SUB;
+          tl.n_sub = s + 1;
+        } else if (idx < p.nz_sub + p.nr_sub) {
+          tl.bmap[s] = 1;
+          tl.brow[s] = (idx - p.nz_sub) * SUB;
+          tl.n_sub = s + 1;
+        }
+      }
+      tl.epi = EPI_Z;  // per sub-tile: Z or LOGIT, resolved in the epilogue
+      tl.ocol = 2 * n;
+    } else {
+      const int q = n - p.n_zr_tiles;
+      const int j = q / p.g_blocks, fb = q % p.g_blocks;
+      tl.n_sub = 2;
+      tl.bmap[0] = 2;
+      tl.bmap[1] = 3;
+      tl.brow[0] = tl.brow[1] = fb * SUB;
+      tl.bz[0] = tl.bz[1] = j;
+      tl.epi = EPI_SITU;
+      tl.ocol = j * p.G + fb * SUB;
+    }
+  } else {
+    const int mt = t / p.n_tiles, n = t % p.n_tiles;
+    const int4 e = p.tiles[mt];
+    tl.expert = e.x;
+    tl.m0 = e.y;
+    tl.rows = e.z;
+    tl.bz[0] = tl.bz[1] = e.x;
+    if (MODE == ROUTED1) {
+      tl.n_sub = 2;
+      tl.bmap[0] = 0;
+      tl.bmap[1] = 1;
+      tl.brow[0] = tl.brow[1] = n * SUB;
+      tl.epi = EPI_SITU;
+      tl.ocol = n * SUB;
+    } else {
+      tl.n_sub = (n * 2 * SUB + SUB < p.L) ? 2 : 1;
+      tl.bmap[0] = tl.bmap[1] = 0;
+      tl.brow[0] = n * 2 * SUB;
+      tl.brow[1] = n * 2 * SUB + SUB;
+      tl.epi = EPI_STORE;
+      tl.ocol = n * 2 * SUB;
+    }
+  }
+  return tl;
+}
+
+template <int MODE>
+__device__ __forceinline__ int k_blocks(const Params& p) {
+  return MODE == FINAL ? p.S * p.kb0 + p.kb1 : p.kb0;
+}
+
+__device__ __forceinline__ const CUtensorMap* bmap_ptr(const Params& p, int i) {
+  return i == 0 ? &p.tmB0 : i == 1 ? &p.tmB1 : i == 2 ? &p.tmB2 : &p.tmB3;
+}
+
+// ------------------------------------------------------------- producer
+template <int MODE>
+__device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t* full,
+                                        uint64_t* empty, volatile int* abort_flag) {
+  int stage = 0;
+  uint32_t phase = 0;
+  int issued_parity[STAGES];
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+  const int total = total_tiles<MODE>(p);
+  const int nkb = k_blocks<MODE>(p);
+  bool ok = true;
+  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    const Tile tl = decode_tile<MODE>(p, t);
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      const uint32_t a_dst = smem_u32(ring + stage * STAGE_BYTES);
+      const uint32_t b_dst = a_dst + A_BYTES;
+      const uint32_t bar = smem_u32(&full[stage]);
+      mbar_expect_tx(bar, A_BYTES + tl.n_sub * SUB_BYTES);
+      if (MODE == FINAL) {
+        const int kb_sh = p.S * p.kb0;
+        if (kb < kb_sh) {
+          const int j = kb / p.kb0, kk = (kb % p.kb0) * BK;
+          tma_load_2d(a_dst, &p.tmA0, bar, j * p.G + kk, tl.m0);
+          for (int s = 0; s < tl.n_sub; ++s)
+            tma_load_3d(b_dst + s * SUB_BYTES, &p.tmB0, bar, kk, tl.brow[s], j);
+        } else {
+          const int kk = (kb - kb_sh) * BK;
+          tma_load_2d(a_dst, &p.tmA1, bar, kk, tl.m0);
+          for (int s = 0; s < tl.n_sub; ++s)
+            tma_load_2d(b_dst + s * SUB_BYTES, &p.tmB1, bar, kk, tl.brow[s]);
+        }
+      } else {
+        const int kk = kb * BK;
+        tma_load_2d(a_dst, &p.tmA0, bar, kk, tl.m0);
+        for (int s = 0; s < tl.n_sub; ++s) {
+          const int m = tl.bmap[s];
+          if (MODE == XPASS && m < 2)
+            tma_load_2d(b_dst + s * SUB_BYTES, bmap_ptr(p, m), bar, kk, tl.brow[s]);
+          else
+            tma_load_3d(b_dst + s * SUB_BYTES, bmap_ptr(p, m), bar, kk, tl.brow[s], tl.bz[s]);
+        }
+      }
+      issued_parity[stage] = (int)phase;
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  // drain: every load this thread issued has landed before the CTA exits
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s)
+    if (issued_parity[s] >= 0) {
+      volatile int no_abort = 0;
+      mbar_wait(smem_u32(&full[s]), (uint32_t)issued_parity[s], &no_abort, p.status);
+    }
+}
+
+// ------------------------------------------------------------ MMA issuer
+template <int MODE>
+__device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64_t* full,
+                                          uint64_t* empty, uint64_t* tfull, uint64_t* tempty,
+                                          uint64_t* drain, uint32_t tmem, volatile int* abort_flag) {
+  int stage = 0;
+  uint32_t phase = 0;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  const int total = total_tiles<MODE>(p);
+  const int nkb = k_blocks<MODE>(p);
+  bool ok = true;
+  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    const Tile tl = decode_tile<MODE>(p, t);
+    const uint32_t idesc = instr_desc(tl.n_sub * SUB);
+    if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.status)) break;
+    tc_fence_after();
+    const uint32_t d_tmem = tmem + acc * ACC_COLS;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a_addr = smem_u32(ring + stage * STAGE_BYTES);
+      const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+      for (int k = 0; k < BK / 16; ++k) {
+        tc_mma(d_tmem, smem_desc(a_addr + k * 32), smem_desc(b_addr + k * 32), idesc,
+               (kb > 0 || k > 0) ? 1u : 0u);
+      }
+      tc_commit(smem_u32(&empty[stage]));
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    if (!ok) break;
+    tc_commit(smem_u32(&tfull[acc]));
+    if (++acc == 2) {
+      acc = 0;
+      acc_phase ^= 1u;
+    }
+  }
+  // drain: all MMAs this thread issued are complete before TMEM is freed
+  tc_commit(smem_u32(drain));
+  volatile int no_abort = 0;
+  mbar_wait(smem_u32(drain), 0, &no_abort, p.status);
+}
+
+// ------------------------------------------------------------- epilogue
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32], int valid) {
+  // valid: number of leading columns to write (multiple of 8)
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    if (g * 8 < valid) {
+      uint4 w;
+      w.x = pack_bf16(v[g * 8 + 0], v[g * 8 + 1]);
+      w.y = pack_bf16(v[g * 8 + 2], v[g * 8 + 3]);
+      w.z = pack_bf16(v[g * 8 + 4], v[g * 8 + 5]);
+      w.w = pack_bf16(v[g * 8 + 6], v[g * 8 + 7]);
+      reinterpret_cast<uint4*>(dst)[g] = w;
+    }
+  }
+}
+
+template <int MODE>
+__device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint64_t* tempty,
+                                         uint32_t tmem, volatile int* abort_flag) {
+  const int ew = (threadIdx.x >> 5) & 3;  // TMEM lane quarter this warp may access
+  const int lane = threadIdx.x & 31;
+  const int r = ew * 32 + lane;           // tile row of this thread
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  const int total = total_tiles<MODE>(p);
+  for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    const Tile tl = decode_tile<MODE>(p, t);
+    if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.status)) break;
+    tc_fence_after();
+    const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * ACC_COLS;
+    const bool row_ok = r < tl.rows;
+    const int64_t grow = (int64_t)tl.m0 + r;
+    if (tl.epi == EPI_SITU) {
+      // columns [0,128) hold gate pre-activations, [128,256) the matching up ones
+      int width;
+      __nv_bfloat16* out;
+      int64_t ld;
+      if (MODE == XPASS) {
+        width = p.G - (tl.ocol - (tl.ocol / p.G) * p.G);  // hidden units left in this expert
+        out = static_cast<__nv_bfloat16*>(p.out2);
+        ld = p.ld2;
+      } else {
+        width = p.F - tl.ocol;
+        out = static_cast<__nv_bfloat16*>(p.out0);
+        ld = p.ld0;
+      }
+#pragma unroll 1
+      for (int c = 0; c < SUB / 32; ++c) {
+        float g[32], u[32];
+        tc_ld32(tbase + c * 32, g);
+        tc_ld32(tbase + SUB + c * 32, u);
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) g[i] = situ_fast(g[i], u[i], p);
+          store_bf16x32(out + grow * ld + tl.ocol + c * 32, g, width - c * 32);
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int s = 0; s < tl.n_sub; ++s) {
+#pragma unroll 1
+        for (int c = 0; c < SUB / 32; ++c) {
+          float v[32];
+          tc_ld32(tbase + s * SUB + c * 32, v);
+          if (!row_ok) continue;
+          if (MODE == XPASS) {
+            if (tl.bmap[s] == 0) {  // z columns
+              const int col = tl.brow[s] + c * 32;
+              store_bf16x32(static_cast<__nv_bfloat16*>(p.out0) + grow * p.ld0 + col, v, p.L - col);
+            } else {                // router logits, fp32
+              const int col = tl.brow[s] + c * 32;
+              float* dst = static_cast<float*>(p.out1) + grow * p.ld1 + col;
+#pragma unroll
+              for (int g4 = 0; g4 < 8; ++g4)
+                if (col + g4 * 4 < p.R)
+                  reinterpret_cast<float4*>(dst)[g4] =
+                      make_float4(v[g4 * 4], v[g4 * 4 + 1], v[g4 * 4 + 2], v[g4 * 4 + 3]);
+            }
+          } else {
+            const int col = tl.ocol + s * SUB + c * 32;
+            const int width = (MODE == FINAL ? p.d : p.L) - col;
+            store_bf16x32(static_cast<__nv_bfloat16*>(p.out0) + grow * p.ld0 + col, v, width);
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+    if (++acc == 2) {
+      acc = 0;
+      acc_phase ^= 1u;
+    }
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull[a]), 1);
+      mbar_init(smem_u32(&tempty[a]), 4);
+    }
+    mbar_init(smem_u32(&drain), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    if ((threadIdx.x & 31) == 0) produce<MODE>(p, ring, full, empty, &abort_flag);
+  } else if (warp == 1) {
+    if ((threadIdx.x & 31) == 0)
+      mma_issue<MODE>(p, ring, full, empty, tfull, tempty, &drain, tmem, &abort_flag);
+  } else {
+    epilogue<MODE>(p, tfull, tempty, tmem, &abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// bf16 tensor [dim2][dim1][dim0] (dim0 contiguous) with a box of 64 x rows
+// (x 1), 128-byte swizzle, zero fill outside the tensor.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                     uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr || dim0 == 0 || dim1 == 0 || dim2 == 0) return false;
+  cuuint64_t dims[3] = {dim0, dim1, dim2};
+  cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
+  cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint32_t rank = dim2 > 1 ? 3 : 2;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+// Always 3D maps for expert-stacked weights (so the kernel can pass 3 coordinates).
+static bool make_map3(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                      uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr || dim0 == 0 || dim1 == 0 || dim2 == 0) return false;
+  cuuint64_t dims[3] = {dim0, dim1, dim2};
+  cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
+  cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int MODE>
+static cudaError_t launch(const Params& p, int grid, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(umma_gemm_kernel<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  if (grid <= 0) return cudaSuccess;
+  umma_gemm_kernel<MODE><<<grid, THREADS, SMEM_BYTES, st>>>(p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+static Params base_params(int32_t* status) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.status = status;
+  return p;
+}
+
+}  // namespace
+
+cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
+  if (a.N == 0) return cudaSuccess;
+  Params p = base_params(status);
+  bool ok = make_map(&p.tmA0, a.x, a.d, a.N, 1, BM) &&
+            (a.L == 0 || make_map(&p.tmB0, a.w_down, a.d, a.L, 1, SUB)) &&
+            (a.R == 0 || make_map(&p.tmB1, a.w_router, a.d, a.R, 1, SUB));
+  if (a.S > 0)
+    ok = ok && make_map3(&p.tmB2, a.ws_g, a.d, a.G, a.S, SUB) &&
+         make_map3(&p.tmB3, a.ws_u, a.d, a.G, a.S, SUB);
+  if (!ok) return cudaErrorInvalidValue;
+  p.M = (int)a.N;
+  p.kb0 = (a.d + BK - 1) / BK;
+  p.L = a.L;
+  p.R = a.R;
+  p.S = a.S;
+  p.G = a.G;
+  p.d = a.d;
+  p.nz_sub = (a.L + SUB - 1) / SUB;
+  p.nr_sub = (a.R + SUB - 1) / SUB;
+  p.n_zr_tiles = (p.nz_sub + p.nr_sub + 1) / 2;
+  p.g_blocks = a.S > 0 ? (a.G + SUB - 1) / SUB : 0;
+  p.n_tiles = p.n_zr_tiles + a.S * p.g_blocks;
+  p.out0 = a.z;
+  p.ld0 = a.L;
+  p.out1 = a.logits;
+  p.ld1 = a.logits_ld;
+  p.out2 = a.hsh;
+  p.ld2 = (int64_t)a.S * a.G;
+  p.beta1 = a.beta1;
+  p.beta2 = a.beta2;
+  p.inv_beta1 = 1.0f / a.beta1;
+  p.inv_beta2 = 1.0f / a.beta2;
+  const int total = (int)((a.N + BM - 1) / BM) * p.n_tiles;
+  return launch<XPASS>(p, std::min(total, num_sms()), st);
+}
+
+cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
+  if (a.N == 0) return cudaSuccess;
+  Params p = base_params(status);
+  bool ok = make_map(&p.tmA1, a.uhat, a.L, a.N, 1, BM) && make_map(&p.tmB1, a.w_up, a.L, a.d, 1, SUB);
+  if (a.S > 0)
+    ok = ok && make_map(&p.tmA0, a.hsh, (uint64_t)a.S * a.G, a.N, 1, BM) &&
+         make_map3(&p.tmB0, a.ws_o, a.G, a.d, a.S, SUB);
+  if (!ok) return cudaErrorInvalidValue;
+  p.M = (int)a.N;
+  p.S = a.S;
+  p.G = a.G;
+  p.kb0 = a.S > 0 ? (a.G + BK - 1) / BK : 0;
+  p.kb1 = (a.L + BK - 1) / BK;
+  p.L = a.L;
+  p.d = a.d;
+  p.n_tiles = (a.d + 2 * SUB - 1) / (2 * SUB);
+  p.out0 = a.y;
+  p.ld0 = a.d;
+  const int total = (int)((a.N + BM - 1) / BM) * p.n_tiles;
+  return launch<FINAL>(p, std::min(total, num_sms()), st);
+}
+
+cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) {
+  if (a.P == 0) return cudaSuccess;
+  Params p = base_params(status);
+  bool ok = make_map(&p.tmA0, a.a, a.L, a.P, 1, BM) && make_map3(&p.tmB0, a.w0, a.L, a.F, a.R, SUB) &&
+            make_map3(&p.tmB1, a.w1, a.L, a.F, a.R, SUB);
+  if (!ok) return cudaErrorInvalidValue;
+  p.kb0 = (a.L + BK - 1) / BK;
+  p.L = a.L;
+  p.F = a.F;
+  p.R = a.R;
+  p.n_tiles = (a.F + SUB - 1) / SUB;
+  p.out0 = a.out;
+  p.ld0 = a.F;
+  p.tiles = a.tiles;
+  p.n_mtiles = a.n_mtiles;
+  p.beta1 = a.beta1;
+  p.beta2 = a.beta2;
+  p.inv_beta1 = 1.0f / a.beta1;
+  p.inv_beta2 = 1.0f / a.beta2;
+  const int64_t bound = (int64_t)a.max_tiles * p.n_tiles;
+  return launch<ROUTED1>(p, (int)std::min<int64_t>(bound, num_sms()), st);
+}
+
+cudaError_t umma_routed2(const RoutedArgs& a, int32_t* status, cudaStream_t st) {
+  if (a.P == 0) return cudaSuccess;
+  Params p = base_params(status);
+  bool ok = make_map(&p.tmA0, a.a, a.F, a.P, 1, BM) && make_map3(&p.tmB0, a.w0, a.F, a.L, a.R, SUB);
+  if (!ok) return cudaErrorInvalidValue;
+  p.kb0 = (a.F + BK - 1) / BK;
+  p.L = a.L;
+  p.F = a.F;
+  p.R = a.R;
+  p.n_tiles = (a.L + 2 * SUB - 1) / (2 * SUB);
+  p.out0 = a.out;
+  p.ld0 = a.L;
+  p.tiles = a.tiles;
+  p.n_mtiles = a.n_mtiles;
+  const int64_t bound = (int64_t)a.max_tiles * p.n_tiles;
+  return launch<ROUTED2>(p, (int)std::min<int64_t>(bound, num_sms()), st);
+}
+
+}  // namespace lmoe

@@ -1,0 +1,65 @@
+// Host interface of the tcgen05 (5th-generation tensor core) GEMM engine.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lmoe {
+
+// x-pass: one pass over x [N, d] computes
+//   z      [N, L]  bf16 = x W_down^T
+//   logits [N, R]  fp32 = x W_r^T          (row stride logits_ld)
+//   hsh    [N, S*G] bf16 = SiTU(x W_g,sh^T, x W_u,sh^T) per shared expert
+struct XpassArgs {
+  const __nv_bfloat16* x;
+  int64_t N;
+  int d;
+  const __nv_bfloat16* w_down;  // [L, d]
+  int L;
+  const __nv_bfloat16* w_router;  // [R, d]
+  int R;
+  const __nv_bfloat16* ws_g;  // [S, G, d]
+  const __nv_bfloat16* ws_u;
+  int S, G;
+  __nv_bfloat16* z;
+  float* logits;
+  int64_t logits_ld;
+  __nv_bfloat16* hsh;
+  float beta1, beta2;
+};
+
+// final: y [N, d] = sum_j hsh[:, jG:(j+1)G] W_o,sh_j^T + uhat W_up^T
+struct FinalArgs {
+  const __nv_bfloat16* hsh;  // [N, S*G]
+  int64_t N;
+  int S, G;
+  const __nv_bfloat16* ws_o;  // [S, d, G]
+  int d;
+  const __nv_bfloat16* uhat;  // [N, L]
+  int L;
+  const __nv_bfloat16* w_up;  // [d, L]
+  __nv_bfloat16* y;
+};
+
+// routed GEMM1: h [P, F] = SiTU(zp W_g,e^T, zp W_u,e^T) per row tile of expert e
+// routed GEMM2: eo [P, L] = h W_o,e^T
+struct RoutedArgs {
+  const __nv_bfloat16* a;  // zp [P, L] (gemm1) or h [P, F] (gemm2)
+  int64_t P;
+  int L, F, R;
+  const __nv_bfloat16* w0;  // gemm1: w_g [R, F, L]; gemm2: w_o [R, L, F]
+  const __nv_bfloat16* w1;  // gemm1: w_u [R, F, L]
+  __nv_bfloat16* out;       // gemm1: h; gemm2: eo
+  const int4* tiles;        // routed row tiles (expert, first row, rows)
+  const int32_t* n_mtiles;
+  int max_tiles;
+  float beta1, beta2;
+};
+
+cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st);
+cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st);
+cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st);
+cudaError_t umma_routed2(const RoutedArgs& a, int32_t* status, cudaStream_t st);
+
+}  // namespace lmoe

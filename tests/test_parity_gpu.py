@@ -229,10 +229,40 @@ def test_forward_edge_cases(label, over, base):
 
 
 def test_forward_saturated_situ():
-    """Weights of std 1: SiTU gates and ups run deep into saturation."""
+    """Expert weights of std 1: SiTU gates and ups run deep into saturation (the
+    router keeps std 0.02 so that its top-k stays well separated)."""
+    from oracle.conditioning import enforce_topk_margin
     wl = W["halfb_uniform"].with_tokens(160).replace(w_std=1.0)
-    inp = prepare(wl)
+    inp = synth.make_inputs(wl)
+    inp["w_router"] = synth.normal(0, "w_router", (wl.n_routed, wl.d), 0.02)
+    enforce_topk_margin(wl, inp)
     y, ids, probs, _, _ = _run_forward(wl, device_inputs(inp))
+    _compare_forward(wl, inp, y, ids, probs)
+
+
+@pytest.mark.parametrize("name,n", [("halfb_uniform", 300), ("mid", 136), ("k3_width", 24)])
+def test_forward_intermediates(name, n):
+    """Each stage of the forward against the oracle: z, router logits, shared
+    hidden units, RMSNorm(u), then y."""
+    wl = W[name].with_tokens(n)
+    inp = prepare(wl)
+    dev = device_inputs(inp)
+    y, ids, probs, _, ws = _run_forward(wl, dev)
+    v = lm.workspace_views(ldims(wl), ws)
+    ow = oracle_weights(inp)
+    x = synth.to_f32(inp["x"]).astype(np.float64)
+    ref = oracle.forward(odims(wl), ow, synth.to_f32(inp["x"]), want=("z", "uhat"))
+    assert rel_err(host(v["z"]), ref["z"]) <= 1e-2, "z"
+    logits = x @ ow["w_router"].astype(np.float64).T
+    assert rel_err(host(v["logits"]), logits) <= 1e-5, "router logits"
+    if wl.n_shared:
+        hs = np.empty((n, wl.n_shared * wl.ff_shared))
+        for t in range(n):
+            for j in range(wl.n_shared):
+                hs[t, j * wl.ff_shared:(j + 1) * wl.ff_shared] = oracle.situ(
+                    ow["ws_g"][j], ow["ws_u"][j], ow["ws_o"][j], x[t], wl.beta1, wl.beta2)[1]
+        assert rel_err(host(v["hsh"]), hs) <= 2e-2, "shared hidden"
+    assert rel_err(host(v["uhat"]), ref["uhat"]) <= 2e-2, "uhat"
     _compare_forward(wl, inp, y, ids, probs)
 
 
