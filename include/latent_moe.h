@@ -174,6 +174,27 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
  * offsets[7] = ld, the row stride (elements) of the logits. */
 LMOE_API lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offsets, int32_t n);
 
+/* moe_dispatch without a workspace: the same permutation, bit for bit, for
+ * callers that cannot provide device scratch memory -- for example a plugin
+ * host that gives a kernel only its tensors, a memory pool that is capped and
+ * full, or a thread that must not enter the device allocator.  The pages have
+ * no counterpart; it exists for such callers.
+ *   The sort's scratch (per-block histograms, routed tile list, status word)
+ *   is one fixed 1 MiB array in device memory, defined by the library; every
+ *   GPU that loads the library holds it until the process exits.  The call
+ *   allocates nothing.  Sizes whose scratch exceeds the array --
+ *   4 * (64 + ceil(N*k / 4096) * R rounded up to a multiple of 4
+ *   + 4 * (N*k/128 + R + 1)) bytes > 1 MiB --
+ *   return LMOE_EUNSUPPORTED with a message, before any launch.
+ *   The first call on a device looks the array's address up (make it before
+ *   any stream capture).  All calls share the array and it keeps the last
+ *   call's contents, so calls that overlap on the GPU race: serialise them.
+ *   Out-of-range ids are dropped as in moe_dispatch but not reported.
+ * Arguments and outputs as in moe_dispatch. */
+LMOE_API lmoe_status moe_dispatch_noalloc(const lmoe_dims* dims, const int32_t* ids,
+                                          int32_t* counts, int32_t* offsets, int32_t* perm_token,
+                                          int32_t* inv_pair, lmoe_stream stream);
+
 /* Zeroes the workspace header (status word and scheduling counters).  Call
  * once on a new workspace before its first use. */
 LMOE_API lmoe_status lmoe_workspace_init(void* ws, size_t ws_bytes, lmoe_stream stream);

@@ -60,6 +60,7 @@ _sigs = {
     "lmoe_workspace_size_host": (ctypes.c_size_t, [_DP]),
     "moe_route": (_S, [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_dispatch": (_S, [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_dispatch_noalloc": (_S, [_DP, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn": (_S, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (_S, [_DP, _P, _P, _P, _P, _P, _P]),
     "latent_moe_forward": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, _P, _P, _P, _P,
@@ -162,6 +163,14 @@ def moe_dispatch(dims, ids, counts, offsets, perm_token, inv_pair, ws, stream=No
     _check(_lib.moe_dispatch(ctypes.byref(dims), _ptr(ids), _ptr(counts), _ptr(offsets),
                              _ptr(perm_token), _ptr(inv_pair), _ptr(ws), ws.numel(),
                              _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_noalloc(dims, ids, counts, offsets, perm_token, inv_pair, stream=None):
+    """moe_dispatch for callers that cannot provide a workspace (the library's
+    fixed device scratch array is used; calls must not overlap on the GPU)."""
+    _check(_lib.moe_dispatch_noalloc(ctypes.byref(dims), _ptr(ids), _ptr(counts), _ptr(offsets),
+                                     _ptr(perm_token), _ptr(inv_pair), _stream(stream)),
+           "moe_dispatch_noalloc")
 
 
 def moe_expert_ffn(dims, z, perm_token, offsets, w_g, w_u, w_o, expert_out, ws, stream=None):

@@ -18,6 +18,7 @@ static thread_local std::string g_last_error;
 static thread_local uint64_t g_launches = 0;
 
 void count_launch(int n) { g_launches += (uint64_t)n; }
+void set_last_error(const char* msg) { g_last_error = msg; }
 
 // --------------------------------------------------------------- profiling
 // Optional CUDA-event brackets around the launches of one named kernel, on the

@@ -74,5 +74,7 @@ cudaError_t launch_capped_wait(int32_t* flag, int32_t* status, int cap_ms, cudaS
 
 // Launch counter (api.cu)
 void count_launch(int n = 1);
+// Sets the per-thread message returned by lmoe_last_error (api.cu).
+void set_last_error(const char* msg);
 
 }  // namespace lmoe
