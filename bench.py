@@ -292,13 +292,28 @@ def main():
     clk = clocks.stop()
     launches = lm.launch_count()
     lm.profile_enable(None)
-    k_ms, k_n = lm.profile_read()
+    k_ms, k_n = lm.profile_read(prof_tag)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
     value = world * wl.n_tokens / (ms_per_step / 1e3)
     if lm.get_device_status(ws) != lm.OK:
         raise SystemExit("device status not OK after the timed region")
+
+    # per-kernel breakdown (a separate pass with every kernel bracketed by events)
+    lm.profile_enable("*")
+    for _ in range(min(args.steps, 20)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    lm.profile_enable(None)
+    breakdown = {}
+    for tag in ("xpass", "route", "dispatch", "gather", "expert_gemm1", "expert_gemm2", "combine",
+                "final"):
+        ms, n = lm.profile_read(tag)
+        if n:
+            breakdown[tag] = round(ms / min(args.steps, 20) * 1e3, 2)
+    lm.profile_read()
 
     # end to end through the host entry point: pinned x in, y out, copies timed
     ws_h = lm.alloc_workspace(dims, device=dev, host=True)
@@ -353,6 +368,7 @@ def main():
         "e2e": {"value": world * wl.n_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
         "gpu_launches": launches,
+        "kernel_us": breakdown,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.seed)

@@ -183,9 +183,9 @@ LMOE_API lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offset
  *   is one fixed 1 MiB array in device memory, defined by the library; every
  *   GPU that loads the library holds it until the process exits.  The call
  *   allocates nothing.  Sizes whose scratch exceeds the array --
- *   4 * (64 + ceil(N*k / 4096) * R rounded up to a multiple of 4
- *   + 4 * (N*k/128 + R + 1)) bytes > 1 MiB --
- *   return LMOE_EUNSUPPORTED with a message, before any launch.
+ *   4 * (64 + C * R rounded up to a multiple of 4 + 4 * (N*k/128 + R + 1))
+ *   bytes > 1 MiB, C <= 128 the number of chunks the sort splits the pairs
+ *   into -- return LMOE_EUNSUPPORTED with a message, before any launch.
  *   The first call on a device looks the array's address up (make it before
  *   any stream capture).  All calls share the array and it keeps the last
  *   call's contents, so calls that overlap on the GPU race: serialise them.
@@ -215,12 +215,15 @@ LMOE_API const char* lmoe_status_string(lmoe_status status);
 /* Last error message of this thread (empty string if none). */
 LMOE_API const char* lmoe_last_error(void);
 
-/* Brackets every launch of the kernel named `tag` (NULL or "" turns it off)
- * with CUDA events on its stream.  Tags: "xpass", "route", "dispatch",
- * "gather", "expert_gemm1", "expert_gemm2", "combine", "final". */
-LMOE_API lmoe_status lmoe_profile_enable(const char* tag);
-/* Waits for the recorded events; returns the summed device time (ms) and the
- * number of bracketed launches since the last read, then clears them. */
+/* Brackets every launch of the kernels named in `tags` (a comma-separated
+ * list, "*" for all, NULL or "" to turn it off) with CUDA events on their
+ * stream.  Tags: "xpass", "route", "dispatch", "gather", "expert_gemm1",
+ * "expert_gemm2", "combine", "final". */
+LMOE_API lmoe_status lmoe_profile_enable(const char* tags);
+/* Waits for the recorded events of kernel `tag` (NULL: every tag); returns the
+ * summed device time (ms) and the number of bracketed launches since the last
+ * read of that tag, and clears them. */
+LMOE_API lmoe_status lmoe_profile_read_tag(const char* tag, double* total_ms, int64_t* launches);
 LMOE_API lmoe_status lmoe_profile_read(double* total_ms, int64_t* launches);
 
 /* Number of kernel launches the library issued on this thread since the last

@@ -76,6 +76,8 @@ _sigs = {
     "lmoe_profile_enable": (_S, [ctypes.c_char_p]),
     "lmoe_workspace_layout": (_S, [_DP, ctypes.POINTER(ctypes.c_size_t), ctypes.c_int32]),
     "lmoe_profile_read": (_S, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
+    "lmoe_profile_read_tag": (_S, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
+                                   ctypes.POINTER(ctypes.c_int64)]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -213,15 +215,17 @@ def launch_count(reset: bool = False) -> int:
     return _lib.lmoe_launch_count(1 if reset else 0)
 
 
-def profile_enable(tag):
-    """Brackets every launch of kernel ``tag`` with CUDA events (None: off)."""
-    _check(_lib.lmoe_profile_enable(None if tag is None else tag.encode()), "lmoe_profile_enable")
+def profile_enable(tags):
+    """Brackets every launch of the kernels in ``tags`` ("a,b", "*" or None: off)."""
+    _check(_lib.lmoe_profile_enable(None if tags is None else tags.encode()), "lmoe_profile_enable")
 
 
-def profile_read():
-    """(summed device ms, launches) of the bracketed kernel since the last read."""
+def profile_read(tag=None):
+    """(summed device ms, launches) of the bracketed kernel ``tag`` (None: all)
+    since the last read."""
     ms, n = ctypes.c_double(), ctypes.c_int64()
-    _check(_lib.lmoe_profile_read(ctypes.byref(ms), ctypes.byref(n)), "lmoe_profile_read")
+    _check(_lib.lmoe_profile_read_tag(None if tag is None else tag.encode(), ctypes.byref(ms),
+                                      ctypes.byref(n)), "lmoe_profile_read_tag")
     return ms.value, n.value
 
 

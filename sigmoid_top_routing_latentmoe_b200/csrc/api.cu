@@ -21,20 +21,28 @@ void count_launch(int n) { g_launches += (uint64_t)n; }
 void set_last_error(const char* msg) { g_last_error = msg; }
 
 // --------------------------------------------------------------- profiling
-// Optional CUDA-event brackets around the launches of one named kernel, on the
-// stream they are launched on.  Off unless lmoe_profile_enable names a tag.
+// Optional CUDA-event brackets around the launches of named kernels, on the
+// stream they are launched on.  Off unless lmoe_profile_enable names tags.
 struct ProfRec {
+  std::string tag;
   cudaEvent_t a, b;
 };
-static thread_local std::string g_prof_tag;
+static thread_local std::string g_prof_tags;  // "" off, "*" all, else ",tag1,tag2,"
 static thread_local std::vector<ProfRec> g_prof;
+
+static bool prof_wanted(const char* tag) {
+  if (g_prof_tags.empty()) return false;
+  if (g_prof_tags == "*") return true;
+  return g_prof_tags.find("," + std::string(tag) + ",") != std::string::npos;
+}
 
 struct ProfScope {
   bool on = false;
   cudaStream_t st;
   ProfRec r{};
   ProfScope(const char* tag, cudaStream_t s) : st(s) {
-    if (g_prof_tag.empty() || g_prof_tag != tag) return;
+    if (!prof_wanted(tag)) return;
+    r.tag = tag;
     if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) return;
     on = cudaEventRecord(r.a, st) == cudaSuccess;
   }
@@ -210,18 +218,21 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
   return LMOE_OK;
 }
 
+// z != nullptr: also writes the sorted rows of z to the workspace (the A
+// operand of the routed GEMMs).
 static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t* counts,
                                 int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
-                                cudaStream_t st) {
+                                cudaStream_t st, const void* z = nullptr) {
   const Layout L = layout(d, false);
   DispatchScratch s;
   s.block_counts = at<int32_t>(ws, L.block_counts);
   s.status = &at<WsHeader>(ws, L.header)->status;
   s.n_mtiles = &at<WsHeader>(ws, L.header)->n_mtiles;
   s.tiles = at<int4>(ws, L.tiles);
+  const int es = d->dtype == LMOE_BF16 ? 2 : 4;
   ProfScope ps("dispatch", st);
-  LMOE_CUDA(launch_dispatch(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm, inv, s,
-                            st),
+  LMOE_CUDA(launch_dispatch_gather(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm,
+                                   inv, s, z, z ? at<char>(ws, L.zp) : nullptr, d->latent * es, st),
             "dispatch");
   return LMOE_OK;
 }
@@ -230,7 +241,7 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
 template <typename T>
 static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32_t* perm,
                                   const void* w_g, const void* w_u, const void* w_o, void* eo,
-                                  void* ws, cudaStream_t st) {
+                                  void* ws, cudaStream_t st, bool rows_sorted = false) {
   const Layout L = layout(d, false);
   const int64_t P = d->n_tokens * d->top_k;
   if (P == 0) return LMOE_OK;
@@ -239,7 +250,7 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   T* h = at<T>(ws, L.h);
   const int4* tiles = at<int4>(ws, L.tiles);
   const int32_t* n_tiles = &at<WsHeader>(ws, L.header)->n_mtiles;
-  {
+  if (!rows_sorted) {
     ProfScope ps("gather", st);
     LMOE_CUDA(launch_gather_rows<T>((const T*)z, perm, P, Lt, zp, st), "gather");
   }
@@ -315,6 +326,7 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
     a.ws_g = (const __nv_bfloat16*)w->ws_g; a.ws_u = (const __nv_bfloat16*)w->ws_u; a.S = S; a.G = G;
     a.z = (__nv_bfloat16*)z; a.logits = logits; a.logits_ld = L.logits_ld;
     a.hsh = (__nv_bfloat16*)hsh; a.beta1 = d->beta1; a.beta2 = d->beta2;
+    a.bias = w->expert_bias; a.ids = ids; a.probs = probs; a.top_k = d->top_k;
     ProfScope ps("xpass", st);
     LMOE_CUDA(umma_xpass(a, status, st), "x-pass (tcgen05)");
   } else {
@@ -338,16 +350,18 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
   }
   // step 2: routing (top-k + normalisation from the x-pass logits on the tcgen05 path)
   if (tc) {
-    ProfScope ps("route", st);
-    LMOE_CUDA(launch_route_topk(logits, L.logits_ld, w->expert_bias, N, d->n_routed, d->top_k, ids,
-                                probs, st),
-              "route_topk");
+    if (d->n_routed > 32) {  // R <= 32 is routed inside the x-pass epilogue
+      ProfScope ps("route", st);
+      LMOE_CUDA(launch_route_topk(logits, L.logits_ld, w->expert_bias, N, d->n_routed, d->top_k,
+                                  ids, probs, st),
+                "route_topk");
+    }
   } else {
     LMOE_TRY(run_route<T>(d, x, w->w_router, w->expert_bias, ids, probs, ws, st));
   }
   // step 3: dispatch, routed experts, combine + RMSNorm
-  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st));
-  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st));
+  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, z));
+  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st, true));
   {
     ProfScope ps("combine", st);
     LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, d->top_k, Lt, d->rms_eps, uhat,
@@ -609,15 +623,26 @@ const char* lmoe_status_string(lmoe_status s) {
 
 const char* lmoe_last_error(void) { return g_last_error.c_str(); }
 
-lmoe_status lmoe_profile_enable(const char* tag) {
-  g_prof_tag = tag ? tag : "";
+lmoe_status lmoe_profile_enable(const char* tags) {
+  if (tags == nullptr || tags[0] == 0) {
+    g_prof_tags.clear();
+  } else if (std::string(tags) == "*") {
+    g_prof_tags = "*";
+  } else {
+    g_prof_tags = "," + std::string(tags) + ",";
+  }
   return LMOE_OK;
 }
 
-lmoe_status lmoe_profile_read(double* total_ms, int64_t* launches) {
+lmoe_status lmoe_profile_read_tag(const char* tag, double* total_ms, int64_t* launches) {
   double tot = 0.0;
   int64_t n = 0;
+  std::vector<ProfRec> keep;
   for (auto& r : g_prof) {
+    if (tag != nullptr && r.tag != tag) {
+      keep.push_back(r);
+      continue;
+    }
     float ms = 0.0f;
     LMOE_CUDA(cudaEventSynchronize(r.b), "event sync");
     LMOE_CUDA(cudaEventElapsedTime(&ms, r.a, r.b), "elapsed");
@@ -626,10 +651,14 @@ lmoe_status lmoe_profile_read(double* total_ms, int64_t* launches) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
   }
-  g_prof.clear();
+  g_prof.swap(keep);
   if (total_ms) *total_ms = tot;
   if (launches) *launches = n;
   return LMOE_OK;
+}
+
+lmoe_status lmoe_profile_read(double* total_ms, int64_t* launches) {
+  return lmoe_profile_read_tag(nullptr, total_ms, launches);
 }
 
 uint64_t lmoe_launch_count(int32_t reset) {

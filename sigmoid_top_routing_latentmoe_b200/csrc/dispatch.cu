@@ -1,176 +1,197 @@
 // Pair permutation (kda/layers/latent_moe.py LatentMoE._routed_u; sec-07
 // sparse dispatch, step 1): the N*k (token, expert) pairs, flattened
 // token-major, are stably sorted by expert id -- the pages' argsort(stable) +
-// bincount + cumsum -- as a deterministic three-pass counting sort:
-//   1. per-block histograms of a fixed chunk of pairs,
-//   2. one block scans them (per expert over blocks, then over experts) into
-//      counts, offsets and each block's starting slot per expert, and writes
-//      the routed row-tile list (expert, first row, rows) used by the GEMMs,
-//   3. each block ranks its pairs in pair order inside each expert and
-//      scatters perm_token / inv_pair.
-// No step depends on atomic ordering, so the output is bit-exact.
+// bincount + cumsum -- as a deterministic counting sort over chunks of pairs:
+//   1. hist:    one CTA per chunk counts its pairs per expert,
+//   2. scan:    one CTA turns the chunk counts into each chunk's first slot
+//               per expert, the per-expert counts and offsets, and the routed
+//               row-tile list (expert, first row, rows) the GEMMs walk,
+//   3. scatter: one CTA per chunk ranks its pairs in pair order inside each
+//               expert, writes perm_token / inv_pair and, in the fused
+//               forward, copies each pair's z row to its sorted slot.
+// No result depends on the order of atomic operations: bit-exact.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace lmoe {
 namespace {
 
-constexpr int kChunk = 4096;       // pairs per block
-constexpr int kThreads = 256;      // 8 warps
+constexpr int kThreads = 256;  // 8 warps per chunk
 constexpr int kWarps = kThreads / 32;
-constexpr int kPerWarp = kChunk / kWarps;  // 512 pairs, walked 32 at a time
+constexpr int kMaxChunks = 128;
+
+// Pairs per chunk: at least 256 (one 32-pair step per warp), and large enough
+// that there are at most kMaxChunks chunks.
+int64_t chunk_pairs(int64_t n_pairs) {
+  const int64_t per = (n_pairs + kMaxChunks - 1) / kMaxChunks;
+  const int64_t step = 32 * kWarps;
+  return std::max<int64_t>(step, (per + step - 1) / step * step);
+}
 
 __global__ void __launch_bounds__(kThreads) hist_kernel(const int32_t* __restrict__ ids,
-                                                        int64_t n_pairs, int R,
-                                                        int32_t* __restrict__ block_counts,
+                                                        int64_t n_pairs, int64_t chunk, int R,
+                                                        int32_t* __restrict__ chunk_counts,
                                                         int32_t* __restrict__ status) {
   extern __shared__ int32_t hist[];
   for (int e = threadIdx.x; e < R; e += kThreads) hist[e] = 0;
   __syncthreads();
-  const int64_t base = (int64_t)blockIdx.x * kChunk;
-  for (int j = threadIdx.x; j < kChunk; j += kThreads) {
-    int64_t p = base + j;
-    if (p < n_pairs) {
-      int e = ids[p];
-      if ((unsigned)e < (unsigned)R)
-        atomicAdd(&hist[e], 1);
-      else
-        record_status(status, kStatusDevice);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t per_warp = chunk / kWarps;
+  const int64_t p0 = (int64_t)blockIdx.x * chunk + warp * per_warp;
+  const int64_t p1 = min(n_pairs, p0 + per_warp);
+  for (int64_t q = p0; q < p1; q += 32) {
+    const int64_t p = q + lane;
+    int e = p < p1 ? ids[p] : -1;
+    if (p < p1 && (unsigned)e >= (unsigned)R) {
+      record_status(status, kStatusDevice);
+      e = -1;
     }
+    // one shared-memory add per distinct expert among the warp's 32 pairs
+    const unsigned same = __match_any_sync(0xffffffffu, e < 0 ? -1 - lane : e);
+    if (e >= 0 && (same & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[e], __popc(same));
   }
   __syncthreads();
   for (int e = threadIdx.x; e < R; e += kThreads)
-    block_counts[(int64_t)blockIdx.x * R + e] = hist[e];
+    chunk_counts[(int64_t)blockIdx.x * R + e] = hist[e];
 }
 
-// Single block.  block_counts[b, e] becomes the first sorted slot of block b's
-// pairs of expert e.
-__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_counts,
-                                                    int n_blocks, int R, int32_t* __restrict__ counts,
+// Block-wide exclusive scan of one value per thread; *total gets the sum.
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_sums,
+                                                        int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int32_t inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int32_t o = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += o;
+  }
+  if (lane == 31) warp_sums[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t ws = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int32_t o = __shfl_up_sync(0xffffffffu, ws, off);
+      if (lane >= off) ws += o;
+    }
+    if (lane < nw) warp_sums[lane] = ws;
+    if (lane == nw - 1) *total = ws;
+  }
+  __syncthreads();
+  const int32_t excl = inc - v + (warp > 0 ? warp_sums[warp - 1] : 0);
+  __syncthreads();
+  return excl;
+}
+
+// One CTA of 1024 threads.  chunk_counts[c, e] becomes the number of pairs of
+// expert e in chunks before c.
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_counts,
+                                                    int n_chunks, int R,
+                                                    int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ n_mtiles,
                                                     int4* __restrict__ tiles) {
-  extern __shared__ int32_t sm[];  // [R] counts, then [R] tile starts
-  int32_t* cnt = sm;
-  int32_t* tstart = sm + R;
   __shared__ int32_t warp_sums[32];
+  __shared__ int32_t totals[2];
   __shared__ int32_t carry[2];
-  // per-expert exclusive scan over blocks
-  for (int e = threadIdx.x; e < R; e += blockDim.x) {
-    int32_t run = 0;
-    for (int b = 0; b < n_blocks; ++b) {
-      int32_t c = block_counts[(int64_t)b * R + e];
-      block_counts[(int64_t)b * R + e] = run;
-      run += c;
-    }
-    cnt[e] = run;
-  }
-  if (threadIdx.x == 0) { carry[0] = 0; carry[1] = 0; }
-  __syncthreads();
-  // exclusive scan over experts of counts (-> offsets) and of tile counts
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (threadIdx.x == 0) carry[0] = carry[1] = 0;
   for (int base = 0; base < R; base += blockDim.x) {
-    int e = base + threadIdx.x;
-    int32_t c = (e < R) ? cnt[e] : 0;
-    int32_t nt = (c + kTileM - 1) / kTileM;
-    // scan pair counts
-    for (int pass = 0; pass < 2; ++pass) {
-      int32_t v = pass == 0 ? c : nt;
-      int32_t inc = v;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        int32_t o = __shfl_up_sync(0xffffffffu, inc, off);
-        if (lane >= off) inc += o;
+    const int e = base + threadIdx.x;
+    int32_t c = 0;
+    if (e < R) {
+      for (int b = 0; b < n_chunks; ++b) {
+        const int32_t v = chunk_counts[(int64_t)b * R + e];
+        chunk_counts[(int64_t)b * R + e] = c;
+        c += v;
       }
-      if (lane == 31) warp_sums[warp] = inc;
-      __syncthreads();
-      if (warp == 0) {
-        int32_t ws = lane < nw ? warp_sums[lane] : 0;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          int32_t o = __shfl_up_sync(0xffffffffu, ws, off);
-          if (lane >= off) ws += o;
-        }
-        if (lane < nw) warp_sums[lane] = ws;  // inclusive over warps
-      }
-      __syncthreads();
-      int32_t excl = inc - v + (warp > 0 ? warp_sums[warp - 1] : 0) + carry[pass];
-      if (e < R) {
-        if (pass == 0) {
-          offsets[e] = excl;
-          counts[e] = c;
-        } else {
-          tstart[e] = excl;
-        }
-      }
-      __syncthreads();
-      if (threadIdx.x == blockDim.x - 1) carry[pass] = excl + v;
-      __syncthreads();
     }
+    __syncthreads();
+    const int32_t nt = (c + kTileM - 1) / kTileM;
+    const int32_t ex_c = block_exclusive_scan(c, warp_sums, &totals[0]) + carry[0];
+    const int32_t ex_t = block_exclusive_scan(nt, warp_sums, &totals[1]) + carry[1];
+    if (e < R) {
+      counts[e] = c;
+      offsets[e] = ex_c;
+      for (int j = 0; j * kTileM < c; ++j)
+        tiles[ex_t + j] = make_int4(e, ex_c + j * kTileM, min(kTileM, c - j * kTileM), 0);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      carry[0] += totals[0];
+      carry[1] += totals[1];
+    }
+    __syncthreads();
   }
   if (threadIdx.x == 0) {
     offsets[R] = carry[0];
     *n_mtiles = carry[1];
   }
-  __syncthreads();
-  // tile list: expert e owns tiles [tstart[e], tstart[e] + ceil(cnt/128))
-  for (int e = warp; e < R; e += nw) {
-    int32_t c = cnt[e];
-    int32_t nt = (c + kTileM - 1) / kTileM;
-    int32_t off = offsets[e];
-    for (int j = lane; j < nt; j += 32) {
-      int32_t rows = min(kTileM, c - j * kTileM);
-      tiles[tstart[e] + j] = make_int4(e, off + j * kTileM, rows, 0);
-    }
-  }
 }
 
-__global__ void __launch_bounds__(kThreads) scatter_kernel(const int32_t* __restrict__ ids,
-                                                           int64_t n_pairs, int k, int R,
-                                                           const int32_t* __restrict__ block_first,
-                                                           const int32_t* __restrict__ offsets,
-                                                           int32_t* __restrict__ perm_token,
-                                                           int32_t* __restrict__ inv_pair) {
-  extern __shared__ int32_t wcnt[];  // [kWarps][R]: per-warp counts, then running slots
+// Ranks each chunk's pairs inside their expert in pair order and scatters.
+// With z != nullptr it also copies z[token] to row `slot` of zp (row_vecs
+// 16-byte vectors per row).
+__global__ void __launch_bounds__(kThreads) scatter_kernel(
+    const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int k, int R,
+    const int32_t* __restrict__ chunk_first, const int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair, const uint4* __restrict__ z,
+    uint4* __restrict__ zp, int row_vecs) {
+  extern __shared__ int32_t wcnt[];  // [kWarps][R]: per-warp counts, then first slots
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * R; i += kThreads) wcnt[i] = 0;
   __syncthreads();
-  const int64_t base = (int64_t)blockIdx.x * kChunk + (int64_t)warp * kPerWarp;
-  // pass 1: per-warp histogram of its contiguous sub-range
-  for (int j = lane; j < kPerWarp; j += 32) {
-    int64_t p = base + j;
-    if (p < n_pairs) {
-      int e = ids[p];
-      if ((unsigned)e < (unsigned)R) atomicAdd(&wcnt[warp * R + e], 1);
-    }
+  const int64_t per_warp = chunk / kWarps;
+  const int64_t p0 = (int64_t)blockIdx.x * chunk + warp * per_warp;
+  const int64_t p1 = min(n_pairs, p0 + per_warp);
+  int32_t* my = wcnt + warp * R;
+  // pass 1: this warp's counts per expert (only this warp writes its row)
+  for (int64_t q = p0; q < p1; q += 32) {
+    const int64_t p = q + lane;
+    const int e = p < p1 ? ids[p] : -1;
+    const bool valid = (unsigned)e < (unsigned)R;
+    const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1 - lane);
+    if (valid && (same & ((1u << lane) - 1u)) == 0) my[e] += __popc(same);
   }
   __syncthreads();
-  // pass 2: first slot of each warp's pairs of expert e
+  // pass 2: first sorted slot of each warp's pairs of expert e
   for (int e = threadIdx.x; e < R; e += kThreads) {
-    int32_t run = offsets[e] + block_first[(int64_t)blockIdx.x * R + e];
+    int32_t run = offsets[e] + chunk_first[(int64_t)blockIdx.x * R + e];
     for (int w = 0; w < kWarps; ++w) {
-      int32_t c = wcnt[w * R + e];
+      const int32_t c = wcnt[w * R + e];
       wcnt[w * R + e] = run;
       run += c;
     }
   }
   __syncthreads();
-  // pass 3: walk the sub-range in pair order, 32 pairs at a time
-  for (int j0 = 0; j0 < kPerWarp; j0 += 32) {
-    int64_t p = base + j0 + lane;
-    bool valid = p < n_pairs;
-    int e = valid ? ids[p] : -1;
-    valid = valid && (unsigned)e < (unsigned)R;
-    unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1 - lane);
-    unsigned lower = same & ((1u << lane) - 1u);
-    int32_t slot = 0;
-    if (valid) slot = wcnt[warp * R + e] + __popc(lower);
+  // pass 3: walk the warp's pairs in order, 32 at a time
+  for (int64_t q = p0; q < p1; q += 32) {
+    const int64_t p = q + lane;
+    const int e = p < p1 ? ids[p] : -1;
+    const bool valid = (unsigned)e < (unsigned)R;
+    const unsigned same = __match_any_sync(0xffffffffu, valid ? e : -1 - lane);
+    const unsigned lower = same & ((1u << lane) - 1u);
+    int32_t slot = -1;
+    if (valid) slot = my[e] + __popc(lower);
     __syncwarp();
-    if (valid && lower == 0) wcnt[warp * R + e] += __popc(same);
+    if (valid && lower == 0) my[e] += __popc(same);
     __syncwarp();
+    const int32_t tok = (int32_t)((uint32_t)p / (uint32_t)k);  // pairs < 2^31
     if (valid) {
-      perm_token[slot] = (int32_t)(p / k);
+      perm_token[slot] = tok;
       inv_pair[p] = slot;
+    }
+    if (z != nullptr) {
+      // the warp copies its (up to) 32 rows, one row at a time, 16 bytes per lane
+      for (int j = 0; j < 32; ++j) {
+        const int32_t s_j = __shfl_sync(0xffffffffu, slot, j);
+        const int32_t t_j = __shfl_sync(0xffffffffu, tok, j);
+        if (s_j < 0) continue;
+        const uint4* src = z + (int64_t)t_j * row_vecs;
+        uint4* dst = zp + (int64_t)s_j * row_vecs;
+        for (int v = lane; v < row_vecs; v += 32) dst[v] = src[v];
+      }
     }
   }
 }
@@ -207,46 +228,65 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int R,
   int32_t t = inc - mine;
   for (int e = e0; e < e1; ++e) {
     const int32_t off = offsets[e], c = offsets[e + 1] - off;
-    for (int j = 0; j * kTileM < c; ++j) tiles[t++] = make_int4(e, off + j * kTileM, min(kTileM, c - j * kTileM), 0);
+    for (int j = 0; j * kTileM < c; ++j)
+      tiles[t++] = make_int4(e, off + j * kTileM, min(kTileM, c - j * kTileM), 0);
   }
   if (lane == 31) *n_mtiles = inc;
 }
 
+template <typename K>
+cudaError_t set_smem(K* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 }  // namespace
+
+int dispatch_blocks(int64_t n_pairs) {
+  const int64_t chunk = chunk_pairs(n_pairs);
+  return (int)((n_pairs + chunk - 1) / chunk);
+}
+
+cudaError_t launch_dispatch_gather(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
+                                   int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
+                                   const DispatchScratch& s, const void* z, void* zp,
+                                   int row_bytes, cudaStream_t st) {
+  const int64_t n_pairs = n * k;
+  const int64_t chunk = chunk_pairs(n_pairs);
+  const int nb = dispatch_blocks(n_pairs);
+  if (nb > 0) {
+    cudaError_t e = set_smem(hist_kernel, R * sizeof(int32_t));
+    if (e != cudaSuccess) return e;
+    hist_kernel<<<nb, kThreads, R * sizeof(int32_t), st>>>(ids, n_pairs, chunk, R,
+                                                           s.block_counts, s.status);
+    count_launch();
+  }
+  scan_kernel<<<1, 1024, 0, st>>>(s.block_counts, nb, R, counts, offsets, s.n_mtiles, s.tiles);
+  count_launch();
+  if (nb > 0) {
+    const size_t smem = (size_t)kWarps * R * sizeof(int32_t);
+    cudaError_t e = set_smem(scatter_kernel, smem);
+    if (e != cudaSuccess) return e;
+    scatter_kernel<<<nb, kThreads, smem, st>>>(ids, n_pairs, chunk, k, R, s.block_counts, offsets,
+                                               perm_token, inv_pair,
+                                               static_cast<const uint4*>(z),
+                                               static_cast<uint4*>(zp), row_bytes / 16);
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
+                            int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
+                            const DispatchScratch& s, cudaStream_t st) {
+  return launch_dispatch_gather(ids, n, k, R, counts, offsets, perm_token, inv_pair, s, nullptr,
+                                nullptr, 0, st);
+}
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
                                cudaStream_t st) {
   build_tiles_kernel<<<1, 32, 0, st>>>(offsets, R, n_mtiles, tiles);
   count_launch();
-  return cudaGetLastError();
-}
-
-int dispatch_blocks(int64_t n_pairs) { return (int)((n_pairs + kChunk - 1) / kChunk); }
-
-cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
-                            int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
-                            const DispatchScratch& s, cudaStream_t st) {
-  const int64_t n_pairs = n * k;
-  const int nb = dispatch_blocks(n_pairs);
-  if (nb > 0) {
-    hist_kernel<<<nb, kThreads, R * sizeof(int32_t), st>>>(ids, n_pairs, R, s.block_counts,
-                                                           s.status);
-    count_launch();
-  }
-  scan_kernel<<<1, 1024, 2 * R * sizeof(int32_t), st>>>(s.block_counts, nb, R, counts, offsets,
-                                                        s.n_mtiles, s.tiles);
-  count_launch();
-  if (nb > 0) {
-    size_t smem = (size_t)kWarps * R * sizeof(int32_t);
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    scatter_kernel<<<nb, kThreads, smem, st>>>(ids, n_pairs, k, R, s.block_counts, offsets,
-                                               perm_token, inv_pair);
-    count_launch();
-  }
   return cudaGetLastError();
 }
 

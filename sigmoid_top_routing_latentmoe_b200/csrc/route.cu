@@ -76,38 +76,51 @@ __device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (
   for (int slot = lane; slot < k; slot += 32) probs_row[slot] = probs_row[slot] / den;
 }
 
-// One warp per token.  W_r rows are read through L1/L2 (R <= 32 rows).
-// Each lane accumulates its share of d for every expert, then a butterfly
-// reduction leaves lane e holding expert e's logit.
-template <typename T>
+// One warp per token, RMAX >= R accumulators per lane.  Each lane reads x and
+// the matching slice of every W_r row in 16-byte vectors (W_r stays in L1/L2),
+// so lane j owns columns [8j, 8j+8) of every 256-column block.  A butterfly
+// transpose-reduction then leaves lane e holding expert e's logit.
+template <typename T, int RMAX>
 __global__ void __launch_bounds__(256) route_gemv_kernel(const T* __restrict__ x,
                                                          const T* __restrict__ w_r,
                                                          const float* __restrict__ bias, int64_t n,
                                                          int d, int R, int k,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ probs) {
+  constexpr int E = 16 / sizeof(T);  // elements per 16-byte vector
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= n) return;
-  const T* xr = x + t * d;
-  float acc[32];
+  const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
+  const int nvec = d / E;
+  float acc[RMAX];
 #pragma unroll
-  for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
-  for (int i = lane; i < d; i += 32) {
-    float xv = to_f(xr[i]);
+  for (int e = 0; e < RMAX; ++e) acc[e] = 0.0f;
+  for (int v = lane; v < nvec; v += 32) {
+    const uint4 xv = xr[v];
+    const T* xe = reinterpret_cast<const T*>(&xv);
+    float xf[E];
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (e < R) acc[e] = fmaf(to_f(w_r[(int64_t)e * d + i]), xv, acc[e]);
+    for (int i = 0; i < E; ++i) xf[i] = to_f(xe[i]);
+#pragma unroll
+    for (int e = 0; e < RMAX; ++e) {
+      if (e < R) {
+        const uint4 wv = reinterpret_cast<const uint4*>(w_r + (int64_t)e * d)[v];
+        const T* we = reinterpret_cast<const T*>(&wv);
+#pragma unroll
+        for (int i = 0; i < E; ++i) acc[e] = fmaf(to_f(we[i]), xf[i], acc[e]);
+      }
+    }
   }
-  // transpose-reduce: after the loop lane e holds sum over lanes of acc[e]
+  // sum over lanes; lane e keeps expert e
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
+  for (int e = 0; e < RMAX; ++e) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
   }
   float logit = 0.0f;
 #pragma unroll
-  for (int e = 0; e < 32; ++e)
+  for (int e = 0; e < RMAX; ++e)
     if (e == lane) logit = acc[e];
   float s[1], key[1];
   s[0] = sigmoid_f(logit);
@@ -144,7 +157,12 @@ cudaError_t launch_route_gemv(const T* x, const T* w_r, const float* bias, int64
   if (n == 0) return cudaSuccess;
   const int warps = 8;
   int64_t blocks = (n + warps - 1) / warps;
-  route_gemv_kernel<T><<<(unsigned)blocks, warps * 32, 0, st>>>(x, w_r, bias, n, d, R, k, ids, probs);
+  if (R <= 16)
+    route_gemv_kernel<T, 16><<<(unsigned)blocks, warps * 32, 0, st>>>(x, w_r, bias, n, d, R, k, ids,
+                                                                       probs);
+  else
+    route_gemv_kernel<T, 32><<<(unsigned)blocks, warps * 32, 0, st>>>(x, w_r, bias, n, d, R, k, ids,
+                                                                       probs);
   count_launch();
   return cudaGetLastError();
 }

@@ -25,6 +25,7 @@
 // Every mbarrier wait is capped: after ~2 s the kernel records LMOE_ETIMEOUT,
 // stops issuing work, drains what it issued, frees its TMEM and returns.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 #include <cstring>
@@ -36,21 +37,35 @@
 namespace lmoe {
 namespace {
 
-constexpr int BM = 128;          // tile rows (TMEM lanes)
+constexpr int BM = 128;          // rows per CTA (TMEM lanes)
 constexpr int BK = 64;           // K per stage: 64 bf16 = one 128-byte swizzle row
-constexpr int SUB = 128;         // rows of one B sub-tile
-constexpr int STAGES = 4;
+constexpr int SUB = 128;         // rows of a full B sub-tile
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int SUB_BYTES = SUB * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + 2 * SUB_BYTES;  // 48 KB
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
-constexpr int THREADS = 192;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+constexpr int EPI_WARPS = 8;    // two warps per TMEM lane quarter, splitting the columns
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint64_t WAIT_CAP_NS = 2000000000ull;
 
+// CG = 1: one CTA computes a 128-row tile and loads every B sub-tile.
+// CG = 2: a CTA pair (cluster of 2) computes a 256-row tile with
+//         tcgen05.mma.cta_group::2; each CTA loads its own 128 rows of A and
+//         one of the two B sub-tiles (half of N), so each SM streams half of
+//         B per FLOP.
+template <int CG>
+struct Cfg {
+  static constexpr int B_BYTES = (CG == 1 ? 2 : 1) * SUB * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB or 32 KB
+  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  static constexpr int MT = BM * CG;                     // tile rows
+};
+
 enum Mode { XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3 };
-enum Epi { EPI_Z = 1, EPI_LOGIT = 2, EPI_SITU = 3, EPI_STORE = 4 };
+enum Epi { EPI_Z = 1, EPI_SITU = 3, EPI_STORE = 4 };
+// B sub-tile sources of the x-pass: 0 W_down, 1 W_r, 2 W_g,sh, 3 W_u,sh,
+// 5 zero padding (a box outside W_r: loads zeros, stores nothing).
+constexpr int kPadMap = 5;
 
 struct Params {
   CUtensorMap tmA0, tmA1;              // A operands (FINAL: h_sh, uhat)
@@ -60,6 +75,12 @@ struct Params {
   int kb0, kb1;                        // K blocks (FINAL: per shared expert, then uhat)
   int S, G, L, R, F, d;
   int nz_sub, nr_sub, n_zr_tiles, g_blocks;
+  int bn;                              // FINAL / ROUTED2 tile width: 128, 192 or 256
+  int fuse_topk;                       // XPASS: top-k in the epilogue (R <= 32)
+  int top_k;
+  const float* bias;
+  int32_t* ids;
+  float* probs;
   void* out0;
   void* out1;
   void* out2;
@@ -67,12 +88,16 @@ struct Params {
   const int4* tiles;
   const int32_t* n_mtiles;
   int32_t* status;
-  float beta1, beta2, inv_beta1, inv_beta2;
+  float beta1, beta2, inv_beta1, inv_beta2, beta12;
 };
 
 struct Tile {
-  int m0, rows, expert, n_sub;
-  int bmap[2], brow[2], bz[2], epi, ocol;
+  int m0, rows, n_sub;
+  int ncols;                    // MMA N: sum of the sub-tiles' rows
+  int bmap[2], brow[2], bz[2];  // B source map, first row, expert (3-D maps)
+  int srows[2];                 // rows of each sub-tile load
+  int scol[2];                  // accumulator / output column of each sub-tile
+  int epi, ocol;
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -191,11 +216,33 @@ __device__ __forceinline__ float tanh_fast(float v) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
   return r;
 }
-// SiTU-GLU hidden unit: beta1 tanh(a/beta1) sigmoid(a) * beta2 tanh(c/beta2).
-__device__ __forceinline__ float situ_fast(float a, float c, const Params& p) {
-  float gate = p.beta1 * tanh_fast(a * p.inv_beta1) * __fdividef(1.0f, 1.0f + __expf(-a));
-  float up = p.beta2 * tanh_fast(c * p.inv_beta2);
-  return gate * up;
+__device__ __forceinline__ uint32_t tanh_h2(uint32_t v) {
+  uint32_t r;
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(r) : "r"(v));
+  return r;
+}
+// Two SiTU-GLU hidden units at once, packed to bf16x2:
+//   h = beta1 tanh(a/beta1) sigmoid(a) * beta2 tanh(c/beta2),
+//   sigmoid(a) = 1/2 + tanh(a/2)/2,
+// the three tanh on f16x2 pairs (one MUFU op per pair), the product of the
+// bounded factors (each |.| <= 1) in f16x2, the scale beta1*beta2 in fp32.
+__device__ __forceinline__ uint32_t situ2_bf16(float a0, float a1, float c0, float c1,
+                                               const Params& p) {
+  const __half2 x1 = __floats2half2_rn(a0 * p.inv_beta1, a1 * p.inv_beta1);
+  const __half2 x2 = __floats2half2_rn(a0 * 0.5f, a1 * 0.5f);
+  const __half2 x3 = __floats2half2_rn(c0 * p.inv_beta2, c1 * p.inv_beta2);
+  uint32_t u1 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x1));
+  uint32_t u2 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x2));
+  uint32_t u3 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x3));
+  const __half2 t1 = *reinterpret_cast<__half2*>(&u1);
+  const __half2 t2 = *reinterpret_cast<__half2*>(&u2);
+  const __half2 t3 = *reinterpret_cast<__half2*>(&u3);
+  const __half2 half = __float2half2_rn(0.5f);
+  const __half2 sg = __hfma2(t2, half, half);
+  const __half2 h = __hmul2(__hmul2(t1, sg), t3);
+  const float2 f = __half22float2(h);
+  __nv_bfloat162 o = __floats2bfloat162_rn(f.x * p.beta12, f.y * p.beta12);
+  return *reinterpret_cast<uint32_t*>(&o);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -203,30 +250,106 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ---------------------------------------------------------- cluster helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA loads of one CTA of a pair; the transaction bytes land on the barrier
+// at `bar` (a cluster address: the leader CTA's barrier).
+__device__ __forceinline__ void tma2_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                             int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma2_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                             int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc2_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive (when the issuing thread's MMAs complete) on the barrier at this
+// offset in both CTAs of the pair.
+__device__ __forceinline__ void tc2_commit_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128 * CG, N = n.
+template <int CG>
+__device__ __forceinline__ uint32_t instr_desc_cg(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)((BM * CG) >> 4) << 24);
+}
+
 // ---------------------------------------------------------- tile decoding
-template <int MODE>
+template <int MODE, int CG>
 __device__ __forceinline__ int total_tiles(const Params& p) {
-  if (MODE == XPASS || MODE == FINAL) return ((p.M + BM - 1) / BM) * p.n_tiles;
+  if (MODE == XPASS || MODE == FINAL) return ((p.M + Cfg<CG>::MT - 1) / Cfg<CG>::MT) * p.n_tiles;
   return (*p.n_mtiles) * p.n_tiles;
 }
 
-template <int MODE>
+template <int MODE, int CG>
 __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
   Tile tl;
   tl.bz[0] = tl.bz[1] = 0;
+  tl.srows[0] = tl.srows[1] = SUB;
+  tl.scol[0] = 0;
+  tl.scol[1] = SUB;
   if (MODE == XPASS || MODE == FINAL) {
-    const int m_tiles = (p.M + BM - 1) / BM;
+    constexpr int MT = Cfg<CG>::MT;
+    const int m_tiles = (p.M + MT - 1) / MT;
     const int mt = t % m_tiles, n = t / m_tiles;
-    tl.m0 = mt * BM;
-    tl.rows = min(BM, p.M - tl.m0);
-    tl.expert = 0;
+    tl.m0 = mt * MT;
+    tl.rows = min(MT, p.M - tl.m0);
     if (MODE == FINAL) {
-      tl.n_sub = (n * 2 * SUB + SUB < p.d) ? 2 : 1;
+      const int n0 = n * p.bn;
+      if (CG == 2) {  // each CTA loads half of the tile's columns
+        tl.n_sub = 2;
+        tl.srows[0] = tl.srows[1] = p.bn / 2;
+        tl.scol[1] = p.bn / 2;
+        tl.brow[0] = n0;
+        tl.brow[1] = n0 + p.bn / 2;
+        tl.ncols = p.bn;
+      } else {
+        tl.n_sub = (p.bn > SUB && n0 + SUB < p.d) ? 2 : 1;
+        tl.srows[1] = p.bn - SUB;
+        tl.brow[0] = n0;
+        tl.brow[1] = n0 + SUB;
+        tl.ncols = tl.n_sub == 2 ? p.bn : SUB;
+      }
       tl.bmap[0] = tl.bmap[1] = 0;
-      tl.brow[0] = n * 2 * SUB;
-      tl.brow[1] = n * 2 * SUB + SUB;
       tl.epi = EPI_STORE;
-      tl.ocol = n * 2 * SUB;
+      tl.ocol = n0;
     } else if (n < p.n_zr_tiles) {
       tl.n_sub = 0;
       for (int s = 0; s < 2; ++s) {
@@ -239,10 +362,15 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
           tl.bmap[s] = 1;
           tl.brow[s] = (idx - p.nz_sub) * SUB;
           tl.n_sub = s + 1;
+        } else {  // a pair tile always loads two sub-tiles: pad with zeros
+          tl.bmap[s] = kPadMap;
+          tl.brow[s] = p.nr_sub * SUB;
         }
       }
-      tl.epi = EPI_Z;  // per sub-tile: Z or LOGIT, resolved in the epilogue
-      tl.ocol = 2 * n;
+      if (CG == 2) tl.n_sub = 2;
+      tl.epi = EPI_Z;  // per sub-tile: z, routing or padding, resolved in the epilogue
+      tl.ocol = 0;
+      tl.ncols = tl.n_sub * SUB;
     } else {
       const int q = n - p.n_zr_tiles;
       const int j = q / p.g_blocks, fb = q % p.g_blocks;
@@ -253,11 +381,11 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
       tl.bz[0] = tl.bz[1] = j;
       tl.epi = EPI_SITU;
       tl.ocol = j * p.G + fb * SUB;
+      tl.ncols = 2 * SUB;
     }
   } else {
     const int mt = t / p.n_tiles, n = t % p.n_tiles;
     const int4 e = p.tiles[mt];
-    tl.expert = e.x;
     tl.m0 = e.y;
     tl.rows = e.z;
     tl.bz[0] = tl.bz[1] = e.x;
@@ -268,13 +396,18 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
       tl.brow[0] = tl.brow[1] = n * SUB;
       tl.epi = EPI_SITU;
       tl.ocol = n * SUB;
+      tl.ncols = 2 * SUB;
     } else {
-      tl.n_sub = (n * 2 * SUB + SUB < p.L) ? 2 : 1;
-      tl.bmap[0] = tl.bmap[1] = 0;
-      tl.brow[0] = n * 2 * SUB;
-      tl.brow[1] = n * 2 * SUB + SUB;
+      const int n0 = n * p.bn;
+      tl.n_sub = (p.bn > SUB && n0 + SUB < p.L) ? 2 : 1;
+      tl.bmap[0] = 0;
+      tl.bmap[1] = 1;  // map 1: the (bn - 128)-row box
+      tl.brow[0] = n0;
+      tl.brow[1] = n0 + SUB;
+      tl.srows[1] = p.bn - SUB;
+      tl.ncols = tl.n_sub == 2 ? p.bn : SUB;
       tl.epi = EPI_STORE;
-      tl.ocol = n * 2 * SUB;
+      tl.ocol = n0;
     }
   }
   return tl;
@@ -289,84 +422,121 @@ __device__ __forceinline__ const CUtensorMap* bmap_ptr(const Params& p, int i) {
   return i == 0 ? &p.tmB0 : i == 1 ? &p.tmB1 : i == 2 ? &p.tmB2 : &p.tmB3;
 }
 
+// Loads one B sub-tile (CG = 1 loads into the CTA's own barrier; CG = 2 into
+// the leader's).
+template <int CG>
+__device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* map, bool three_d,
+                                       uint32_t bar, int kk, int row, int z) {
+  if (CG == 1) {
+    if (three_d)
+      tma_load_3d(dst, map, bar, kk, row, z);
+    else
+      tma_load_2d(dst, map, bar, kk, row);
+  } else {
+    if (three_d)
+      tma2_load_3d(dst, map, bar, kk, row, z);
+    else
+      tma2_load_2d(dst, map, bar, kk, row);
+  }
+}
+
 // ------------------------------------------------------------- producer
-template <int MODE>
+template <int MODE, int CG>
 __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t* full,
-                                        uint64_t* empty, volatile int* abort_flag) {
+                                        uint64_t* empty, volatile int* abort_flag, uint32_t rank,
+                                        int unit, int n_units) {
+  using C = Cfg<CG>;
   int stage = 0;
   uint32_t phase = 0;
-  int issued_parity[STAGES];
+  int issued_parity[C::STAGES];
 #pragma unroll
-  for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
-  const int total = total_tiles<MODE>(p);
+  for (int s = 0; s < C::STAGES; ++s) issued_parity[s] = -1;
+  const int total = total_tiles<MODE, CG>(p);
   const int nkb = k_blocks<MODE>(p);
   bool ok = true;
-  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-    const Tile tl = decode_tile<MODE>(p, t);
+  for (int t = unit; t < total && ok; t += n_units) {
+    const Tile tl = decode_tile<MODE, CG>(p, t);
+    const int arow = tl.m0 + (CG == 2 ? BM * (int)rank : 0);
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.status)) {
         ok = false;
         break;
       }
-      const uint32_t a_dst = smem_u32(ring + stage * STAGE_BYTES);
+      const uint32_t a_dst = smem_u32(ring + stage * C::STAGE_BYTES);
       const uint32_t b_dst = a_dst + A_BYTES;
-      const uint32_t bar = smem_u32(&full[stage]);
-      mbar_expect_tx(bar, A_BYTES + tl.n_sub * SUB_BYTES);
+      const uint32_t own_bar = smem_u32(&full[stage]);
+      const uint32_t bar = CG == 1 ? own_bar : map_to_rank(own_bar, 0);
+      if (CG == 1 || rank == 0)
+        mbar_expect_tx(own_bar, CG * A_BYTES + tl.ncols * BK * 2);
+      // sub-tiles this CTA loads: all of them (CG = 1) or the one of its rank
+      const int s0 = CG == 1 ? 0 : (int)rank;
+      const int s1 = CG == 1 ? tl.n_sub : (int)rank + 1;
       if (MODE == FINAL) {
         const int kb_sh = p.S * p.kb0;
         if (kb < kb_sh) {
           const int j = kb / p.kb0, kk = (kb % p.kb0) * BK;
-          tma_load_2d(a_dst, &p.tmA0, bar, j * p.G + kk, tl.m0);
-          for (int s = 0; s < tl.n_sub; ++s)
-            tma_load_3d(b_dst + s * SUB_BYTES, &p.tmB0, bar, kk, tl.brow[s], j);
+          if (CG == 1) tma_load_2d(a_dst, &p.tmA0, bar, j * p.G + kk, arow);
+          else tma2_load_2d(a_dst, &p.tmA0, bar, j * p.G + kk, arow);
+          for (int s = s0; s < s1; ++s)
+            load_b<CG>(b_dst + (CG == 1 ? s * SUB * BK * 2 : 0), s == 0 ? &p.tmB0 : &p.tmB2, true,
+                       bar, kk, tl.brow[s], j);
         } else {
           const int kk = (kb - kb_sh) * BK;
-          tma_load_2d(a_dst, &p.tmA1, bar, kk, tl.m0);
-          for (int s = 0; s < tl.n_sub; ++s)
-            tma_load_2d(b_dst + s * SUB_BYTES, &p.tmB1, bar, kk, tl.brow[s]);
+          if (CG == 1) tma_load_2d(a_dst, &p.tmA1, bar, kk, arow);
+          else tma2_load_2d(a_dst, &p.tmA1, bar, kk, arow);
+          for (int s = s0; s < s1; ++s)
+            load_b<CG>(b_dst + (CG == 1 ? s * SUB * BK * 2 : 0), s == 0 ? &p.tmB1 : &p.tmB3, false,
+                       bar, kk, tl.brow[s], 0);
         }
       } else {
         const int kk = kb * BK;
-        tma_load_2d(a_dst, &p.tmA0, bar, kk, tl.m0);
-        for (int s = 0; s < tl.n_sub; ++s) {
-          const int m = tl.bmap[s];
-          if (MODE == XPASS && m < 2)
-            tma_load_2d(b_dst + s * SUB_BYTES, bmap_ptr(p, m), bar, kk, tl.brow[s]);
-          else
-            tma_load_3d(b_dst + s * SUB_BYTES, bmap_ptr(p, m), bar, kk, tl.brow[s], tl.bz[s]);
+        if (CG == 1) tma_load_2d(a_dst, &p.tmA0, bar, kk, arow);
+        else tma2_load_2d(a_dst, &p.tmA0, bar, kk, arow);
+        for (int s = s0; s < s1; ++s) {
+          int m = tl.bmap[s];
+          const bool pad = (MODE == XPASS && m == kPadMap);
+          if (pad) m = 1;
+          const bool three_d = !(MODE == XPASS && m < 2);
+          load_b<CG>(b_dst + (CG == 1 ? s * SUB * BK * 2 : 0), bmap_ptr(p, m), three_d, bar, kk,
+                     tl.brow[s], tl.bz[s]);
         }
       }
       issued_parity[stage] = (int)phase;
-      if (++stage == STAGES) {
+      if (++stage == C::STAGES) {
         stage = 0;
         phase ^= 1u;
       }
     }
   }
-  // drain: every load this thread issued has landed before the CTA exits
+  // drain: every load issued into this CTA's barriers has landed before exit
+  // (a pair's loads all land on the leader's barriers)
+  if (CG == 1 || rank == 0) {
 #pragma unroll
-  for (int s = 0; s < STAGES; ++s)
-    if (issued_parity[s] >= 0) {
-      volatile int no_abort = 0;
-      mbar_wait(smem_u32(&full[s]), (uint32_t)issued_parity[s], &no_abort, p.status);
-    }
+    for (int s = 0; s < C::STAGES; ++s)
+      if (issued_parity[s] >= 0) {
+        volatile int no_abort = 0;
+        mbar_wait(smem_u32(&full[s]), (uint32_t)issued_parity[s], &no_abort, p.status);
+      }
+  }
 }
 
 // ------------------------------------------------------------ MMA issuer
-template <int MODE>
+template <int MODE, int CG>
 __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64_t* full,
                                           uint64_t* empty, uint64_t* tfull, uint64_t* tempty,
-                                          uint64_t* drain, uint32_t tmem, volatile int* abort_flag) {
+                                          uint64_t* drain, uint32_t tmem, volatile int* abort_flag,
+                                          int unit, int n_units) {
+  using C = Cfg<CG>;
   int stage = 0;
   uint32_t phase = 0;
   int acc = 0;
   uint32_t acc_phase = 0;
-  const int total = total_tiles<MODE>(p);
+  const int total = total_tiles<MODE, CG>(p);
   const int nkb = k_blocks<MODE>(p);
   bool ok = true;
-  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-    const Tile tl = decode_tile<MODE>(p, t);
-    const uint32_t idesc = instr_desc(tl.n_sub * SUB);
+  for (int t = unit; t < total && ok; t += n_units) {
+    const Tile tl = decode_tile<MODE, CG>(p, t);
+    const uint32_t idesc = instr_desc_cg<CG>(tl.ncols);
     if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.status)) break;
     tc_fence_after();
     const uint32_t d_tmem = tmem + acc * ACC_COLS;
@@ -376,28 +546,40 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
         break;
       }
       tc_fence_after();
-      const uint32_t a_addr = smem_u32(ring + stage * STAGE_BYTES);
+      const uint32_t a_addr = smem_u32(ring + stage * C::STAGE_BYTES);
       const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
       for (int k = 0; k < BK / 16; ++k) {
-        tc_mma(d_tmem, smem_desc(a_addr + k * 32), smem_desc(b_addr + k * 32), idesc,
-               (kb > 0 || k > 0) ? 1u : 0u);
+        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+        if (CG == 1)
+          tc_mma(d_tmem, smem_desc(a_addr + k * 32), smem_desc(b_addr + k * 32), idesc, accum);
+        else
+          tc2_mma(d_tmem, smem_desc(a_addr + k * 32), smem_desc(b_addr + k * 32), idesc, accum);
       }
-      tc_commit(smem_u32(&empty[stage]));
-      if (++stage == STAGES) {
+      if (CG == 1)
+        tc_commit(smem_u32(&empty[stage]));
+      else
+        tc2_commit_both(smem_u32(&empty[stage]));
+      if (++stage == C::STAGES) {
         stage = 0;
         phase ^= 1u;
       }
     }
     if (!ok) break;
-    tc_commit(smem_u32(&tfull[acc]));
+    if (CG == 1)
+      tc_commit(smem_u32(&tfull[acc]));
+    else
+      tc2_commit_both(smem_u32(&tfull[acc]));
     if (++acc == 2) {
       acc = 0;
       acc_phase ^= 1u;
     }
   }
   // drain: all MMAs this thread issued are complete before TMEM is freed
-  tc_commit(smem_u32(drain));
+  if (CG == 1)
+    tc_commit(smem_u32(drain));
+  else
+    tc2_commit_both(smem_u32(drain));
   volatile int no_abort = 0;
   mbar_wait(smem_u32(drain), 0, &no_abort, p.status);
 }
@@ -418,17 +600,59 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&
   }
 }
 
-template <int MODE>
+// K3 routing of one row from its fp32 logits (R <= 32, one TMEM chunk):
+// s = sigmoid(l), T = TopK(s + b, k) in descending key order (ties to the
+// lower expert), p = s_T / max(sum s_T, 1e-9).  Same operations, in the same
+// order, as the standalone top-k kernel.
+__device__ __forceinline__ void route_row32(const Params& p, const float (&lg)[32], int64_t row) {
+  float sc[32], key[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    sc[e] = 1.0f / (1.0f + expf(-lg[e]));
+    key[e] = (e < p.R) ? sc[e] + (p.bias != nullptr ? p.bias[e] : 0.0f) : -INFINITY;
+  }
+  float den = 0.0f;
+  int32_t* ids = p.ids + row * p.top_k;
+  float* probs = p.probs + row * p.top_k;
+#pragma unroll 1
+  for (int slot = 0; slot < p.top_k; ++slot) {
+    int best = 0;
+    float bk = key[0];
+#pragma unroll
+    for (int e = 1; e < 32; ++e)
+      if (key[e] > bk) {
+        bk = key[e];
+        best = e;
+      }
+    float sel = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (e == best) {
+        sel = sc[e];
+        key[e] = -INFINITY;
+      }
+    ids[slot] = best;
+    probs[slot] = sel;
+    den += sel;
+  }
+  den = fmaxf(den, 1e-9f);
+#pragma unroll 1
+  for (int slot = 0; slot < p.top_k; ++slot) probs[slot] = probs[slot] / den;
+}
+
+template <int MODE, int CG>
 __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint64_t* tempty,
-                                         uint32_t tmem, volatile int* abort_flag) {
+                                         uint32_t tmem, volatile int* abort_flag, uint32_t rank,
+                                         int unit, int n_units) {
   const int ew = (threadIdx.x >> 5) & 3;  // TMEM lane quarter this warp may access
+  const int half = ((threadIdx.x >> 5) - 2) >> 2;  // which of the two column halves
   const int lane = threadIdx.x & 31;
-  const int r = ew * 32 + lane;           // tile row of this thread
+  const int r = ew * 32 + lane + (CG == 2 ? BM * (int)rank : 0);  // tile row of this thread
   int acc = 0;
   uint32_t acc_phase = 0;
-  const int total = total_tiles<MODE>(p);
-  for (int t = blockIdx.x; t < total; t += gridDim.x) {
-    const Tile tl = decode_tile<MODE>(p, t);
+  const int total = total_tiles<MODE, CG>(p);
+  for (int t = unit; t < total; t += n_units) {
+    const Tile tl = decode_tile<MODE, CG>(p, t);
     if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.status)) break;
     tc_fence_after();
     const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * ACC_COLS;
@@ -449,30 +673,49 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         ld = p.ld0;
       }
 #pragma unroll 1
-      for (int c = 0; c < SUB / 32; ++c) {
+      for (int c = half; c < SUB / 32; c += 2) {
         float g[32], u[32];
         tc_ld32(tbase + c * 32, g);
         tc_ld32(tbase + SUB + c * 32, u);
         if (row_ok) {
+          __nv_bfloat16* dst = out + grow * ld + tl.ocol + c * 32;
+          const int valid = width - c * 32;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) g[i] = situ_fast(g[i], u[i], p);
-          store_bf16x32(out + grow * ld + tl.ocol + c * 32, g, width - c * 32);
+          for (int q = 0; q < 4; ++q) {
+            if (q * 8 < valid) {
+              uint4 w;
+              w.x = situ2_bf16(g[q * 8 + 0], g[q * 8 + 1], u[q * 8 + 0], u[q * 8 + 1], p);
+              w.y = situ2_bf16(g[q * 8 + 2], g[q * 8 + 3], u[q * 8 + 2], u[q * 8 + 3], p);
+              w.z = situ2_bf16(g[q * 8 + 4], g[q * 8 + 5], u[q * 8 + 4], u[q * 8 + 5], p);
+              w.w = situ2_bf16(g[q * 8 + 6], g[q * 8 + 7], u[q * 8 + 6], u[q * 8 + 7], p);
+              reinterpret_cast<uint4*>(dst)[q] = w;
+            }
+          }
         }
       }
     } else {
 #pragma unroll 1
       for (int s = 0; s < tl.n_sub; ++s) {
+        if (MODE == XPASS && tl.bmap[s] == kPadMap) continue;
+        if (MODE == XPASS && tl.bmap[s] == 1 && p.fuse_topk) {
+          // all R <= 32 router logits of this row sit in one 32-column chunk
+          if (half == 0) {
+            float lg[32];
+            tc_ld32(tbase + tl.scol[s], lg);
+            if (row_ok) route_row32(p, lg, grow);
+          }
+          continue;
+        }
 #pragma unroll 1
-        for (int c = 0; c < SUB / 32; ++c) {
+        for (int c = half; c < tl.srows[s] / 32; c += 2) {
           float v[32];
-          tc_ld32(tbase + s * SUB + c * 32, v);
+          tc_ld32(tbase + tl.scol[s] + c * 32, v);
           if (!row_ok) continue;
           if (MODE == XPASS) {
+            const int col = tl.brow[s] + c * 32;
             if (tl.bmap[s] == 0) {  // z columns
-              const int col = tl.brow[s] + c * 32;
               store_bf16x32(static_cast<__nv_bfloat16*>(p.out0) + grow * p.ld0 + col, v, p.L - col);
             } else {                // router logits, fp32
-              const int col = tl.brow[s] + c * 32;
               float* dst = static_cast<float*>(p.out1) + grow * p.ld1 + col;
 #pragma unroll
               for (int g4 = 0; g4 < 8; ++g4)
@@ -481,7 +724,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
                       make_float4(v[g4 * 4], v[g4 * 4 + 1], v[g4 * 4 + 2], v[g4 * 4 + 3]);
             }
           } else {
-            const int col = tl.ocol + s * SUB + c * 32;
+            const int col = tl.ocol + tl.scol[s] + c * 32;
             const int width = (MODE == FINAL ? p.d : p.L) - col;
             store_bf16x32(static_cast<__nv_bfloat16*>(p.out0) + grow * p.ld0 + col, v, width);
           }
@@ -490,7 +733,12 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+    if (lane == 0) {
+      if (CG == 1)
+        mbar_arrive(smem_u32(&tempty[acc]));
+      else  // the leader's MMA thread waits for both CTAs' epilogues
+        mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[acc]), 0));
+    }
     if (++acc == 2) {
       acc = 0;
       acc_phase ^= 1u;
@@ -498,56 +746,78 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
   }
 }
 
-template <int MODE>
+template <int MODE, int CG>
 __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
+  using C = Cfg<CG>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  __shared__ __align__(8) uint64_t full[C::STAGES], empty[C::STAGES], tfull[2], tempty[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0;
+  const int unit = CG == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int n_units = CG == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), 4);
+      mbar_init(smem_u32(&tempty[a]), EPI_WARPS * CG);
     }
     mbar_init(smem_u32(&drain), 1);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&tmem_slot)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (CG == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&tmem_slot)),
+                   "r"(TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&tmem_slot)),
+                   "r"(TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) produce<MODE>(p, ring, full, empty, &abort_flag);
-  } else if (warp == 1) {
     if ((threadIdx.x & 31) == 0)
-      mma_issue<MODE>(p, ring, full, empty, tfull, tempty, &drain, tmem, &abort_flag);
+      produce<MODE, CG>(p, ring, full, empty, &abort_flag, rank, unit, n_units);
+  } else if (warp == 1) {
+    if ((threadIdx.x & 31) == 0 && rank == 0)
+      mma_issue<MODE, CG>(p, ring, full, empty, tfull, tempty, &drain, tmem, &abort_flag, unit,
+                          n_units);
   } else {
-    epilogue<MODE>(p, tfull, tempty, tmem, &abort_flag);
+    epilogue<MODE, CG>(p, tfull, tempty, tmem, &abort_flag, rank, unit, n_units);
   }
 
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();  // neither CTA frees TMEM or exits while its pair still works
   tc_fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
-                 : "memory");
+    if (CG == 1)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(TMEM_COLS)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(TMEM_COLS)
+                   : "memory");
   }
 }
 
@@ -612,19 +882,56 @@ static int num_sms() {
   return n;
 }
 
-template <int MODE>
+// grid: CTAs (CG = 1) or CTA pairs (CG = 2).
+template <int MODE, int CG>
 static cudaError_t launch(const Params& p, int grid, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(umma_gemm_kernel<MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(umma_gemm_kernel<MODE, CG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<CG>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   if (grid <= 0) return cudaSuccess;
-  umma_gemm_kernel<MODE><<<grid, THREADS, SMEM_BYTES, st>>>(p);
+  if (CG == 1) {
+    umma_gemm_kernel<MODE, 1><<<grid, THREADS, Cfg<CG>::SMEM_BYTES, st>>>(p);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * grid, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg<CG>::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeClusterDimension;
+    attrs[0].val.clusterDim.x = 2;
+    attrs[0].val.clusterDim.y = 1;
+    attrs[0].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, umma_gemm_kernel<MODE, CG>, p);
+    if (e != cudaSuccess) return e;
+  }
   count_launch();
   return cudaGetLastError();
+}
+
+// Tile width for the plain-store GEMMs: the one of 256, 192, 128 columns that
+// minimises (waves of tiles over the SMs) x (columns per tile), ties to the
+// wider tile.
+static int pick_bn(int m_tiles, int width, int units) {
+  int best = 256;
+  int64_t best_cost = -1;
+  for (int bn : {256, 192, 128}) {
+    const int64_t tiles = (int64_t)m_tiles * ((width + bn - 1) / bn);
+    const int64_t waves = (tiles + units - 1) / units;
+    const int64_t cost = waves * bn;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
 }
 
 static Params base_params(int32_t* status) {
@@ -668,17 +975,28 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   p.beta2 = a.beta2;
   p.inv_beta1 = 1.0f / a.beta1;
   p.inv_beta2 = 1.0f / a.beta2;
-  const int total = (int)((a.N + BM - 1) / BM) * p.n_tiles;
-  return launch<XPASS>(p, std::min(total, num_sms()), st);
+  p.beta12 = a.beta1 * a.beta2;
+  p.fuse_topk = (a.ids != nullptr && a.R <= 32) ? 1 : 0;
+  p.top_k = a.top_k;
+  p.bias = a.bias;
+  p.ids = a.ids;
+  p.probs = a.probs;
+  const int total = (int)((a.N + 2 * BM - 1) / (2 * BM)) * p.n_tiles;
+  return launch<XPASS, 2>(p, std::min(total, num_sms() / 2), st);
 }
 
 cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
   if (a.N == 0) return cudaSuccess;
   Params p = base_params(status);
-  bool ok = make_map(&p.tmA1, a.uhat, a.L, a.N, 1, BM) && make_map(&p.tmB1, a.w_up, a.L, a.d, 1, SUB);
+  const int m_tiles = (int)((a.N + 2 * BM - 1) / (2 * BM));
+  p.bn = pick_bn(m_tiles, a.d, num_sms() / 2);
+  const uint32_t hb = p.bn / 2;  // rows of B each CTA of the pair loads
+  bool ok = make_map(&p.tmA1, a.uhat, a.L, a.N, 1, BM) && make_map(&p.tmB1, a.w_up, a.L, a.d, 1, hb) &&
+            make_map(&p.tmB3, a.w_up, a.L, a.d, 1, hb);
   if (a.S > 0)
     ok = ok && make_map(&p.tmA0, a.hsh, (uint64_t)a.S * a.G, a.N, 1, BM) &&
-         make_map3(&p.tmB0, a.ws_o, a.G, a.d, a.S, SUB);
+         make_map3(&p.tmB0, a.ws_o, a.G, a.d, a.S, hb) &&
+         make_map3(&p.tmB2, a.ws_o, a.G, a.d, a.S, hb);
   if (!ok) return cudaErrorInvalidValue;
   p.M = (int)a.N;
   p.S = a.S;
@@ -687,11 +1005,11 @@ cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
   p.kb1 = (a.L + BK - 1) / BK;
   p.L = a.L;
   p.d = a.d;
-  p.n_tiles = (a.d + 2 * SUB - 1) / (2 * SUB);
+  p.n_tiles = (a.d + p.bn - 1) / p.bn;
   p.out0 = a.y;
   p.ld0 = a.d;
-  const int total = (int)((a.N + BM - 1) / BM) * p.n_tiles;
-  return launch<FINAL>(p, std::min(total, num_sms()), st);
+  const int total = m_tiles * p.n_tiles;
+  return launch<FINAL, 2>(p, std::min(total, num_sms() / 2), st);
 }
 
 cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) {
@@ -713,26 +1031,29 @@ cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   p.beta2 = a.beta2;
   p.inv_beta1 = 1.0f / a.beta1;
   p.inv_beta2 = 1.0f / a.beta2;
+  p.beta12 = a.beta1 * a.beta2;
   const int64_t bound = (int64_t)a.max_tiles * p.n_tiles;
-  return launch<ROUTED1>(p, (int)std::min<int64_t>(bound, num_sms()), st);
+  return launch<ROUTED1, 1>(p, (int)std::min<int64_t>(bound, num_sms()), st);
 }
 
 cudaError_t umma_routed2(const RoutedArgs& a, int32_t* status, cudaStream_t st) {
   if (a.P == 0) return cudaSuccess;
   Params p = base_params(status);
-  bool ok = make_map(&p.tmA0, a.a, a.F, a.P, 1, BM) && make_map3(&p.tmB0, a.w0, a.F, a.L, a.R, SUB);
+  p.bn = pick_bn((int)((a.P + BM - 1) / BM) + a.R / 2, a.L, num_sms());
+  bool ok = make_map(&p.tmA0, a.a, a.F, a.P, 1, BM) && make_map3(&p.tmB0, a.w0, a.F, a.L, a.R, SUB) &&
+            (p.bn == SUB || make_map3(&p.tmB1, a.w0, a.F, a.L, a.R, p.bn - SUB));
   if (!ok) return cudaErrorInvalidValue;
   p.kb0 = (a.F + BK - 1) / BK;
   p.L = a.L;
   p.F = a.F;
   p.R = a.R;
-  p.n_tiles = (a.L + 2 * SUB - 1) / (2 * SUB);
+  p.n_tiles = (a.L + p.bn - 1) / p.bn;
   p.out0 = a.out;
   p.ld0 = a.L;
   p.tiles = a.tiles;
   p.n_mtiles = a.n_mtiles;
   const int64_t bound = (int64_t)a.max_tiles * p.n_tiles;
-  return launch<ROUTED2>(p, (int)std::min<int64_t>(bound, num_sms()), st);
+  return launch<ROUTED2, 1>(p, (int)std::min<int64_t>(bound, num_sms()), st);
 }
 
 }  // namespace lmoe

@@ -27,6 +27,12 @@ struct XpassArgs {
   int64_t logits_ld;
   __nv_bfloat16* hsh;
   float beta1, beta2;
+  // When R <= 32 and ids != nullptr the epilogue also routes each row (K3 top-k
+  // + L1 normalisation with bias b) and writes ids/probs instead of logits.
+  const float* bias;
+  int32_t* ids;
+  float* probs;
+  int top_k;
 };
 
 // final: y [N, d] = sum_j hsh[:, jG:(j+1)G] W_o,sh_j^T + uhat W_up^T

@@ -253,8 +253,9 @@ def test_forward_intermediates(name, n):
     x = synth.to_f32(inp["x"]).astype(np.float64)
     ref = oracle.forward(odims(wl), ow, synth.to_f32(inp["x"]), want=("z", "uhat"))
     assert rel_err(host(v["z"]), ref["z"]) <= 1e-2, "z"
-    logits = x @ ow["w_router"].astype(np.float64).T
-    assert rel_err(host(v["logits"]), logits) <= 1e-5, "router logits"
+    if wl.n_routed > 32:   # up to 32 experts the x-pass routes in its epilogue, no logits
+        logits = x @ ow["w_router"].astype(np.float64).T
+        assert rel_err(host(v["logits"]), logits) <= 1e-5, "router logits"
     if wl.n_shared:
         hs = np.empty((n, wl.n_shared * wl.ff_shared))
         for t in range(n):
