@@ -56,7 +56,7 @@ def kernel_work(wl: synth.Workload, tag: str):
         return "tensor", 2.0 * P * L * 2 * F
     if tag == "expert_gemm2":
         return "tensor", 2.0 * P * F * L
-    if tag == "final":
+    if tag == "final":      # shared output projection + W_up RMSNorm(u), one accumulator
         return "tensor", 2.0 * N * (S * G + L) * d
     if tag == "combine":    # read k expert rows + ids/probs, write uhat
         return "hbm", float(P * L * es + P * 8 + N * L * es)
@@ -218,6 +218,8 @@ def main():
     ap.add_argument("--profile-kernel", default=None,
                     help="kernel tag for the roofline line (default: the largest GEMM)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the kernels every step instead of replaying a CUDA graph")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -271,8 +273,26 @@ def main():
     prof_tag = args.profile_kernel or "xpass"
     bound, work = kernel_work(wl, prof_tag)
     lm.profile_read()                       # drop anything recorded so far
-    lm.profile_enable(prof_tag)
     clocks = ClockSampler(local)
+
+    # One step is captured once in a CUDA graph (with the dominant kernel
+    # bracketed by events) and replayed; --eager launches it every step.
+    graph = None
+    launches_per_step = None
+    if not args.eager:
+        lm.launch_count(reset=True)
+        lm.profile_enable(prof_tag)
+        graph = torch.cuda.CUDAGraph()
+        cap_stream = torch.cuda.Stream(dev)
+        cap_stream.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap_stream):
+            step()
+        lm.profile_enable(None)
+        launches_per_step = lm.launch_count(reset=True)
+        graph.replay()
+        torch.cuda.synchronize()
+    else:
+        lm.profile_enable(prof_tag)
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -280,19 +300,31 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     lm.launch_count(reset=True)
+    k_ms, k_n = 0.0, 0
     clocks.start()
     for i in range(args.steps):
         flush.zero_()                        # L2 flushed between timed steps (outside the events)
         starts[i].record(stream)
-        step()
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
         ends[i].record(stream)
+        if graph is not None:                # the graph re-records its events on every replay
+            ms_i, n_i = lm.profile_peek(prof_tag)
+            k_ms += ms_i
+            k_n += n_i
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    launches = lm.launch_count()
-    lm.profile_enable(None)
-    k_ms, k_n = lm.profile_read(prof_tag)
+    if graph is not None:
+        launches = launches_per_step * args.steps
+        lm.profile_read()
+    else:
+        launches = lm.launch_count()
+        lm.profile_enable(None)
+        k_ms, k_n = lm.profile_read(prof_tag)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
@@ -359,7 +391,8 @@ def main():
         "config": {"workload": wl.name, "n_tokens": wl.n_tokens, "d": wl.d, "latent": wl.latent,
                    "n_routed": wl.n_routed, "top_k": wl.top_k, "ff_routed": wl.ff_routed,
                    "n_shared": wl.n_shared, "ff_shared": wl.ff_shared,
-                   "parallelism": f"replicas{world}", "l2": "flushed (256 MiB write) between steps"},
+                   "parallelism": f"replicas{world}", "l2": "flushed (256 MiB write) between steps",
+                   "launch": "eager" if args.eager else "cuda graph replay"},
         "layer_roofline": {"flops": wl.flops(), "compulsory_bytes": wl.compulsory_bytes(),
                            "roof_us": roof_s * 1e6, "frac": roof_s / (ms_per_step / 1e3),
                            "peak_source": peaks["source"] + " burst"},

@@ -225,6 +225,9 @@ LMOE_API lmoe_status lmoe_profile_enable(const char* tags);
  * read of that tag, and clears them. */
 LMOE_API lmoe_status lmoe_profile_read_tag(const char* tag, double* total_ms, int64_t* launches);
 LMOE_API lmoe_status lmoe_profile_read(double* total_ms, int64_t* launches);
+/* Like lmoe_profile_read_tag but keeps the event pairs: for launches captured
+ * in a CUDA graph, whose events are recorded again on every replay. */
+LMOE_API lmoe_status lmoe_profile_peek_tag(const char* tag, double* total_ms, int64_t* launches);
 
 /* Number of kernel launches the library issued on this thread since the last
  * reset (instrumentation for benchmarks). */

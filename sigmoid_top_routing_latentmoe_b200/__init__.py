@@ -78,6 +78,8 @@ _sigs = {
     "lmoe_profile_read": (_S, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     "lmoe_profile_read_tag": (_S, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
                                    ctypes.POINTER(ctypes.c_int64)]),
+    "lmoe_profile_peek_tag": (_S, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
+                                   ctypes.POINTER(ctypes.c_int64)]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -226,6 +228,15 @@ def profile_read(tag=None):
     ms, n = ctypes.c_double(), ctypes.c_int64()
     _check(_lib.lmoe_profile_read_tag(None if tag is None else tag.encode(), ctypes.byref(ms),
                                       ctypes.byref(n)), "lmoe_profile_read_tag")
+    return ms.value, n.value
+
+
+def profile_peek(tag=None):
+    """(summed device ms, launches) of the bracketed kernel ``tag``, keeping the
+    events (for launches inside a CUDA graph, re-recorded on every replay)."""
+    ms, n = ctypes.c_double(), ctypes.c_int64()
+    _check(_lib.lmoe_profile_peek_tag(None if tag is None else tag.encode(), ctypes.byref(ms),
+                                      ctypes.byref(n)), "lmoe_profile_peek_tag")
     return ms.value, n.value
 
 

@@ -40,15 +40,20 @@ struct ProfScope {
   bool on = false;
   cudaStream_t st;
   ProfRec r{};
+  unsigned flags = cudaEventRecordDefault;
   ProfScope(const char* tag, cudaStream_t s) : st(s) {
     if (!prof_wanted(tag)) return;
     r.tag = tag;
     if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) return;
-    on = cudaEventRecord(r.a, st) == cudaSuccess;
+    // inside a stream capture the events become event-record nodes of the graph
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+      flags = cudaEventRecordExternal;
+    on = cudaEventRecordWithFlags(r.a, st, flags) == cudaSuccess;
   }
   ~ProfScope() {
     if (!on) return;
-    cudaEventRecord(r.b, st);
+    cudaEventRecordWithFlags(r.b, st, flags);
     g_prof.push_back(r);
   }
 };
@@ -241,7 +246,8 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
 template <typename T>
 static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32_t* perm,
                                   const void* w_g, const void* w_u, const void* w_o, void* eo,
-                                  void* ws, cudaStream_t st, bool rows_sorted = false) {
+                                  void* ws, cudaStream_t st, bool rows_sorted = false,
+                                  int max_ctas = 0) {
   const Layout L = layout(d, false);
   const int64_t P = d->n_tokens * d->top_k;
   if (P == 0) return LMOE_OK;
@@ -263,7 +269,7 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   int32_t* status = &at<WsHeader>(ws, L.header)->status;
   RoutedArgs ra{};
   ra.P = P; ra.L = Lt; ra.F = F; ra.R = d->n_routed; ra.tiles = tiles; ra.n_mtiles = n_tiles;
-  ra.max_tiles = L.max_tiles; ra.beta1 = d->beta1; ra.beta2 = d->beta2;
+  ra.max_tiles = L.max_tiles; ra.beta1 = d->beta1; ra.beta2 = d->beta2; ra.max_units = max_ctas;
   {
     ProfScope ps("expert_gemm1", st);
     if (tc) {
@@ -292,6 +298,71 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   return LMOE_OK;
 }
 
+// bf16 forward on the tensor cores, one stream: the x-pass (z, routing and the
+// shared experts' hidden units), dispatch, the routed experts, combine +
+// RMSNorm, and one GEMM for y = shared + W_up RMSNorm(u).
+static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, const void* x,
+                                  void* y, int32_t* ids_out, float* probs_out, int32_t* counts_out,
+                                  void* ws, cudaStream_t st) {
+  typedef __nv_bfloat16 T;
+  const Layout L = layout(d, false);
+  const int64_t N = d->n_tokens;
+  const int Lt = d->latent, S = d->n_shared, G = d->ff_shared, D = d->d, R = d->n_routed;
+  const int k = d->top_k;
+  int32_t* ids = ids_out ? ids_out : at<int32_t>(ws, L.ids);
+  float* probs = probs_out ? probs_out : at<float>(ws, L.probs);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  T* z = at<T>(ws, L.z);
+  T* hsh = at<T>(ws, L.hsh);
+  T* eo = at<T>(ws, L.eo);
+  T* uhat = at<T>(ws, L.uhat);
+  float* logits = at<float>(ws, L.logits);
+  int32_t* status = &at<WsHeader>(ws, L.header)->status;
+  if (N == 0) {
+    LMOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * R, st), "memset");
+    return LMOE_OK;
+  }
+  // steps 1, 2 and 4 in one pass over x (routing in the epilogue when R <= 32)
+  {
+    XpassArgs a{};
+    a.x = (const T*)x; a.N = N; a.d = D;
+    a.w_down = (const T*)w->w_down; a.L = Lt;
+    a.w_router = (const T*)w->w_router; a.R = R;
+    a.ws_g = (const T*)w->ws_g; a.ws_u = (const T*)w->ws_u; a.S = S; a.G = G;
+    a.z = z; a.logits = logits; a.logits_ld = L.logits_ld;
+    a.hsh = hsh; a.beta1 = d->beta1; a.beta2 = d->beta2;
+    a.bias = w->expert_bias; a.ids = ids; a.probs = probs; a.top_k = k;
+    ProfScope ps("xpass", st);
+    LMOE_CUDA(umma_xpass(a, status, st), "x-pass (tcgen05)");
+  }
+  if (R > 32) {
+    ProfScope ps("route", st);
+    LMOE_CUDA(launch_route_topk(logits, L.logits_ld, w->expert_bias, N, R, k, ids, probs, st),
+              "route_topk");
+  }
+  // step 3: dispatch, routed experts, combine + RMSNorm
+  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st));
+  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st));
+  {
+    ProfScope ps("combine", st);
+    LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, k, Lt, d->rms_eps, uhat, st),
+              "combine");
+  }
+  // step 5: y = shared + W_up uhat in one accumulator
+  {
+    FinalArgs a{};
+    a.hsh = hsh; a.N = N; a.S = S; a.G = G; a.ws_o = (const T*)w->ws_o; a.d = D;
+    a.uhat = uhat; a.L = Lt; a.w_up = (const T*)w->w_up; a.y = (T*)y;
+    ProfScope ps("final", st);
+    LMOE_CUDA(umma_final(a, status, st), "final (tcgen05)");
+  }
+  return LMOE_OK;
+}
+
+// fp32 forward on the CUDA cores (the debug/reference-precision mode).
 template <typename T>
 static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const void* x, void* y,
                                int32_t* ids_out, float* probs_out, int32_t* counts_out, void* ws,
@@ -310,58 +381,31 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
   T* eo = at<T>(ws, L.eo);
   T* uhat = at<T>(ws, L.uhat);
   if (N == 0) {
-    // still produce zero counts
     LMOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * d->n_routed, st), "memset");
     return LMOE_OK;
   }
-  const bool tc = std::is_same<T, __nv_bfloat16>::value;
-  int32_t* status = &at<WsHeader>(ws, L.header)->status;
-  float* logits = at<float>(ws, L.logits);
-  if (tc) {
-    // steps 1, 2 (logits) and 4 (shared hidden units) in one tcgen05 pass over x
-    XpassArgs a{};
-    a.x = (const __nv_bfloat16*)x; a.N = N; a.d = D;
-    a.w_down = (const __nv_bfloat16*)w->w_down; a.L = Lt;
-    a.w_router = (const __nv_bfloat16*)w->w_router; a.R = d->n_routed;
-    a.ws_g = (const __nv_bfloat16*)w->ws_g; a.ws_u = (const __nv_bfloat16*)w->ws_u; a.S = S; a.G = G;
-    a.z = (__nv_bfloat16*)z; a.logits = logits; a.logits_ld = L.logits_ld;
-    a.hsh = (__nv_bfloat16*)hsh; a.beta1 = d->beta1; a.beta2 = d->beta2;
-    a.bias = w->expert_bias; a.ids = ids; a.probs = probs; a.top_k = d->top_k;
+  // step 1: z = W_down x
+  {
+    SimtGemm g{};
+    g.A[0] = x; g.lda[0] = D; g.B[0] = w->w_down; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
+    g.C = z; g.ldc = Lt; g.M = (int)N; g.N = Lt; g.mode = kStore;
     ProfScope ps("xpass", st);
-    LMOE_CUDA(umma_xpass(a, status, st), "x-pass (tcgen05)");
-  } else {
-    // step 1: z = W_down x
-    {
-      SimtGemm g{};
-      g.A[0] = x; g.lda[0] = D; g.B[0] = w->w_down; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
-      g.C = z; g.ldc = Lt; g.M = (int)N; g.N = Lt; g.mode = kStore;
-      ProfScope ps("xpass", st);
-      LMOE_CUDA(launch_simt_gemm<T>(g, st), "down");
-    }
-    // step 4 (independent of routing): h_sh = SiTU hidden of the shared experts
-    if (S > 0) {
-      SimtGemm g{};
-      g.A[0] = x; g.lda[0] = D; g.B[0] = w->ws_g; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
-      g.B_up = w->ws_u; g.C = hsh; g.ldc = (int64_t)S * G; g.M = (int)N; g.N = S * G;
-      g.beta1 = d->beta1; g.beta2 = d->beta2; g.mode = kSitu;
-      ProfScope ps("xpass", st);
-      LMOE_CUDA(launch_simt_gemm<T>(g, st), "shared gemm1");
-    }
+    LMOE_CUDA(launch_simt_gemm<T>(g, st), "down");
   }
-  // step 2: routing (top-k + normalisation from the x-pass logits on the tcgen05 path)
-  if (tc) {
-    if (d->n_routed > 32) {  // R <= 32 is routed inside the x-pass epilogue
-      ProfScope ps("route", st);
-      LMOE_CUDA(launch_route_topk(logits, L.logits_ld, w->expert_bias, N, d->n_routed, d->top_k,
-                                  ids, probs, st),
-                "route_topk");
-    }
-  } else {
-    LMOE_TRY(run_route<T>(d, x, w->w_router, w->expert_bias, ids, probs, ws, st));
+  // step 4 (independent of routing): h_sh = SiTU hidden of the shared experts
+  if (S > 0) {
+    SimtGemm g{};
+    g.A[0] = x; g.lda[0] = D; g.B[0] = w->ws_g; g.ldb[0] = D; g.K[0] = D; g.nseg = 1;
+    g.B_up = w->ws_u; g.C = hsh; g.ldc = (int64_t)S * G; g.M = (int)N; g.N = S * G;
+    g.beta1 = d->beta1; g.beta2 = d->beta2; g.mode = kSitu;
+    ProfScope ps("xpass", st);
+    LMOE_CUDA(launch_simt_gemm<T>(g, st), "shared gemm1");
   }
+  // step 2: routing
+  LMOE_TRY(run_route<T>(d, x, w->w_router, w->expert_bias, ids, probs, ws, st));
   // step 3: dispatch, routed experts, combine + RMSNorm
-  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, z));
-  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st, true));
+  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st));
+  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st));
   {
     ProfScope ps("combine", st);
     LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, d->top_k, Lt, d->rms_eps, uhat,
@@ -369,14 +413,7 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
               "combine");
   }
   // step 5: y = sum_j W_o,sh_j h_sh_j + W_up uhat
-  if (tc) {
-    FinalArgs a{};
-    a.hsh = (const __nv_bfloat16*)hsh; a.N = N; a.S = S; a.G = G;
-    a.ws_o = (const __nv_bfloat16*)w->ws_o; a.d = D; a.uhat = (const __nv_bfloat16*)uhat; a.L = Lt;
-    a.w_up = (const __nv_bfloat16*)w->w_up; a.y = (__nv_bfloat16*)y;
-    ProfScope ps("final", st);
-    LMOE_CUDA(umma_final(a, status, st), "final (tcgen05)");
-  } else {
+  {
     SimtGemm g{};
     int s = 0;
     for (int j = 0; j < S; ++j, ++s) {
@@ -531,7 +568,7 @@ lmoe_status latent_moe_forward(const lmoe_dims* dims, const lmoe_weights* weight
   LMOE_TRY(check_device());
   cudaStream_t st = (cudaStream_t)stream;
   if (dims->dtype == LMOE_BF16)
-    return run_forward<__nv_bfloat16>(dims, weights, x, y, ids_out, probs_out, counts_out, ws, st);
+    return run_forward_tc(dims, weights, x, y, ids_out, probs_out, counts_out, ws, st);
   return run_forward<float>(dims, weights, x, y, ids_out, probs_out, counts_out, ws, st);
 }
 
@@ -552,7 +589,7 @@ lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_weights* w
   if (bytes) LMOE_CUDA(cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st), "H2D x");
   lmoe_status s;
   if (dims->dtype == LMOE_BF16)
-    s = run_forward<__nv_bfloat16>(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st);
+    s = run_forward_tc(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st);
   else
     s = run_forward<float>(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st);
   if (s != LMOE_OK) return s;
@@ -652,6 +689,22 @@ lmoe_status lmoe_profile_read_tag(const char* tag, double* total_ms, int64_t* la
     cudaEventDestroy(r.b);
   }
   g_prof.swap(keep);
+  if (total_ms) *total_ms = tot;
+  if (launches) *launches = n;
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_profile_peek_tag(const char* tag, double* total_ms, int64_t* launches) {
+  double tot = 0.0;
+  int64_t n = 0;
+  for (auto& r : g_prof) {
+    if (tag != nullptr && r.tag != tag) continue;
+    float ms = 0.0f;
+    LMOE_CUDA(cudaEventSynchronize(r.b), "event sync");
+    LMOE_CUDA(cudaEventElapsedTime(&ms, r.a, r.b), "elapsed");
+    tot += ms;
+    ++n;
+  }
   if (total_ms) *total_ms = tot;
   if (launches) *launches = n;
   return LMOE_OK;

@@ -7,6 +7,7 @@
 // the result is deterministic.  Rows are read with 16-byte vectors.
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.h"
 
 namespace lmoe {
 namespace {
@@ -17,6 +18,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ eo,
                                                       const float* __restrict__ probs,
                                                       const float* __restrict__ rms_w, int64_t n,
                                                       int k, int L, float eps, T* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int E = 16 / sizeof(T);  // elements per vector
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -74,6 +77,8 @@ __global__ void __launch_bounds__(128) combine_block_kernel(const T* __restrict_
                                                             const float* __restrict__ rms_w,
                                                             int k, int L, float eps,
                                                             T* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int E = 16 / sizeof(T);
   constexpr int UNROLL = 4;
   __shared__ float red[4];
@@ -152,10 +157,9 @@ cudaError_t launch_combine(const T* eo, const int32_t* inv_pair, const float* pr
     const int vpt = (nvec + 127) / 128;
 #define LMOE_COMBINE_BLOCK_CASE(V)                                                     \
     if (vpt <= V) {                                                                    \
-      combine_block_kernel<T, V><<<(unsigned)n, 128, 0, st>>>(eo, inv_pair, probs, rms_w, k, L, \
-                                                              eps, out);               \
       count_launch();                                                                  \
-      return cudaGetLastError();                                                       \
+      return launch_pdl(combine_block_kernel<T, V>, dim3((unsigned)n), dim3(128), 0, st, 1, eo, \
+                        inv_pair, probs, rms_w, k, L, eps, out);                       \
     }
     LMOE_COMBINE_BLOCK_CASE(2)
     LMOE_COMBINE_BLOCK_CASE(4)
@@ -166,10 +170,9 @@ cudaError_t launch_combine(const T* eo, const int32_t* inv_pair, const float* pr
   unsigned blocks = (unsigned)((n + warps - 1) / warps);
 #define LMOE_COMBINE_CASE(V)                                                              \
   if (vpl <= V) {                                                                         \
-    combine_kernel<T, V><<<blocks, warps * 32, 0, st>>>(eo, inv_pair, probs, rms_w, n, k, L, \
-                                                        eps, out);                        \
     count_launch();                                                                       \
-    return cudaGetLastError();                                                            \
+    return launch_pdl(combine_kernel<T, V>, dim3(blocks), dim3(warps * 32), 0, st, 1, eo,    \
+                      inv_pair, probs, rms_w, n, k, L, eps, out);                         \
   }
   LMOE_COMBINE_CASE(1)
   LMOE_COMBINE_CASE(2)

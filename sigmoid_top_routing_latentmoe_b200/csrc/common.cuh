@@ -43,4 +43,14 @@ __device__ __forceinline__ float situ_exact(float a, float c, float beta1, float
   return gate * up;
 }
 
+// Programmatic dependent launch: every kernel of the library lets the next
+// kernel in its stream launch as soon as all of its CTAs have started
+// (pdl_trigger), and waits for the previous kernel to complete -- memory
+// included -- before it touches anything (pdl_wait).  Both are no-ops when
+// the kernel was launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 }  // namespace lmoe

@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.h"
 
 namespace lmoe {
 namespace {
@@ -34,6 +35,8 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const int32_t* __restric
                                                         int64_t n_pairs, int64_t chunk, int R,
                                                         int32_t* __restrict__ chunk_counts,
                                                         int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int32_t hist[];
   for (int e = threadIdx.x; e < R; e += kThreads) hist[e] = 0;
   __syncthreads();
@@ -93,6 +96,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
                                                     int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ n_mtiles,
                                                     int4* __restrict__ tiles) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t totals[2];
   __shared__ int32_t carry[2];
@@ -138,6 +143,8 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
     const int32_t* __restrict__ chunk_first, const int32_t* __restrict__ offsets,
     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair, const uint4* __restrict__ z,
     uint4* __restrict__ zp, int row_vecs) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int32_t wcnt[];  // [kWarps][R]: per-warp counts, then first slots
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * R; i += kThreads) wcnt[i] = 0;
@@ -199,6 +206,8 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
 template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ z, const int32_t* __restrict__ perm_token,
                                    int64_t n_rows, int width, T* __restrict__ zp) {
+  pdl_trigger();
+  pdl_wait();
   // one warp per row, 16-byte vectors
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -214,6 +223,8 @@ __global__ void gather_rows_kernel(const T* __restrict__ z, const int32_t* __res
 // warp: each lane scans a contiguous run of experts.
 __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int R,
                                    int32_t* __restrict__ n_mtiles, int4* __restrict__ tiles) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x;
   const int per = (R + 31) / 32;
   const int e0 = min(R, lane * per), e1 = min(R, e0 + per);
@@ -257,21 +268,24 @@ cudaError_t launch_dispatch_gather(const int32_t* ids, int64_t n, int k, int R, 
   if (nb > 0) {
     cudaError_t e = set_smem(hist_kernel, R * sizeof(int32_t));
     if (e != cudaSuccess) return e;
-    hist_kernel<<<nb, kThreads, R * sizeof(int32_t), st>>>(ids, n_pairs, chunk, R,
-                                                           s.block_counts, s.status);
+    e = launch_pdl(hist_kernel, dim3(nb), dim3(kThreads), R * sizeof(int32_t), st, 1, ids, n_pairs,
+                   chunk, R, s.block_counts, s.status);
     count_launch();
+    if (e != cudaSuccess) return e;
   }
-  scan_kernel<<<1, 1024, 0, st>>>(s.block_counts, nb, R, counts, offsets, s.n_mtiles, s.tiles);
+  cudaError_t e2 = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, 1, s.block_counts, nb, R,
+                              counts, offsets, s.n_mtiles, s.tiles);
   count_launch();
+  if (e2 != cudaSuccess) return e2;
   if (nb > 0) {
     const size_t smem = (size_t)kWarps * R * sizeof(int32_t);
     cudaError_t e = set_smem(scatter_kernel, smem);
     if (e != cudaSuccess) return e;
-    scatter_kernel<<<nb, kThreads, smem, st>>>(ids, n_pairs, chunk, k, R, s.block_counts, offsets,
-                                               perm_token, inv_pair,
-                                               static_cast<const uint4*>(z),
-                                               static_cast<uint4*>(zp), row_bytes / 16);
+    e = launch_pdl(scatter_kernel, dim3(nb), dim3(kThreads), smem, st, 1, ids, n_pairs, chunk, k,
+                   R, (const int32_t*)s.block_counts, (const int32_t*)offsets, perm_token, inv_pair,
+                   static_cast<const uint4*>(z), static_cast<uint4*>(zp), row_bytes / 16);
     count_launch();
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -285,9 +299,8 @@ cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
                                cudaStream_t st) {
-  build_tiles_kernel<<<1, 32, 0, st>>>(offsets, R, n_mtiles, tiles);
   count_launch();
-  return cudaGetLastError();
+  return launch_pdl(build_tiles_kernel, dim3(1), dim3(32), 0, st, 1, offsets, R, n_mtiles, tiles);
 }
 
 template <typename T>
@@ -295,10 +308,9 @@ cudaError_t launch_gather_rows(const T* z, const int32_t* perm_token, int64_t n_
                                T* zp, cudaStream_t st) {
   if (n_rows == 0) return cudaSuccess;
   const int warps = 8;
-  gather_rows_kernel<T><<<(unsigned)((n_rows + warps - 1) / warps), warps * 32, 0, st>>>(
-      z, perm_token, n_rows, width, zp);
   count_launch();
-  return cudaGetLastError();
+  return launch_pdl(gather_rows_kernel<T>, dim3((unsigned)((n_rows + warps - 1) / warps)),
+                    dim3(warps * 32), 0, st, 1, z, perm_token, n_rows, width, zp);
 }
 template cudaError_t launch_gather_rows<float>(const float*, const int32_t*, int64_t, int, float*,
                                                cudaStream_t);

@@ -5,6 +5,7 @@
 // order; equal keys go to the lower expert index.
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.h"
 
 namespace lmoe {
 namespace {
@@ -87,6 +88,8 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(const T* __restrict__ x
                                                          int d, int R, int k,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ probs) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int E = 16 / sizeof(T);  // elements per 16-byte vector
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -134,6 +137,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
                                                          int64_t n, int R, int k,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ probs) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= n) return;
@@ -157,14 +162,15 @@ cudaError_t launch_route_gemv(const T* x, const T* w_r, const float* bias, int64
   if (n == 0) return cudaSuccess;
   const int warps = 8;
   int64_t blocks = (n + warps - 1) / warps;
+  cudaError_t e;
   if (R <= 16)
-    route_gemv_kernel<T, 16><<<(unsigned)blocks, warps * 32, 0, st>>>(x, w_r, bias, n, d, R, k, ids,
-                                                                       probs);
+    e = launch_pdl(route_gemv_kernel<T, 16>, dim3((unsigned)blocks), dim3(warps * 32), 0, st, 1, x,
+                   w_r, bias, n, d, R, k, ids, probs);
   else
-    route_gemv_kernel<T, 32><<<(unsigned)blocks, warps * 32, 0, st>>>(x, w_r, bias, n, d, R, k, ids,
-                                                                       probs);
+    e = launch_pdl(route_gemv_kernel<T, 32>, dim3((unsigned)blocks), dim3(warps * 32), 0, st, 1, x,
+                   w_r, bias, n, d, R, k, ids, probs);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 template cudaError_t launch_route_gemv<float>(const float*, const float*, const float*, int64_t,
                                               int, int, int, int32_t*, float*, cudaStream_t);
@@ -180,9 +186,9 @@ cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias
   int vpl = (R + 31) / 32;
 #define LMOE_TOPK_CASE(V)                                                                  \
   if (vpl <= V) {                                                                          \
-    route_topk_kernel<V><<<blocks, warps * 32, 0, st>>>(logits, ld, bias, n, R, k, ids, probs); \
     count_launch();                                                                        \
-    return cudaGetLastError();                                                             \
+    return launch_pdl(route_topk_kernel<V>, dim3(blocks), dim3(warps * 32), 0, st, 1, logits, \
+                      ld, bias, n, R, k, ids, probs);                                     \
   }
   LMOE_TOPK_CASE(1)
   LMOE_TOPK_CASE(2)

@@ -33,6 +33,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "umma_gemm.h"
+#include "launch.h"
 
 namespace lmoe {
 namespace {
@@ -204,17 +205,6 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
          (2ull << 61);
-}
-// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = n.
-__device__ __forceinline__ uint32_t instr_desc(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(BM >> 4) << 24);
-}
-
-__device__ __forceinline__ float tanh_fast(float v) {
-  float r;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
-  return r;
 }
 __device__ __forceinline__ uint32_t tanh_h2(uint32_t v) {
   uint32_t r;
@@ -793,6 +783,9 @@ __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_cons
   if (CG == 2) cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // everything above overlaps the previous kernel; inputs are read only below
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0)
@@ -894,26 +887,9 @@ static cudaError_t launch(const Params& p, int grid, cudaStream_t st) {
     attr = true;
   }
   if (grid <= 0) return cudaSuccess;
-  if (CG == 1) {
-    umma_gemm_kernel<MODE, 1><<<grid, THREADS, Cfg<CG>::SMEM_BYTES, st>>>(p);
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * grid, 1, 1);
-    cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = Cfg<CG>::SMEM_BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute attrs[1];
-    attrs[0].id = cudaLaunchAttributeClusterDimension;
-    attrs[0].val.clusterDim.x = 2;
-    attrs[0].val.clusterDim.y = 1;
-    attrs[0].val.clusterDim.z = 1;
-    cfg.attrs = attrs;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, umma_gemm_kernel<MODE, CG>, p);
-    if (e != cudaSuccess) return e;
-  }
   count_launch();
-  return cudaGetLastError();
+  return launch_pdl(umma_gemm_kernel<MODE, CG>, dim3(CG * grid), dim3(THREADS),
+                    (size_t)Cfg<CG>::SMEM_BYTES, st, CG, p);
 }
 
 // Tile width for the plain-store GEMMs: the one of 256, 192, 128 columns that
@@ -982,14 +958,16 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   p.ids = a.ids;
   p.probs = a.probs;
   const int total = (int)((a.N + 2 * BM - 1) / (2 * BM)) * p.n_tiles;
-  return launch<XPASS, 2>(p, std::min(total, num_sms() / 2), st);
+  const int units = a.max_units > 0 ? std::min(a.max_units, num_sms() / 2) : num_sms() / 2;
+  return launch<XPASS, 2>(p, std::min(total, units), st);
 }
 
 cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
   if (a.N == 0) return cudaSuccess;
   Params p = base_params(status);
   const int m_tiles = (int)((a.N + 2 * BM - 1) / (2 * BM));
-  p.bn = pick_bn(m_tiles, a.d, num_sms() / 2);
+  const int units = a.max_units > 0 ? std::min(a.max_units, num_sms() / 2) : num_sms() / 2;
+  p.bn = pick_bn(m_tiles, a.d, units);
   const uint32_t hb = p.bn / 2;  // rows of B each CTA of the pair loads
   bool ok = make_map(&p.tmA1, a.uhat, a.L, a.N, 1, BM) && make_map(&p.tmB1, a.w_up, a.L, a.d, 1, hb) &&
             make_map(&p.tmB3, a.w_up, a.L, a.d, 1, hb);
@@ -1009,7 +987,7 @@ cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
   p.out0 = a.y;
   p.ld0 = a.d;
   const int total = m_tiles * p.n_tiles;
-  return launch<FINAL, 2>(p, std::min(total, num_sms() / 2), st);
+  return launch<FINAL, 2>(p, std::min(total, units), st);
 }
 
 cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) {
@@ -1033,13 +1011,15 @@ cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   p.inv_beta2 = 1.0f / a.beta2;
   p.beta12 = a.beta1 * a.beta2;
   const int64_t bound = (int64_t)a.max_tiles * p.n_tiles;
-  return launch<ROUTED1, 1>(p, (int)std::min<int64_t>(bound, num_sms()), st);
+  const int units = a.max_units > 0 ? std::min(a.max_units, num_sms()) : num_sms();
+  return launch<ROUTED1, 1>(p, (int)std::min<int64_t>(bound, units), st);
 }
 
 cudaError_t umma_routed2(const RoutedArgs& a, int32_t* status, cudaStream_t st) {
   if (a.P == 0) return cudaSuccess;
   Params p = base_params(status);
-  p.bn = pick_bn((int)((a.P + BM - 1) / BM) + a.R / 2, a.L, num_sms());
+  const int cap = a.max_units > 0 ? std::min(a.max_units, num_sms()) : num_sms();
+  p.bn = pick_bn((int)((a.P + BM - 1) / BM) + a.R / 2, a.L, cap);
   bool ok = make_map(&p.tmA0, a.a, a.F, a.P, 1, BM) && make_map3(&p.tmB0, a.w0, a.F, a.L, a.R, SUB) &&
             (p.bn == SUB || make_map3(&p.tmB1, a.w0, a.F, a.L, a.R, p.bn - SUB));
   if (!ok) return cudaErrorInvalidValue;
@@ -1053,7 +1033,8 @@ cudaError_t umma_routed2(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   p.tiles = a.tiles;
   p.n_mtiles = a.n_mtiles;
   const int64_t bound = (int64_t)a.max_tiles * p.n_tiles;
-  return launch<ROUTED2, 1>(p, (int)std::min<int64_t>(bound, num_sms()), st);
+  const int units = a.max_units > 0 ? std::min(a.max_units, num_sms()) : num_sms();
+  return launch<ROUTED2, 1>(p, (int)std::min<int64_t>(bound, units), st);
 }
 
 }  // namespace lmoe

@@ -33,6 +33,7 @@ struct XpassArgs {
   int32_t* ids;
   float* probs;
   int top_k;
+  int max_units;  // at most this many CTA pairs (0: one per pair of SMs)
 };
 
 // final: y [N, d] = sum_j hsh[:, jG:(j+1)G] W_o,sh_j^T + uhat W_up^T
@@ -46,6 +47,7 @@ struct FinalArgs {
   int L;
   const __nv_bfloat16* w_up;  // [d, L]
   __nv_bfloat16* y;
+  int max_units;  // at most this many CTA pairs (0: one per pair of SMs)
 };
 
 // routed GEMM1: h [P, F] = SiTU(zp W_g,e^T, zp W_u,e^T) per row tile of expert e
@@ -61,6 +63,7 @@ struct RoutedArgs {
   const int32_t* n_mtiles;
   int max_tiles;
   float beta1, beta2;
+  int max_units;  // at most this many CTAs (0: one per SM)
 };
 
 cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st);
