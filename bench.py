@@ -45,6 +45,24 @@ def _peaks():
 
 
 # Algorithmic work of each kernel (per launch, full workload): FLOPs or bytes.
+def measured_traffic(wl: synth.Workload, tag: str):
+    """DRAM bytes per launch of kernel `tag` from the committed ncu capture, or
+    None when there is none for this workload or the kernel source changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(tag)
+    if not rec or rec.get("workload") != wl.name:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None
+    return float(rec["dram_bytes_per_launch"])
+
+
 def kernel_work(wl: synth.Workload, tag: str):
     N, d, L, R, k, F, S, G = (wl.n_tokens, wl.d, wl.latent, wl.n_routed, wl.top_k, wl.ff_routed,
                               wl.n_shared, wl.ff_shared)
@@ -377,7 +395,7 @@ def main():
             peak = peaks["hbm_gbs"]
             unit = "GB/s"
         roof = {"kernel": prof_tag, "bound": bound, "achieved": achieved, "peak": peak,
-                "unit": unit, "frac": achieved / peak, "traffic": None,
+                "unit": unit, "frac": achieved / peak, "traffic": measured_traffic(wl, prof_tag),
                 "launch_us": k_avg_s * 1e6, "launches": k_n,
                 "peak_source": peaks["source"] + (" sustained" if bound == "tensor" else "")}
     else:
