@@ -63,7 +63,8 @@ typedef void* lmoe_stream; /* cudaStream_t */
 /* Layer sizes (the pages' LatentMoE(hidden_size, latent_size, n_routed, top_k,
  * n_shared, d_ff, beta1, beta2) with B*T flattened to n_tokens and separate
  * routed/shared hidden widths).  Limits: 1 <= top_k <= n_routed <= 4096;
- * d, latent, ff_routed, ff_shared multiples of 64 (bf16) or 8 (fp32);
+ * d, latent, ff_routed, ff_shared multiples of 8 (ragged 64-wide K blocks
+ * and output tiles are zero-filled / masked on the tensor-core path);
  * 0 <= n_shared <= 7; n_tokens * top_k < 2^31. */
 typedef struct {
   int64_t n_tokens; /* N                                    */

@@ -233,6 +233,7 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
   s.block_counts = at<int32_t>(ws, L.block_counts);
   s.status = &at<WsHeader>(ws, L.header)->status;
   s.n_mtiles = &at<WsHeader>(ws, L.header)->n_mtiles;
+  s.ticket = &at<WsHeader>(ws, L.header)->ticket;
   s.tiles = at<int4>(ws, L.tiles);
   const int es = d->dtype == LMOE_BF16 ? 2 : 4;
   ProfScope ps("dispatch", st);
@@ -243,11 +244,12 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
 }
 
 // Routed experts on sorted pairs; the tile list must already be in the workspace.
+// perm holds the token of each sorted pair: its rows of z are first copied in
+// sorted order, the A operand of GEMM1.
 template <typename T>
 static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32_t* perm,
                                   const void* w_g, const void* w_u, const void* w_o, void* eo,
-                                  void* ws, cudaStream_t st, bool rows_sorted = false,
-                                  int max_ctas = 0) {
+                                  void* ws, cudaStream_t st) {
   const Layout L = layout(d, false);
   const int64_t P = d->n_tokens * d->top_k;
   if (P == 0) return LMOE_OK;
@@ -256,7 +258,8 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   T* h = at<T>(ws, L.h);
   const int4* tiles = at<int4>(ws, L.tiles);
   const int32_t* n_tiles = &at<WsHeader>(ws, L.header)->n_mtiles;
-  if (!rows_sorted) {
+  const bool tc = std::is_same<T, __nv_bfloat16>::value;
+  {
     ProfScope ps("gather", st);
     LMOE_CUDA(launch_gather_rows<T>((const T*)z, perm, P, Lt, zp, st), "gather");
   }
@@ -265,11 +268,10 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   g1.B_up = w_u; g1.b_expert_stride = (int64_t)F * Lt;
   g1.C = h; g1.ldc = F; g1.N = F; g1.tiles = tiles; g1.n_tiles = n_tiles;
   g1.max_tiles = L.max_tiles; g1.beta1 = d->beta1; g1.beta2 = d->beta2; g1.mode = kSitu;
-  const bool tc = std::is_same<T, __nv_bfloat16>::value;
   int32_t* status = &at<WsHeader>(ws, L.header)->status;
   RoutedArgs ra{};
   ra.P = P; ra.L = Lt; ra.F = F; ra.R = d->n_routed; ra.tiles = tiles; ra.n_mtiles = n_tiles;
-  ra.max_tiles = L.max_tiles; ra.beta1 = d->beta1; ra.beta2 = d->beta2; ra.max_units = max_ctas;
+  ra.max_tiles = L.max_tiles; ra.beta1 = d->beta1; ra.beta2 = d->beta2;
   {
     ProfScope ps("expert_gemm1", st);
     if (tc) {

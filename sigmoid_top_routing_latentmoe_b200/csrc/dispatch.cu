@@ -31,35 +31,6 @@ int64_t chunk_pairs(int64_t n_pairs) {
   return std::max<int64_t>(step, (per + step - 1) / step * step);
 }
 
-__global__ void __launch_bounds__(kThreads) hist_kernel(const int32_t* __restrict__ ids,
-                                                        int64_t n_pairs, int64_t chunk, int R,
-                                                        int32_t* __restrict__ chunk_counts,
-                                                        int32_t* __restrict__ status) {
-  pdl_trigger();
-  pdl_wait();
-  extern __shared__ int32_t hist[];
-  for (int e = threadIdx.x; e < R; e += kThreads) hist[e] = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t per_warp = chunk / kWarps;
-  const int64_t p0 = (int64_t)blockIdx.x * chunk + warp * per_warp;
-  const int64_t p1 = min(n_pairs, p0 + per_warp);
-  for (int64_t q = p0; q < p1; q += 32) {
-    const int64_t p = q + lane;
-    int e = p < p1 ? ids[p] : -1;
-    if (p < p1 && (unsigned)e >= (unsigned)R) {
-      record_status(status, kStatusDevice);
-      e = -1;
-    }
-    // one shared-memory add per distinct expert among the warp's 32 pairs
-    const unsigned same = __match_any_sync(0xffffffffu, e < 0 ? -1 - lane : e);
-    if (e >= 0 && (same & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[e], __popc(same));
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < R; e += kThreads)
-    chunk_counts[(int64_t)blockIdx.x * R + e] = hist[e];
-}
-
 // Block-wide exclusive scan of one value per thread; *total gets the sum.
 __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_sums,
                                                         int32_t* total) {
@@ -88,16 +59,13 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return excl;
 }
 
-// One CTA of 1024 threads.  chunk_counts[c, e] becomes the number of pairs of
-// expert e in chunks before c.
-__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_counts,
-                                                    int n_chunks, int R,
-                                                    int32_t* __restrict__ counts,
-                                                    int32_t* __restrict__ offsets,
-                                                    int32_t* __restrict__ n_mtiles,
-                                                    int4* __restrict__ tiles) {
-  pdl_trigger();
-  pdl_wait();
+// Run by one CTA (any size): chunk_counts[c, e] becomes the number of pairs
+// of expert e in chunks before c; writes counts, offsets and the tile list.
+// Each thread owns whole experts and reads their chunk column 16 loads at a
+// time, so the loads are in flight together.
+__device__ void scan_chunks(int32_t* __restrict__ chunk_counts, int n_chunks, int R,
+                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                            int32_t* __restrict__ n_mtiles, int4* __restrict__ tiles) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t totals[2];
   __shared__ int32_t carry[2];
@@ -106,10 +74,16 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
     const int e = base + threadIdx.x;
     int32_t c = 0;
     if (e < R) {
-      for (int b = 0; b < n_chunks; ++b) {
-        const int32_t v = chunk_counts[(int64_t)b * R + e];
-        chunk_counts[(int64_t)b * R + e] = c;
-        c += v;
+      for (int b0 = 0; b0 < n_chunks; b0 += 16) {
+        int32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          v[j] = b0 + j < n_chunks ? chunk_counts[(int64_t)(b0 + j) * R + e] : 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (b0 + j < n_chunks) chunk_counts[(int64_t)(b0 + j) * R + e] = c;
+          c += v[j];
+        }
       }
     }
     __syncthreads();
@@ -133,6 +107,61 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ chunk_
     offsets[R] = carry[0];
     *n_mtiles = carry[1];
   }
+}
+
+// One CTA per chunk counts the chunk's pairs per expert; the last CTA to
+// finish (an atomic ticket in the workspace header, reset by that CTA) then
+// runs the scan over all chunks.
+__global__ void __launch_bounds__(kThreads) hist_scan_kernel(
+    const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int R,
+    int32_t* __restrict__ chunk_counts, int32_t* __restrict__ status, int32_t* __restrict__ ticket,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ n_mtiles,
+    int4* __restrict__ tiles) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ int32_t hist[];
+  __shared__ int32_t last;
+  for (int e = threadIdx.x; e < R; e += kThreads) hist[e] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t per_warp = chunk / kWarps;
+  const int64_t p0 = (int64_t)blockIdx.x * chunk + warp * per_warp;
+  const int64_t p1 = min(n_pairs, p0 + per_warp);
+  for (int64_t q = p0; q < p1; q += 32) {
+    const int64_t p = q + lane;
+    int e = p < p1 ? ids[p] : -1;
+    if (p < p1 && (unsigned)e >= (unsigned)R) {
+      record_status(status, kStatusDevice);
+      e = -1;
+    }
+    // one shared-memory add per distinct expert among the warp's 32 pairs
+    const unsigned same = __match_any_sync(0xffffffffu, e < 0 ? -1 - lane : e);
+    if (e >= 0 && (same & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[e], __popc(same));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < R; e += kThreads)
+    chunk_counts[(int64_t)blockIdx.x * R + e] = hist[e];
+  // publish this chunk, then take a ticket; the last ticket scans
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  scan_chunks(chunk_counts, gridDim.x, R, counts, offsets, n_mtiles, tiles);
+  if (threadIdx.x == 0) *ticket = 0;  // ready for the next call
+}
+
+// No pairs at all: every count and offset is zero, no tiles.
+__global__ void empty_scan_kernel(int R, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                  int32_t* __restrict__ n_mtiles) {
+  pdl_trigger();
+  pdl_wait();
+  for (int e = threadIdx.x; e <= R; e += blockDim.x) {
+    if (e < R) counts[e] = 0;
+    offsets[e] = 0;
+  }
+  if (threadIdx.x == 0) *n_mtiles = 0;
 }
 
 // Ranks each chunk's pairs inside their expert in pair order and scatters.
@@ -265,18 +294,20 @@ cudaError_t launch_dispatch_gather(const int32_t* ids, int64_t n, int k, int R, 
   const int64_t n_pairs = n * k;
   const int64_t chunk = chunk_pairs(n_pairs);
   const int nb = dispatch_blocks(n_pairs);
+  cudaError_t e0;
   if (nb > 0) {
-    cudaError_t e = set_smem(hist_kernel, R * sizeof(int32_t));
+    cudaError_t e = set_smem(hist_scan_kernel, R * sizeof(int32_t));
     if (e != cudaSuccess) return e;
-    e = launch_pdl(hist_kernel, dim3(nb), dim3(kThreads), R * sizeof(int32_t), st, 1, ids, n_pairs,
-                   chunk, R, s.block_counts, s.status);
+    e = launch_pdl(hist_scan_kernel, dim3(nb), dim3(kThreads), R * sizeof(int32_t), st, 1, ids,
+                   n_pairs, chunk, R, s.block_counts, s.status, s.ticket, counts, offsets,
+                   s.n_mtiles, s.tiles);
     count_launch();
     if (e != cudaSuccess) return e;
+  } else {
+    e0 = launch_pdl(empty_scan_kernel, dim3(1), dim3(32), 0, st, 1, R, counts, offsets, s.n_mtiles);
+    count_launch();
+    if (e0 != cudaSuccess) return e0;
   }
-  cudaError_t e2 = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, 1, s.block_counts, nb, R,
-                              counts, offsets, s.n_mtiles, s.tiles);
-  count_launch();
-  if (e2 != cudaSuccess) return e2;
   if (nb > 0) {
     const size_t smem = (size_t)kWarps * R * sizeof(int32_t);
     cudaError_t e = set_smem(scatter_kernel, smem);

@@ -216,6 +216,8 @@ EDGE = [
     ("pages_toy_dff96", dict(ff_routed=96, ff_shared=96)),
     ("no_shared", dict(n_shared=0)),
     ("ragged_1000", dict(n_tokens=1000)),
+    # widths that are multiples of 8 but not of 64: ragged K blocks, masked columns
+    ("odd_widths", dict(d=200, latent=104, ff_routed=72, ff_shared=136)),
 ]
 
 
