@@ -223,11 +223,9 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
   return LMOE_OK;
 }
 
-// z != nullptr: also writes the sorted rows of z to the workspace (the A
-// operand of the routed GEMMs).
 static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t* counts,
                                 int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
-                                cudaStream_t st, const void* z = nullptr) {
+                                cudaStream_t st) {
   const Layout L = layout(d, false);
   DispatchScratch s;
   s.block_counts = at<int32_t>(ws, L.block_counts);
@@ -235,10 +233,9 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
   s.n_mtiles = &at<WsHeader>(ws, L.header)->n_mtiles;
   s.ticket = &at<WsHeader>(ws, L.header)->ticket;
   s.tiles = at<int4>(ws, L.tiles);
-  const int es = d->dtype == LMOE_BF16 ? 2 : 4;
   ProfScope ps("dispatch", st);
-  LMOE_CUDA(launch_dispatch_gather(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm,
-                                   inv, s, z, z ? at<char>(ws, L.zp) : nullptr, d->latent * es, st),
+  LMOE_CUDA(launch_dispatch(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm, inv,
+                            s, st),
             "dispatch");
   return LMOE_OK;
 }

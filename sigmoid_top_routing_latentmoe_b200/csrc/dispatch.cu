@@ -7,8 +7,7 @@
 //               per expert, the per-expert counts and offsets, and the routed
 //               row-tile list (expert, first row, rows) the GEMMs walk,
 //   3. scatter: one CTA per chunk ranks its pairs in pair order inside each
-//               expert, writes perm_token / inv_pair and, in the fused
-//               forward, copies each pair's z row to its sorted slot.
+//               expert and writes perm_token / inv_pair.
 // No result depends on the order of atomic operations: bit-exact.
 #include <algorithm>
 
@@ -59,42 +58,89 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return excl;
 }
 
-// Run by one CTA (any size): chunk_counts[c, e] becomes the number of pairs
-// of expert e in chunks before c; writes counts, offsets and the tile list.
-// Each thread owns whole experts and reads their chunk column 16 loads at a
-// time, so the loads are in flight together.
+// Run by one CTA of kThreads threads: chunk_counts[c, e] becomes the number
+// of pairs of expert e in chunks before c; writes counts, offsets and the tile
+// list.  Experts go in groups whose chunk columns fit the kScanInts-int smem
+// buffer `buf`: one coalesced load of the group's counts (expert-major in
+// smem, rows of C + 1 ints so that neither the transposing stores nor the
+// column walks hit one bank), then each expert's column is scanned by `tpe`
+// threads of one warp (a serial sum over a segment of chunks, then a shuffle
+// scan over the segments), and the prefixes go back with one coalesced store.
+constexpr int kScanInts = 16384;
 __device__ void scan_chunks(int32_t* __restrict__ chunk_counts, int n_chunks, int R,
-                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                            int32_t* __restrict__ n_mtiles, int4* __restrict__ tiles) {
+                            int32_t* __restrict__ buf, int32_t* __restrict__ counts,
+                            int32_t* __restrict__ offsets, int32_t* __restrict__ n_mtiles,
+                            int4* __restrict__ tiles) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t totals[2];
   __shared__ int32_t carry[2];
+  __shared__ int32_t ecount[kThreads];
   if (threadIdx.x == 0) carry[0] = carry[1] = 0;
-  for (int base = 0; base < R; base += blockDim.x) {
-    const int e = base + threadIdx.x;
-    int32_t c = 0;
-    if (e < R) {
-      for (int b0 = 0; b0 < n_chunks; b0 += 16) {
-        int32_t v[16];
+  const int C = n_chunks, C1 = n_chunks + 1;
+  const int group = min(R, min(kThreads, kScanInts / C1));  // experts per group
+  int tpe = 1;  // threads per expert: a power of two, at most 32
+  while (tpe * 2 <= 32 && tpe * 2 * group <= kThreads) tpe *= 2;
+  const int seg = (C + tpe - 1) / tpe;  // chunks per thread
+  for (int e0 = 0; e0 < R; e0 += group) {
+    const int ne = min(group, R - e0);
+    // 16 loads in flight per thread
+    for (int i0 = 0; i0 < C * ne; i0 += 16 * kThreads) {
+      int32_t v[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          v[j] = b0 + j < n_chunks ? chunk_counts[(int64_t)(b0 + j) * R + e] : 0;
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + u * kThreads + threadIdx.x;
+        if (i < C * ne) {
+          const int c = i / ne;
+          v[u] = chunk_counts[(int64_t)c * R + e0 + (i - c * ne)];
+        }
+      }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if (b0 + j < n_chunks) chunk_counts[(int64_t)(b0 + j) * R + e] = c;
-          c += v[j];
+      for (int u = 0; u < 16; ++u) {
+        const int i = i0 + u * kThreads + threadIdx.x;
+        if (i < C * ne) {
+          const int c = i / ne, j = i - c * ne;
+          buf[j * C1 + c] = v[u];
         }
       }
     }
     __syncthreads();
-    const int32_t nt = (c + kTileM - 1) / kTileM;
-    const int32_t ex_c = block_exclusive_scan(c, warp_sums, &totals[0]) + carry[0];
+    const int j = threadIdx.x / tpe, part = threadIdx.x - j * tpe;
+    const bool active = j < ne;
+    const int c0 = min(C, part * seg), c1 = min(C, c0 + seg);
+    int32_t sum = 0;
+    if (active)
+      for (int c = c0; c < c1; ++c) sum += buf[j * C1 + c];
+    // exclusive scan of the segment sums of expert j (tpe lanes of one warp)
+    int32_t inc = sum;
+    for (int off = 1; off < tpe; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, inc, off, tpe);
+      if (part >= off) inc += o;
+    }
+    if (active) {
+      int32_t run = inc - sum;
+      for (int c = c0; c < c1; ++c) {
+        const int32_t v = buf[j * C1 + c];
+        buf[j * C1 + c] = run;
+        run += v;
+      }
+      if (part == tpe - 1) ecount[j] = inc;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < C * ne; i += kThreads) {
+      const int c = i / ne, jj = i - c * ne;
+      chunk_counts[(int64_t)c * R + e0 + jj] = buf[jj * C1 + c];
+    }
+    // counts, offsets and tiles of the group's experts
+    const int e = e0 + threadIdx.x;
+    const int32_t cnt = threadIdx.x < ne ? ecount[threadIdx.x] : 0;
+    const int32_t nt = (cnt + kTileM - 1) / kTileM;
+    const int32_t ex_c = block_exclusive_scan(cnt, warp_sums, &totals[0]) + carry[0];
     const int32_t ex_t = block_exclusive_scan(nt, warp_sums, &totals[1]) + carry[1];
-    if (e < R) {
-      counts[e] = c;
+    if (threadIdx.x < ne) {
+      counts[e] = cnt;
       offsets[e] = ex_c;
-      for (int j = 0; j * kTileM < c; ++j)
-        tiles[ex_t + j] = make_int4(e, ex_c + j * kTileM, min(kTileM, c - j * kTileM), 0);
+      for (int t = 0; t * kTileM < cnt; ++t)
+        tiles[ex_t + t] = make_int4(e, ex_c + t * kTileM, min(kTileM, cnt - t * kTileM), 0);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -148,7 +194,7 @@ __global__ void __launch_bounds__(kThreads) hist_scan_kernel(
   __syncthreads();
   if (!last) return;
   __threadfence();
-  scan_chunks(chunk_counts, gridDim.x, R, counts, offsets, n_mtiles, tiles);
+  scan_chunks(chunk_counts, gridDim.x, R, hist, counts, offsets, n_mtiles, tiles);
   if (threadIdx.x == 0) *ticket = 0;  // ready for the next call
 }
 
@@ -165,13 +211,10 @@ __global__ void empty_scan_kernel(int R, int32_t* __restrict__ counts, int32_t* 
 }
 
 // Ranks each chunk's pairs inside their expert in pair order and scatters.
-// With z != nullptr it also copies z[token] to row `slot` of zp (row_vecs
-// 16-byte vectors per row).
 __global__ void __launch_bounds__(kThreads) scatter_kernel(
     const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int k, int R,
     const int32_t* __restrict__ chunk_first, const int32_t* __restrict__ offsets,
-    int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair, const uint4* __restrict__ z,
-    uint4* __restrict__ zp, int row_vecs) {
+    int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ int32_t wcnt[];  // [kWarps][R]: per-warp counts, then first slots
@@ -217,17 +260,6 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
     if (valid) {
       perm_token[slot] = tok;
       inv_pair[p] = slot;
-    }
-    if (z != nullptr) {
-      // the warp copies its (up to) 32 rows, one row at a time, 16 bytes per lane
-      for (int j = 0; j < 32; ++j) {
-        const int32_t s_j = __shfl_sync(0xffffffffu, slot, j);
-        const int32_t t_j = __shfl_sync(0xffffffffu, tok, j);
-        if (s_j < 0) continue;
-        const uint4* src = z + (int64_t)t_j * row_vecs;
-        uint4* dst = zp + (int64_t)s_j * row_vecs;
-        for (int v = lane; v < row_vecs; v += 32) dst[v] = src[v];
-      }
     }
   }
 }
@@ -287,18 +319,19 @@ int dispatch_blocks(int64_t n_pairs) {
   return (int)((n_pairs + chunk - 1) / chunk);
 }
 
-cudaError_t launch_dispatch_gather(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
-                                   int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
-                                   const DispatchScratch& s, const void* z, void* zp,
-                                   int row_bytes, cudaStream_t st) {
+cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
+                            int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
+                            const DispatchScratch& s, cudaStream_t st) {
   const int64_t n_pairs = n * k;
   const int64_t chunk = chunk_pairs(n_pairs);
   const int nb = dispatch_blocks(n_pairs);
   cudaError_t e0;
   if (nb > 0) {
-    cudaError_t e = set_smem(hist_scan_kernel, R * sizeof(int32_t));
+    // hist doubles as the scan's buffer in the last CTA
+    const size_t smem = (size_t)std::max(R, kScanInts) * sizeof(int32_t);
+    cudaError_t e = set_smem(hist_scan_kernel, smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(hist_scan_kernel, dim3(nb), dim3(kThreads), R * sizeof(int32_t), st, 1, ids,
+    e = launch_pdl(hist_scan_kernel, dim3(nb), dim3(kThreads), smem, st, 1, ids,
                    n_pairs, chunk, R, s.block_counts, s.status, s.ticket, counts, offsets,
                    s.n_mtiles, s.tiles);
     count_launch();
@@ -313,20 +346,13 @@ cudaError_t launch_dispatch_gather(const int32_t* ids, int64_t n, int k, int R, 
     cudaError_t e = set_smem(scatter_kernel, smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(scatter_kernel, dim3(nb), dim3(kThreads), smem, st, 1, ids, n_pairs, chunk, k,
-                   R, (const int32_t*)s.block_counts, (const int32_t*)offsets, perm_token, inv_pair,
-                   static_cast<const uint4*>(z), static_cast<uint4*>(zp), row_bytes / 16);
+                   R, (const int32_t*)s.block_counts, (const int32_t*)offsets, perm_token, inv_pair);
     count_launch();
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
-                            int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
-                            const DispatchScratch& s, cudaStream_t st) {
-  return launch_dispatch_gather(ids, n, k, R, counts, offsets, perm_token, inv_pair, s, nullptr,
-                                nullptr, 0, st);
-}
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
                                cudaStream_t st) {

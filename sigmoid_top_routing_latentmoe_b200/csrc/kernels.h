@@ -28,12 +28,6 @@ int dispatch_blocks(int64_t n_pairs);
 cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
                             const DispatchScratch& s, cudaStream_t st);
-// The same, and also zp[slot] = z[token] for every pair (row_bytes per row,
-// a multiple of 16): the sorted A rows of the routed GEMMs.
-cudaError_t launch_dispatch_gather(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
-                                   int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
-                                   const DispatchScratch& s, const void* z, void* zp,
-                                   int row_bytes, cudaStream_t st);
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
                                cudaStream_t st);
 // zp[r, :] = z[perm_token[r], :]

@@ -8,9 +8,11 @@
 //   warp 1   MMA issuer: tcgen05.mma.kind::f16 (bf16 x bf16 -> fp32) into a
 //            double-buffered TMEM accumulator (2 x 256 columns), and the
 //            TMEM allocator,
-//   warps 2-5 epilogue: tcgen05.ld of the accumulator, the fused epilogue of
+//   warps 2-9 epilogue: tcgen05.ld of the accumulator, the fused epilogue of
 //            the GEMM (bf16/fp32 store, or the SiTU-GLU hidden unit of a
-//            gate/up column pair), 16-byte global stores.
+//            gate/up column pair), then bf16 blocks of 32 rows x 64 columns
+//            transposed through a per-warp smem buffer so that every global
+//            store instruction writes whole 128-byte row segments.
 // The four GEMMs (sec-07 compute flow; kda/layers/latent_moe.py):
 //   XPASS   x [N, d] against [W_down | W_r | (W_g,sh, W_u,sh) pairs]: z, the
 //           router logits (step 2) and the shared experts' SiTU hidden units
@@ -58,7 +60,8 @@ struct Cfg {
   static constexpr int B_BYTES = (CG == 1 ? 2 : 1) * SUB * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB or 32 KB
   static constexpr int STAGES = CG == 1 ? 4 : 6;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  static constexpr int EPI_STAGE = 32 * 128;             // per epilogue warp: 32 rows x 128 B
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * EPI_STAGE + 1024;
   static constexpr int MT = BM * CG;                     // tile rows
 };
 
@@ -200,6 +203,51 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two 32-column TMEM loads in flight before one wait.
+__device__ __forceinline__ void tc_ld32x2(uint32_t ta, float (&va)[32], uint32_t tb,
+                                          float (&vb)[32]) {
+  uint32_t r[32], q[32];
+#define LMOE_TC_LD32(ADDR, R)                                                                   \
+  asm volatile(                                                                                 \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                                 \
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"                                 \
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"               \
+      : "=r"(R[0]), "=r"(R[1]), "=r"(R[2]), "=r"(R[3]), "=r"(R[4]), "=r"(R[5]), "=r"(R[6]),     \
+        "=r"(R[7]), "=r"(R[8]), "=r"(R[9]), "=r"(R[10]), "=r"(R[11]), "=r"(R[12]),             \
+        "=r"(R[13]), "=r"(R[14]), "=r"(R[15]), "=r"(R[16]), "=r"(R[17]), "=r"(R[18]),          \
+        "=r"(R[19]), "=r"(R[20]), "=r"(R[21]), "=r"(R[22]), "=r"(R[23]), "=r"(R[24]),          \
+        "=r"(R[25]), "=r"(R[26]), "=r"(R[27]), "=r"(R[28]), "=r"(R[29]), "=r"(R[30]),          \
+        "=r"(R[31])                                                                             \
+      : "r"(ADDR))
+  LMOE_TC_LD32(ta, r);
+  LMOE_TC_LD32(tb, q);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    va[i] = __uint_as_float(r[i]);
+    vb[i] = __uint_as_float(q[i]);
+  }
+}
+// Four 32-column TMEM loads in flight before one wait.
+__device__ __forceinline__ void tc_ld32x4(uint32_t ta, float (&va)[32], uint32_t tb,
+                                          float (&vb)[32], uint32_t tc, float (&vc)[32],
+                                          uint32_t td, float (&vd)[32]) {
+  uint32_t r[32], q[32], x[32], y[32];
+  LMOE_TC_LD32(ta, r);
+  LMOE_TC_LD32(tb, q);
+  LMOE_TC_LD32(tc, x);
+  LMOE_TC_LD32(td, y);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    va[i] = __uint_as_float(r[i]);
+    vb[i] = __uint_as_float(q[i]);
+    vc[i] = __uint_as_float(x[i]);
+    vd[i] = __uint_as_float(y[i]);
+  }
+}
+#undef LMOE_TC_LD32
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
 // core groups 1024 bytes apart (SBO), descriptor version 1 (sm_100).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
@@ -214,24 +262,35 @@ __device__ __forceinline__ uint32_t tanh_h2(uint32_t v) {
 // Two SiTU-GLU hidden units at once, packed to bf16x2:
 //   h = beta1 tanh(a/beta1) sigmoid(a) * beta2 tanh(c/beta2),
 //   sigmoid(a) = 1/2 + tanh(a/2)/2,
-// the three tanh on f16x2 pairs (one MUFU op per pair), the product of the
-// bounded factors (each |.| <= 1) in f16x2, the scale beta1*beta2 in fp32.
+// on f16x2 pairs: a and c are rounded to f16 once and scaled there, the three
+// tanh are one MUFU op per pair, the bounded factors (each |.| <= 1) and the
+// scale beta1*beta2 (|h| <= beta1*beta2) are multiplied in f16x2.  An |a| or
+// |c| beyond the f16 range rounds to infinity, where every tanh saturates to
+// its limit +-1 as it should.
+struct SituConsts {
+  __half2 inv_b1, inv_b2, b12, half;
+};
+__device__ __forceinline__ SituConsts situ_consts(const Params& p) {
+  return {__float2half2_rn(p.inv_beta1), __float2half2_rn(p.inv_beta2),
+          __float2half2_rn(p.beta12), __float2half2_rn(0.5f)};
+}
 __device__ __forceinline__ uint32_t situ2_bf16(float a0, float a1, float c0, float c1,
-                                               const Params& p) {
-  const __half2 x1 = __floats2half2_rn(a0 * p.inv_beta1, a1 * p.inv_beta1);
-  const __half2 x2 = __floats2half2_rn(a0 * 0.5f, a1 * 0.5f);
-  const __half2 x3 = __floats2half2_rn(c0 * p.inv_beta2, c1 * p.inv_beta2);
+                                               const SituConsts& k) {
+  const __half2 a = __floats2half2_rn(a0, a1);
+  const __half2 c = __floats2half2_rn(c0, c1);
+  const __half2 x1 = __hmul2(a, k.inv_b1);
+  const __half2 x2 = __hmul2(a, k.half);
+  const __half2 x3 = __hmul2(c, k.inv_b2);
   uint32_t u1 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x1));
   uint32_t u2 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x2));
   uint32_t u3 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x3));
   const __half2 t1 = *reinterpret_cast<__half2*>(&u1);
   const __half2 t2 = *reinterpret_cast<__half2*>(&u2);
   const __half2 t3 = *reinterpret_cast<__half2*>(&u3);
-  const __half2 half = __float2half2_rn(0.5f);
-  const __half2 sg = __hfma2(t2, half, half);
-  const __half2 h = __hmul2(__hmul2(t1, sg), t3);
+  const __half2 sg = __hfma2(t2, k.half, k.half);
+  const __half2 h = __hmul2(__hmul2(__hmul2(t1, sg), t3), k.b12);
   const float2 f = __half22float2(h);
-  __nv_bfloat162 o = __floats2bfloat162_rn(f.x * p.beta12, f.y * p.beta12);
+  __nv_bfloat162 o = __floats2bfloat162_rn(f.x, f.y);
   return *reinterpret_cast<uint32_t*>(&o);
 }
 
@@ -575,18 +634,51 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
 }
 
 // ------------------------------------------------------------- epilogue
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32], int valid) {
-  // valid: number of leading columns to write (multiple of 8)
+// A 32-row x 128-byte block of this warp (lane i holds row i as 32 words: 64
+// bf16 or 32 fp32 columns) goes through the warp's 4 KB smem buffer: rows of
+// 128 bytes whose 16-byte chunks are XOR-swizzled by (row mod 8), so that the
+// row-wise writes and the column-wise reads are both free of bank conflicts.
+// Read back, each store instruction covers 4 rows x 128 contiguous bytes
+// instead of 32 rows x 16 bytes.  rows / bytes: how many of the block's rows
+// and leading bytes of each row (a multiple of 16) exist; ld in bytes.
+__device__ __forceinline__ void warp_store_block(uint32_t stage, const uint32_t (&w)[32],
+                                                 char* base, int64_t ld, int rows, int bytes) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    if (g * 8 < valid) {
-      uint4 w;
-      w.x = pack_bf16(v[g * 8 + 0], v[g * 8 + 1]);
-      w.y = pack_bf16(v[g * 8 + 2], v[g * 8 + 3]);
-      w.z = pack_bf16(v[g * 8 + 4], v[g * 8 + 5]);
-      w.w = pack_bf16(v[g * 8 + 6], v[g * 8 + 7]);
-      reinterpret_cast<uint4*>(dst)[g] = w;
-    }
+  for (int q = 0; q < 8; ++q)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                     stage + lane * 128 + ((q ^ (lane & 7)) << 4)),
+                 "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                 : "memory");
+  __syncwarp();
+  const int q = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = i * 4 + (lane >> 3);
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(stage + row * 128 + ((q ^ (row & 7)) << 4))
+                 : "memory");
+    if (row < rows && q * 16 < bytes)
+      *reinterpret_cast<uint4*>(base + (int64_t)row * ld + q * 16) = v;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void warp_store_bf16(uint32_t stage, const uint32_t (&w)[32],
+                                                __nv_bfloat16* base, int64_t ld, int rows,
+                                                int cols) {
+  warp_store_block(stage, w, reinterpret_cast<char*>(base), ld * 2, rows, cols * 2);
+}
+
+// 64 fp32 accumulator columns -> 32 packed bf16x2 words.
+__device__ __forceinline__ void pack_block(const float (&a)[32], const float (&b)[32],
+                                           uint32_t (&w)[32]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    w[j] = pack_bf16(a[2 * j], a[2 * j + 1]);
+    w[16 + j] = pack_bf16(b[2 * j], b[2 * j + 1]);
   }
 }
 
@@ -632,12 +724,13 @@ __device__ __forceinline__ void route_row32(const Params& p, const float (&lg)[3
 
 template <int MODE, int CG>
 __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint64_t* tempty,
-                                         uint32_t tmem, volatile int* abort_flag, uint32_t rank,
-                                         int unit, int n_units) {
+                                         uint32_t tmem, uint32_t stage, volatile int* abort_flag,
+                                         uint32_t rank, int unit, int n_units) {
   const int ew = (threadIdx.x >> 5) & 3;  // TMEM lane quarter this warp may access
-  const int half = ((threadIdx.x >> 5) - 2) >> 2;  // which of the two column halves
+  const int half = ((threadIdx.x >> 5) - 2) >> 2;  // which half of the column blocks
   const int lane = threadIdx.x & 31;
-  const int r = ew * 32 + lane + (CG == 2 ? BM * (int)rank : 0);  // tile row of this thread
+  const int wrow = ew * 32 + (CG == 2 ? BM * (int)rank : 0);  // first tile row of this warp
+  const SituConsts sk = situ_consts(p);
   int acc = 0;
   uint32_t acc_phase = 0;
   const int total = total_tiles<MODE, CG>(p);
@@ -646,10 +739,13 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
     if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.status)) break;
     tc_fence_after();
     const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * ACC_COLS;
-    const bool row_ok = r < tl.rows;
-    const int64_t grow = (int64_t)tl.m0 + r;
-    if (tl.epi == EPI_SITU) {
-      // columns [0,128) hold gate pre-activations, [128,256) the matching up ones
+    const int rows = min(32, tl.rows - wrow);  // rows of this warp inside the tile
+    const int64_t grow0 = (int64_t)tl.m0 + wrow;
+    if (rows <= 0) {
+      // nothing of this warp's rows exists in the tile
+    } else if (tl.epi == EPI_SITU) {
+      // columns [0,128) hold gate pre-activations, [128,256) the matching up ones;
+      // this warp writes hidden units [64 half, 64 half + 64)
       int width;
       __nv_bfloat16* out;
       int64_t ld;
@@ -662,63 +758,77 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         out = static_cast<__nv_bfloat16*>(p.out0);
         ld = p.ld0;
       }
-#pragma unroll 1
-      for (int c = half; c < SUB / 32; c += 2) {
-        float g[32], u[32];
-        tc_ld32(tbase + c * 32, g);
-        tc_ld32(tbase + SUB + c * 32, u);
-        if (row_ok) {
-          __nv_bfloat16* dst = out + grow * ld + tl.ocol + c * 32;
-          const int valid = width - c * 32;
+      const int cols = min(64, width - half * 64);
+      if (cols > 0) {
+        uint32_t w[32];
+        {
+          float g0[32], u0[32], g1[32], u1[32];
+          const uint32_t c0 = half * 64;
+          tc_ld32x4(tbase + c0, g0, tbase + SUB + c0, u0, tbase + c0 + 32, g1,
+                    tbase + SUB + c0 + 32, u1);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (q * 8 < valid) {
-              uint4 w;
-              w.x = situ2_bf16(g[q * 8 + 0], g[q * 8 + 1], u[q * 8 + 0], u[q * 8 + 1], p);
-              w.y = situ2_bf16(g[q * 8 + 2], g[q * 8 + 3], u[q * 8 + 2], u[q * 8 + 3], p);
-              w.z = situ2_bf16(g[q * 8 + 4], g[q * 8 + 5], u[q * 8 + 4], u[q * 8 + 5], p);
-              w.w = situ2_bf16(g[q * 8 + 6], g[q * 8 + 7], u[q * 8 + 6], u[q * 8 + 7], p);
-              reinterpret_cast<uint4*>(dst)[q] = w;
-            }
+          for (int j = 0; j < 16; ++j) {
+            w[j] = situ2_bf16(g0[2 * j], g0[2 * j + 1], u0[2 * j], u0[2 * j + 1], sk);
+            w[16 + j] = situ2_bf16(g1[2 * j], g1[2 * j + 1], u1[2 * j], u1[2 * j + 1], sk);
           }
         }
+        warp_store_bf16(stage, w, out + grow0 * ld + tl.ocol + half * 64, ld, rows, cols);
       }
-    } else {
+    } else if (MODE == XPASS) {
 #pragma unroll 1
       for (int s = 0; s < tl.n_sub; ++s) {
-        if (MODE == XPASS && tl.bmap[s] == kPadMap) continue;
-        if (MODE == XPASS && tl.bmap[s] == 1 && p.fuse_topk) {
-          // all R <= 32 router logits of this row sit in one 32-column chunk
-          if (half == 0) {
-            float lg[32];
-            tc_ld32(tbase + tl.scol[s], lg);
-            if (row_ok) route_row32(p, lg, grow);
+        if (tl.bmap[s] == kPadMap) continue;
+        if (tl.bmap[s] == 1) {  // router logits
+          if (p.fuse_topk) {
+            // all R <= 32 router logits of a row sit in one 32-column chunk
+            if (half == 0) {
+              float lg[32];
+              tc_ld32(tbase + tl.scol[s], lg);
+              if (lane < rows) route_row32(p, lg, grow0 + lane);
+            }
+            continue;
+          }
+#pragma unroll 1
+          for (int c = half; c < tl.srows[s] / 32; c += 2) {
+            float v[32];
+            tc_ld32(tbase + tl.scol[s] + c * 32, v);
+            if (lane >= rows) continue;
+            const int col = tl.brow[s] + c * 32;
+            float* dst = static_cast<float*>(p.out1) + (grow0 + lane) * p.ld1 + col;
+#pragma unroll
+            for (int g4 = 0; g4 < 8; ++g4)
+              if (col + g4 * 4 < p.R)
+                reinterpret_cast<float4*>(dst)[g4] =
+                    make_float4(v[g4 * 4], v[g4 * 4 + 1], v[g4 * 4 + 2], v[g4 * 4 + 3]);
           }
           continue;
         }
+        // z columns [brow + 64 half, +64)
+        const int col = tl.brow[s] + half * 64;
+        const int cols = min(64, p.L - col);
+        if (cols <= 0) continue;
+        float a[32], b[32];
+        tc_ld32x2(tbase + tl.scol[s] + half * 64, a, tbase + tl.scol[s] + half * 64 + 32, b);
+        uint32_t w[32];
+        pack_block(a, b, w);
+        warp_store_bf16(stage, w, static_cast<__nv_bfloat16*>(p.out0) + grow0 * p.ld0 + col,
+                        p.ld0, rows, cols);
+      }
+    } else {
+      // FINAL / ROUTED2: accumulator columns [0, ncols) are output columns
+      // [ocol, ocol + ncols); this warp writes the 64-column blocks half, half + 2
+      const int width = (MODE == FINAL ? p.d : p.L) - tl.ocol;
+      const int ncols = min(tl.ncols, width);
 #pragma unroll 1
-        for (int c = half; c < tl.srows[s] / 32; c += 2) {
-          float v[32];
-          tc_ld32(tbase + tl.scol[s] + c * 32, v);
-          if (!row_ok) continue;
-          if (MODE == XPASS) {
-            const int col = tl.brow[s] + c * 32;
-            if (tl.bmap[s] == 0) {  // z columns
-              store_bf16x32(static_cast<__nv_bfloat16*>(p.out0) + grow * p.ld0 + col, v, p.L - col);
-            } else {                // router logits, fp32
-              float* dst = static_cast<float*>(p.out1) + grow * p.ld1 + col;
-#pragma unroll
-              for (int g4 = 0; g4 < 8; ++g4)
-                if (col + g4 * 4 < p.R)
-                  reinterpret_cast<float4*>(dst)[g4] =
-                      make_float4(v[g4 * 4], v[g4 * 4 + 1], v[g4 * 4 + 2], v[g4 * 4 + 3]);
-            }
-          } else {
-            const int col = tl.ocol + tl.scol[s] + c * 32;
-            const int width = (MODE == FINAL ? p.d : p.L) - col;
-            store_bf16x32(static_cast<__nv_bfloat16*>(p.out0) + grow * p.ld0 + col, v, width);
-          }
-        }
+      for (int cb = half; cb * 64 < ncols; cb += 2) {
+        const int cols = min(64, ncols - cb * 64);
+        const int64_t col = tl.ocol + cb * 64;
+        float a[32], b[32];
+        tc_ld32x2(tbase + cb * 64, a, tbase + cb * 64 + 32, b);
+        uint32_t w[32];
+        pack_block(a, b, w);
+        warp_store_bf16(stage, w, static_cast<__nv_bfloat16*>(p.out0) + grow0 * p.ld0 + col,
+                        p.ld0, rows, cols);
       }
     }
     tc_fence_before();
@@ -795,7 +905,9 @@ __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_cons
       mma_issue<MODE, CG>(p, ring, full, empty, tfull, tempty, &drain, tmem, &abort_flag, unit,
                           n_units);
   } else {
-    epilogue<MODE, CG>(p, tfull, tempty, tmem, &abort_flag, rank, unit, n_units);
+    const uint32_t stage =
+        smem_u32(ring) + C::STAGES * C::STAGE_BYTES + (warp - 2) * C::EPI_STAGE;
+    epilogue<MODE, CG>(p, tfull, tempty, tmem, stage, &abort_flag, rank, unit, n_units);
   }
 
   tc_fence_before();
