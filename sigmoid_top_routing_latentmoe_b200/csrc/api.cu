@@ -231,7 +231,6 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
   s.block_counts = at<int32_t>(ws, L.block_counts);
   s.status = &at<WsHeader>(ws, L.header)->status;
   s.n_mtiles = &at<WsHeader>(ws, L.header)->n_mtiles;
-  s.ticket = &at<WsHeader>(ws, L.header)->ticket;
   s.tiles = at<int4>(ws, L.tiles);
   ProfScope ps("dispatch", st);
   LMOE_CUDA(launch_dispatch(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm, inv,

@@ -20,8 +20,7 @@ constexpr int kTileM = 128;
 struct WsHeader {
   int32_t status;        // 0, or the first failure code recorded on the device
   int32_t n_mtiles;      // number of routed row tiles (written by dispatch)
-  int32_t ticket;        // chunks of the dispatch histogram done (zero between calls)
-  int32_t pad[61];
+  int32_t pad[62];
 };
 
 __device__ __forceinline__ float to_f(float v) { return v; }

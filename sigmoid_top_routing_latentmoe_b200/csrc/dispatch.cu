@@ -3,11 +3,14 @@
 // token-major, are stably sorted by expert id -- the pages' argsort(stable) +
 // bincount + cumsum -- as a deterministic counting sort over chunks of pairs:
 //   1. hist:    one CTA per chunk counts its pairs per expert,
-//   2. scan:    one CTA turns the chunk counts into each chunk's first slot
-//               per expert, the per-expert counts and offsets, and the routed
-//               row-tile list (expert, first row, rows) the GEMMs walk,
-//   3. scatter: one CTA per chunk ranks its pairs in pair order inside each
-//               expert and writes perm_token / inv_pair.
+//   2. colscan: (large count matrices only) one CTA per 32 experts turns
+//               each expert's column of chunk counts into exclusive prefixes
+//               and the expert's total,
+//   3. scatter: one CTA per chunk derives each expert's first sorted slot for
+//               its chunk (offsets = exclusive scan of the totals), ranks its
+//               pairs in pair order inside each expert and writes perm_token /
+//               inv_pair; CTA 0 also writes counts, offsets and the routed
+//               row-tile list (expert, first row, rows) the GEMMs walk.
 // No result depends on the order of atomic operations: bit-exact.
 #include <algorithm>
 
@@ -58,115 +61,19 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
   return excl;
 }
 
-// Run by one CTA of kThreads threads: chunk_counts[c, e] becomes the number
-// of pairs of expert e in chunks before c; writes counts, offsets and the tile
-// list.  Experts go in groups whose chunk columns fit the kScanInts-int smem
-// buffer `buf`: one coalesced load of the group's counts (expert-major in
-// smem, rows of C + 1 ints so that neither the transposing stores nor the
-// column walks hit one bank), then each expert's column is scanned by `tpe`
-// threads of one warp (a serial sum over a segment of chunks, then a shuffle
-// scan over the segments), and the prefixes go back with one coalesced store.
-constexpr int kScanInts = 16384;
-__device__ void scan_chunks(int32_t* __restrict__ chunk_counts, int n_chunks, int R,
-                            int32_t* __restrict__ buf, int32_t* __restrict__ counts,
-                            int32_t* __restrict__ offsets, int32_t* __restrict__ n_mtiles,
-                            int4* __restrict__ tiles) {
-  __shared__ int32_t warp_sums[32];
-  __shared__ int32_t totals[2];
-  __shared__ int32_t carry[2];
-  __shared__ int32_t ecount[kThreads];
-  if (threadIdx.x == 0) carry[0] = carry[1] = 0;
-  const int C = n_chunks, C1 = n_chunks + 1;
-  const int group = min(R, min(kThreads, kScanInts / C1));  // experts per group
-  int tpe = 1;  // threads per expert: a power of two, at most 32
-  while (tpe * 2 <= 32 && tpe * 2 * group <= kThreads) tpe *= 2;
-  const int seg = (C + tpe - 1) / tpe;  // chunks per thread
-  for (int e0 = 0; e0 < R; e0 += group) {
-    const int ne = min(group, R - e0);
-    // 16 loads in flight per thread
-    for (int i0 = 0; i0 < C * ne; i0 += 16 * kThreads) {
-      int32_t v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = i0 + u * kThreads + threadIdx.x;
-        if (i < C * ne) {
-          const int c = i / ne;
-          v[u] = chunk_counts[(int64_t)c * R + e0 + (i - c * ne)];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = i0 + u * kThreads + threadIdx.x;
-        if (i < C * ne) {
-          const int c = i / ne, j = i - c * ne;
-          buf[j * C1 + c] = v[u];
-        }
-      }
-    }
-    __syncthreads();
-    const int j = threadIdx.x / tpe, part = threadIdx.x - j * tpe;
-    const bool active = j < ne;
-    const int c0 = min(C, part * seg), c1 = min(C, c0 + seg);
-    int32_t sum = 0;
-    if (active)
-      for (int c = c0; c < c1; ++c) sum += buf[j * C1 + c];
-    // exclusive scan of the segment sums of expert j (tpe lanes of one warp)
-    int32_t inc = sum;
-    for (int off = 1; off < tpe; off <<= 1) {
-      const int32_t o = __shfl_up_sync(0xffffffffu, inc, off, tpe);
-      if (part >= off) inc += o;
-    }
-    if (active) {
-      int32_t run = inc - sum;
-      for (int c = c0; c < c1; ++c) {
-        const int32_t v = buf[j * C1 + c];
-        buf[j * C1 + c] = run;
-        run += v;
-      }
-      if (part == tpe - 1) ecount[j] = inc;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < C * ne; i += kThreads) {
-      const int c = i / ne, jj = i - c * ne;
-      chunk_counts[(int64_t)c * R + e0 + jj] = buf[jj * C1 + c];
-    }
-    // counts, offsets and tiles of the group's experts
-    const int e = e0 + threadIdx.x;
-    const int32_t cnt = threadIdx.x < ne ? ecount[threadIdx.x] : 0;
-    const int32_t nt = (cnt + kTileM - 1) / kTileM;
-    const int32_t ex_c = block_exclusive_scan(cnt, warp_sums, &totals[0]) + carry[0];
-    const int32_t ex_t = block_exclusive_scan(nt, warp_sums, &totals[1]) + carry[1];
-    if (threadIdx.x < ne) {
-      counts[e] = cnt;
-      offsets[e] = ex_c;
-      for (int t = 0; t * kTileM < cnt; ++t)
-        tiles[ex_t + t] = make_int4(e, ex_c + t * kTileM, min(kTileM, cnt - t * kTileM), 0);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      carry[0] += totals[0];
-      carry[1] += totals[1];
-    }
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    offsets[R] = carry[0];
-    *n_mtiles = carry[1];
-  }
-}
+// Chunk-count matrices up to this many ints are scanned inside the scatter
+// kernel (every CTA walks the columns it needs); larger ones get a column-scan
+// kernel first.
+constexpr int kSmallScan = 8192;
 
-// One CTA per chunk counts the chunk's pairs per expert; the last CTA to
-// finish (an atomic ticket in the workspace header, reset by that CTA) then
-// runs the scan over all chunks.
-__global__ void __launch_bounds__(kThreads) hist_scan_kernel(
-    const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int R,
-    int32_t* __restrict__ chunk_counts, int32_t* __restrict__ status, int32_t* __restrict__ ticket,
-    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ n_mtiles,
-    int4* __restrict__ tiles) {
+// One CTA per chunk counts the chunk's pairs per expert.
+__global__ void __launch_bounds__(kThreads) hist_kernel(const int32_t* __restrict__ ids,
+                                                        int64_t n_pairs, int64_t chunk, int R,
+                                                        int32_t* __restrict__ chunk_counts,
+                                                        int32_t* __restrict__ status) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ int32_t hist[];
-  __shared__ int32_t last;
   for (int e = threadIdx.x; e < R; e += kThreads) hist[e] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -187,15 +94,49 @@ __global__ void __launch_bounds__(kThreads) hist_scan_kernel(
   __syncthreads();
   for (int e = threadIdx.x; e < R; e += kThreads)
     chunk_counts[(int64_t)blockIdx.x * R + e] = hist[e];
-  // publish this chunk, then take a ticket; the last ticket scans
-  __threadfence();
+}
+
+// Large count matrices: one CTA per 32 experts turns each column of chunk
+// counts into its exclusive prefix over the chunks (in place) and writes the
+// expert's total.  The block is staged in smem (rows padded to 33 ints); a
+// warp scans one expert with each lane owning consecutive chunks.
+__global__ void __launch_bounds__(kThreads) colscan_kernel(int32_t* __restrict__ chunk_counts,
+                                                           int C, int R,
+                                                           int32_t* __restrict__ counts) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int32_t col[kMaxChunks][33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e0 = blockIdx.x * 32;
+  const bool in = e0 + lane < R;
+  for (int c = warp; c < C; c += kWarps)
+    col[c][lane] = in ? chunk_counts[(int64_t)c * R + e0 + lane] : 0;
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+  const int per = (C + 31) / 32;  // chunks per lane (<= 4)
+  for (int j = warp; j < 32; j += kWarps) {
+    const int c0 = lane * per;
+    int32_t s = 0;
+    for (int i = 0; i < per; ++i)
+      if (c0 + i < C) s += col[c0 + i][j];
+    int32_t inc = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += o;
+    }
+    int32_t run = inc - s;
+    for (int i = 0; i < per; ++i)
+      if (c0 + i < C) {
+        const int32_t v = col[c0 + i][j];
+        col[c0 + i][j] = run;
+        run += v;
+      }
+    const int32_t total = __shfl_sync(0xffffffffu, inc, 31);
+    if (lane == 0 && e0 + j < R) counts[e0 + j] = total;
+  }
   __syncthreads();
-  if (!last) return;
-  __threadfence();
-  scan_chunks(chunk_counts, gridDim.x, R, hist, counts, offsets, n_mtiles, tiles);
-  if (threadIdx.x == 0) *ticket = 0;  // ready for the next call
+  for (int c = warp; c < C; c += kWarps)
+    if (in) chunk_counts[(int64_t)c * R + e0 + lane] = col[c][lane];
 }
 
 // No pairs at all: every count and offset is zero, no tiles.
@@ -211,18 +152,75 @@ __global__ void empty_scan_kernel(int R, int32_t* __restrict__ counts, int32_t* 
 }
 
 // Ranks each chunk's pairs inside their expert in pair order and scatters.
+// Prologue: every CTA derives, for each expert, its chunk's first sorted slot
+// -- offsets[e] (an exclusive scan of the per-expert totals) plus the pairs of
+// expert e in earlier chunks -- from the chunk counts: summed here when
+// `prefixed` is 0, or read as the column scan left them.  CTA 0 also writes
+// counts (unless prefixed), offsets and the routed row-tile list.
 __global__ void __launch_bounds__(kThreads) scatter_kernel(
-    const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int k, int R,
-    const int32_t* __restrict__ chunk_first, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int k, int R, int C,
+    const int32_t* __restrict__ chunk_counts, int prefixed, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ n_mtiles, int4* __restrict__ tiles,
     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ int32_t wcnt[];  // [kWarps][R]: per-warp counts, then first slots
+  // [kWarps][R] per-warp counts, then first slots; [R] this chunk's first slot
+  extern __shared__ int32_t wcnt[];
+  int32_t* base = wcnt + kWarps * R;
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t totals[2];
+  __shared__ int32_t carry[2];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int cb = blockIdx.x;
   for (int i = threadIdx.x; i < kWarps * R; i += kThreads) wcnt[i] = 0;
+  if (threadIdx.x == 0) carry[0] = carry[1] = 0;
   __syncthreads();
+  for (int e0 = 0; e0 < R; e0 += kThreads) {
+    const int e = e0 + threadIdx.x;
+    int32_t first = 0, tot = 0;
+    if (e < R) {
+      if (prefixed) {
+        first = chunk_counts[(int64_t)cb * R + e];
+        tot = counts[e];
+      } else {
+        for (int c0 = 0; c0 < C; c0 += 16) {
+          int32_t v[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            v[u] = c0 + u < C ? chunk_counts[(int64_t)(c0 + u) * R + e] : 0;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            first += c0 + u < cb ? v[u] : 0;
+            tot += v[u];
+          }
+        }
+      }
+    }
+    const int32_t nt = (tot + kTileM - 1) / kTileM;
+    const int32_t ex_c = block_exclusive_scan(tot, warp_sums, &totals[0]) + carry[0];
+    const int32_t ex_t = block_exclusive_scan(nt, warp_sums, &totals[1]) + carry[1];
+    if (e < R) {
+      base[e] = ex_c + first;
+      if (cb == 0) {
+        if (!prefixed) counts[e] = tot;
+        offsets[e] = ex_c;
+        for (int t = 0; t * kTileM < tot; ++t)
+          tiles[ex_t + t] = make_int4(e, ex_c + t * kTileM, min(kTileM, tot - t * kTileM), 0);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      carry[0] += totals[0];
+      carry[1] += totals[1];
+    }
+    __syncthreads();
+  }
+  if (cb == 0 && threadIdx.x == 0) {
+    offsets[R] = carry[0];
+    *n_mtiles = carry[1];
+  }
   const int64_t per_warp = chunk / kWarps;
-  const int64_t p0 = (int64_t)blockIdx.x * chunk + warp * per_warp;
+  const int64_t p0 = (int64_t)cb * chunk + warp * per_warp;
   const int64_t p1 = min(n_pairs, p0 + per_warp);
   int32_t* my = wcnt + warp * R;
   // pass 1: this warp's counts per expert (only this warp writes its row)
@@ -236,7 +234,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
   __syncthreads();
   // pass 2: first sorted slot of each warp's pairs of expert e
   for (int e = threadIdx.x; e < R; e += kThreads) {
-    int32_t run = offsets[e] + chunk_first[(int64_t)blockIdx.x * R + e];
+    int32_t run = base[e];
     for (int w = 0; w < kWarps; ++w) {
       const int32_t c = wcnt[w * R + e];
       wcnt[w * R + e] = run;
@@ -325,31 +323,32 @@ cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t
   const int64_t n_pairs = n * k;
   const int64_t chunk = chunk_pairs(n_pairs);
   const int nb = dispatch_blocks(n_pairs);
-  cudaError_t e0;
-  if (nb > 0) {
-    // hist doubles as the scan's buffer in the last CTA
-    const size_t smem = (size_t)std::max(R, kScanInts) * sizeof(int32_t);
-    cudaError_t e = set_smem(hist_scan_kernel, smem);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(hist_scan_kernel, dim3(nb), dim3(kThreads), smem, st, 1, ids,
-                   n_pairs, chunk, R, s.block_counts, s.status, s.ticket, counts, offsets,
-                   s.n_mtiles, s.tiles);
+  if (nb == 0) {
     count_launch();
-    if (e != cudaSuccess) return e;
-  } else {
-    e0 = launch_pdl(empty_scan_kernel, dim3(1), dim3(32), 0, st, 1, R, counts, offsets, s.n_mtiles);
-    count_launch();
-    if (e0 != cudaSuccess) return e0;
+    return launch_pdl(empty_scan_kernel, dim3(1), dim3(32), 0, st, 1, R, counts, offsets,
+                      s.n_mtiles);
   }
-  if (nb > 0) {
-    const size_t smem = (size_t)kWarps * R * sizeof(int32_t);
-    cudaError_t e = set_smem(scatter_kernel, smem);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(scatter_kernel, dim3(nb), dim3(kThreads), smem, st, 1, ids, n_pairs, chunk, k,
-                   R, (const int32_t*)s.block_counts, (const int32_t*)offsets, perm_token, inv_pair);
+  cudaError_t e = set_smem(hist_kernel, R * sizeof(int32_t));
+  if (e != cudaSuccess) return e;
+  count_launch();
+  e = launch_pdl(hist_kernel, dim3(nb), dim3(kThreads), R * sizeof(int32_t), st, 1, ids, n_pairs,
+                 chunk, R, s.block_counts, s.status);
+  if (e != cudaSuccess) return e;
+  const int prefixed = (int64_t)nb * R > kSmallScan ? 1 : 0;
+  if (prefixed) {
     count_launch();
+    e = launch_pdl(colscan_kernel, dim3((R + 31) / 32), dim3(kThreads), 0, st, 1, s.block_counts,
+                   nb, R, counts);
     if (e != cudaSuccess) return e;
   }
+  const size_t smem = (size_t)(kWarps + 1) * R * sizeof(int32_t);
+  e = set_smem(scatter_kernel, smem);
+  if (e != cudaSuccess) return e;
+  count_launch();
+  e = launch_pdl(scatter_kernel, dim3(nb), dim3(kThreads), smem, st, 1, ids, n_pairs, chunk, k, R,
+                 nb, (const int32_t*)s.block_counts, prefixed, counts, offsets, s.n_mtiles,
+                 s.tiles, perm_token, inv_pair);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

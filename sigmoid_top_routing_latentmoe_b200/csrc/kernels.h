@@ -21,7 +21,6 @@ struct DispatchScratch {
   int32_t* block_counts;  // [n_blocks, R]
   int32_t* status;        // workspace status word
   int32_t* n_mtiles;      // out: number of routed row tiles
-  int32_t* ticket;        // zero between calls: counts the chunks done
   int4* tiles;            // out: [max_tiles] (expert, row0, rows, 0)
 };
 int dispatch_blocks(int64_t n_pairs);

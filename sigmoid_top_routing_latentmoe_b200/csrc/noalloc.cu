@@ -35,7 +35,7 @@ namespace {
 
 // Capacity of the fixed scratch array, in int32 words (1 MiB).
 constexpr int64_t kNoAllocWords = 1 << 18;
-constexpr int64_t kHeaderWords = 64;  // [0] status, [1] routed tile count, [2] chunk ticket
+constexpr int64_t kHeaderWords = 64;  // [0] status, [1] routed tile count
 
 static __device__ __align__(256) int32_t g_dispatch_scratch[kNoAllocWords];
 
@@ -123,15 +123,14 @@ LMOE_API lmoe_status moe_dispatch_noalloc(const lmoe_dims* dims, const int32_t* 
   lmoe_status s = scratch_on_current_device(&scratch);
   if (s != LMOE_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  // The status word and the chunk ticket are the scratch that must start at
-  // zero; the histograms and the tile list are fully rewritten by every call.
+  // The status word is the scratch that must start at zero; the histograms
+  // and the tile list are fully rewritten by every call.
   cudaError_t e = cudaMemsetAsync(scratch, 0, kHeaderWords * sizeof(int32_t), st);
   if (e != cudaSuccess) return noalloc_fail(LMOE_ECUDA, "clear status: %s", cudaGetErrorString(e));
   const int64_t hist = (int64_t)dispatch_blocks(N * k) * R;
   DispatchScratch ds;
   ds.status = scratch;
   ds.n_mtiles = scratch + 1;
-  ds.ticket = scratch + 2;
   ds.block_counts = scratch + kHeaderWords;
   ds.tiles = reinterpret_cast<int4*>(scratch + kHeaderWords + (hist + 3) / 4 * 4);
   e = launch_dispatch(ids, N, k, R, counts, offsets, perm_token, inv_pair, ds, st);
