@@ -225,6 +225,70 @@ def run_reference(args, wl):
     return 0
 
 
+def run_memory_kernels(args, wl):
+    """Routing, dispatch and combine called on their own through the C ABI at the
+    workload's shapes (synthetic activations; no expert weights), each timed with
+    CUDA events over --steps calls with L2 flushed in between.  Prints one JSON
+    line per entry point: algorithmic bytes per call (the survey's definitions),
+    time, and the fraction of the roof max(bytes / HBM, FLOPs / bf16 peak)."""
+    import torch
+    import sigmoid_top_routing_latentmoe_b200 as lm
+    torch.cuda.set_device(0)
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    N, d, L, R, k = wl.n_tokens, wl.d, wl.latent, wl.n_routed, wl.top_k
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    es = 2 if wl.dtype == "bf16" else 4
+    P = N * k
+    dims = lm.make_dims(N, d, L, R, k, 0, wl.ff_routed, wl.ff_routed, wl.beta1, wl.beta2,
+                        wl.rms_eps, dt)
+    ws = lm.alloc_workspace(dims)
+    x = torch.randn(N, d, generator=g, device="cuda").to(dt)
+    w_r = (torch.randn(R, d, generator=g, device="cuda") * 0.02).to(dt)
+    ids = torch.empty(N, k, dtype=torch.int32, device="cuda")
+    probs = torch.empty(N, k, dtype=torch.float32, device="cuda")
+    counts = torch.empty(R, dtype=torch.int32, device="cuda")
+    offs = torch.empty(R + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(P, dtype=torch.int32, device="cuda")
+    inv = torch.empty(P, dtype=torch.int32, device="cuda")
+    eo = torch.randn(P, L, generator=g, device="cuda").to(dt)
+    rms_w = torch.ones(L, dtype=torch.float32, device="cuda")
+    u = torch.empty(N, L, dtype=dt, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    calls = {
+        "route": (lambda: lm.moe_route(dims, x, w_r, None, ids, probs, ws),
+                  N * d * es + R * d * es + P * 8, 2.0 * N * d * R),
+        "dispatch": (lambda: lm.moe_dispatch(dims, ids, counts, offs, perm, inv, ws),
+                     P * 4 + P * 8, 0.0),
+        "combine": (lambda: lm.moe_combine(dims, eo, inv, probs, rms_w, u),
+                    P * L * es + P * 8 + N * L * es, 0.0),
+    }
+    peaks = _peaks()
+    for name, (fn, nbytes, flops) in calls.items():
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        us = total / args.steps * 1e3
+        roof_us = max(nbytes / (peaks["hbm_gbs"] * 1e3), flops / (peaks["bf16_tflops"] * 1e6))
+        print(json.dumps({"kernel": name, "workload": wl.name, "us": us, "bytes": nbytes,
+                          "flops": flops, "gb_s": nbytes / us / 1e3,
+                          "hbm_frac": nbytes / us / 1e3 / peaks["hbm_gbs"],
+                          "roof_us": roof_us, "roof_frac": roof_us / us,
+                          "note": ("includes the router-logit GEMM on the tensor cores"
+                                   if R > 32 else "router GEMV on the CUDA cores"
+                                   ) if name == "route" else ""}), flush=True)
+    if lm.get_device_status(ws) != lm.OK:
+        raise SystemExit("device status not OK")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -238,8 +302,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="launch the kernels every step instead of replaying a CUDA graph")
+    ap.add_argument("--memory-kernels", action="store_true",
+                    help="time moe_route / moe_dispatch / moe_combine on their own instead")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
+    if args.memory_kernels:
+        return run_memory_kernels(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     if args.warmup < 3:
