@@ -47,6 +47,7 @@ class _Dims(ctypes.Structure):
         ("beta1", ctypes.c_double),
         ("beta2", ctypes.c_double),
         ("rms_eps", ctypes.c_double),
+        ("router", ctypes.c_int32),
     ]
 
 
@@ -77,8 +78,9 @@ def _load():
                                            _P, _P, _P]
         _lib.orc_rmsnorm_rows.argtypes = [ctypes.c_int64, ctypes.c_int32, _P, _P,
                                           ctypes.c_double, _P]
+        _lib.orc_router_losses.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, _P]
         for f in ("orc_situ", "orc_route", "orc_permute", "orc_forward", "orc_forward_dense",
-                  "orc_rmsnorm_rows"):
+                  "orc_rmsnorm_rows", "orc_router_losses"):
             getattr(_lib, f).restype = None
     return _lib
 
@@ -97,11 +99,12 @@ class Dims:
     beta1: float = 4.0
     beta2: float = 25.0
     rms_eps: float = 1e-6
+    router: int = 0          # 0: K3 sigmoid routing; 1: softmax over the top-k logits
 
     def _c(self) -> _Dims:
         return _Dims(self.n_tokens, self.d, self.latent, self.n_routed, self.top_k,
                      self.n_shared, self.ff_routed, self.ff_shared,
-                     self.beta1, self.beta2, self.rms_eps)
+                     self.beta1, self.beta2, self.rms_eps, self.router)
 
 
 def _f32(a):
@@ -139,7 +142,9 @@ def situ(w_g, w_u, w_o, v, beta1=4.0, beta2=25.0):
 
 
 def route(dims: Dims, x, w_router, expert_bias=None):
-    """K3 routing for all tokens: returns ids [N,k] int32, probs [N,k], keys [N,R], scores [N,R]."""
+    """Routing for all tokens (K3 sigmoid, or dims.router == 1: softmax over the
+    top-k logits): returns ids [N,k] int32, probs [N,k], keys [N,R] (the
+    selection keys), scores [N,R] (sigmoid of the logits)."""
     x, w_router = _f32(x), _f32(w_router)
     b = None if expert_bias is None else _f32(expert_bias)
     N, k, R = dims.n_tokens, dims.top_k, dims.n_routed
@@ -152,6 +157,19 @@ def route(dims: Dims, x, w_router, expert_bias=None):
     _load().orc_route(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(b), _ptr(ids), _ptr(probs),
                       _ptr(keys), _ptr(scores))
     return ids, probs, keys, scores
+
+
+def router_losses(dims: Dims, x, w_router, ids):
+    """Balancing losses before their coefficients: {'aux', 'z', 'frac' [R], 'prob_mean' [R]}."""
+    x, w_router = _f32(x), _f32(w_router)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    R = dims.n_routed
+    assert x.shape == (dims.n_tokens, dims.d) and ids.shape == (dims.n_tokens, dims.top_k)
+    out = np.empty(2 + 2 * R, np.float64)
+    c = dims._c()
+    _load().orc_router_losses(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(ids), _ptr(out))
+    return {"aux": float(out[0]), "z": float(out[1]), "frac": out[2:2 + R].copy(),
+            "prob_mean": out[2 + R:].copy()}
 
 
 def permute(ids, n_routed: int):

@@ -54,7 +54,7 @@ def enforce_topk_margin(wl: synth.Workload, inputs: dict, seed: int = 0, margin:
             return {"redrawn": redrawn, "rounds": rnd - 1}
         xf = synth.to_f32(x[todo])
         dims = Dims(len(todo), wl.d, wl.latent, wl.n_routed, wl.top_k, wl.n_shared,
-                    wl.ff_routed, wl.ff_shared)
+                    wl.ff_routed, wl.ff_shared, router=wl.router)
         _, _, keys, _ = route(dims, xf, w_r, b)
         bad = todo[(topk_gap(keys, wl.top_k) < margin) |
                    (order_gap(keys, wl.top_k) < order_margin)]

@@ -17,7 +17,11 @@
  *            SiTU.forward, LatentMoE._route, LatentMoE._routed_u,
  *            LatentMoE.forward.
  *   [tests]  same compare view, tests/integration/test_k3_arch.py:
- *            _dense_moe_forward and test_moe_router_activates_topk_only.
+ *            _dense_moe_forward, test_moe_router_activates_topk_only and
+ *            test_moe_aux_loss_penalizes_collapse.
+ *   [prior]  the lines the compare view removes from LatentMoE.forward: the
+ *            earlier router, TopK on the raw logits with the weights a
+ *            softmax over the k selected logits.
  *
  * Precision: every input arrives as float (bf16 inputs are the exact bf16
  * values widened to float); every product and sum is formed in double and
@@ -50,6 +54,7 @@ typedef struct {
   double beta1;      /* SiTU gate soft cap (4)                    */
   double beta2;      /* SiTU up soft cap (25)                     */
   double rms_eps;    /* RMSNorm epsilon                           */
+  int32_t router;    /* 0: K3 sigmoid routing; 1: softmax over the top-k logits ([prior]) */
 } orc_dims;
 
 /* Logistic function.  The two branches are the same function; the second
@@ -101,11 +106,14 @@ void orc_situ(int32_t dim_in, int32_t ff, double beta1, double beta2,
  *   l = W_r x,  s = sigmoid(l),  T = TopK(s + b, k),
  *   p_i = s_i / max(sum_{j in T} s_j, 1e-9).
  * The bias b enters the selection only; p uses the raw scores s.
+ * router == 1 is the earlier router ([prior]): T = TopK(l, k) on the raw
+ * logits (no bias), p = softmax over the k selected logits,
+ *   p_i = exp(l_i - l_max) / sum_{j in T} exp(l_j - l_max).
  * ids/probs: [k] in slot order (key descending, ties to the lower index).
- * keys (optional): [R] receives s + b. */
-static void orc_route_token(int32_t d, int32_t R, int32_t k, const float* x, const float* w_r,
-                            const float* bias, int32_t* ids, double* probs, double* keys_out,
-                            double* scores_out) {
+ * keys (optional): [R] receives the selection keys (s + b, or l). */
+static void orc_route_token(int32_t d, int32_t R, int32_t k, int32_t router, const float* x,
+                            const float* w_r, const float* bias, int32_t* ids, double* probs,
+                            double* keys_out, double* scores_out) {
   double* l = (double*)malloc(sizeof(double) * (size_t)R);
   double* s = (double*)malloc(sizeof(double) * (size_t)R);
   double* key = (double*)malloc(sizeof(double) * (size_t)R);
@@ -115,7 +123,7 @@ static void orc_route_token(int32_t d, int32_t R, int32_t k, const float* x, con
   orc_linear(w_r, R, d, xv, l);
   for (int32_t e = 0; e < R; ++e) {
     s[e] = orc_sigmoid(l[e]);
-    key[e] = s[e] + (bias ? (double)bias[e] : 0.0);
+    key[e] = router == 1 ? l[e] : s[e] + (bias ? (double)bias[e] : 0.0);
   }
   /* k rounds of "largest remaining key"; strict '>' keeps the lower index on a tie. */
   for (int32_t slot = 0; slot < k; ++slot) {
@@ -127,10 +135,18 @@ static void orc_route_token(int32_t d, int32_t R, int32_t k, const float* x, con
     taken[best] = 1;
     ids[slot] = best;
   }
-  double den = 0.0;
-  for (int32_t slot = 0; slot < k; ++slot) den += s[ids[slot]];
-  if (den < 1e-9) den = 1e-9;
-  for (int32_t slot = 0; slot < k; ++slot) probs[slot] = s[ids[slot]] / den;
+  if (router == 1) {
+    /* softmax over the selected logits; slot 0 holds the largest */
+    const double lmax = l[ids[0]];
+    double den = 0.0;
+    for (int32_t slot = 0; slot < k; ++slot) den += exp(l[ids[slot]] - lmax);
+    for (int32_t slot = 0; slot < k; ++slot) probs[slot] = exp(l[ids[slot]] - lmax) / den;
+  } else {
+    double den = 0.0;
+    for (int32_t slot = 0; slot < k; ++slot) den += s[ids[slot]];
+    if (den < 1e-9) den = 1e-9;
+    for (int32_t slot = 0; slot < k; ++slot) probs[slot] = s[ids[slot]] / den;
+  }
   if (keys_out) memcpy(keys_out, key, sizeof(double) * (size_t)R);
   if (scores_out) memcpy(scores_out, s, sizeof(double) * (size_t)R);
   free(l);
@@ -148,7 +164,7 @@ void orc_route(const orc_dims* dm, const float* x, const float* w_r, const float
   const int32_t d = dm->d, R = dm->n_routed, k = dm->top_k;
 #pragma omp parallel for schedule(dynamic, 16)
   for (int64_t t = 0; t < N; ++t) {
-    orc_route_token(d, R, k, x + t * d, w_r, bias, ids + t * k, probs + t * k,
+    orc_route_token(d, R, k, dm->router, x + t * d, w_r, bias, ids + t * k, probs + t * k,
                     keys ? keys + t * R : NULL, scores ? scores + t * R : NULL);
   }
 }
@@ -230,7 +246,8 @@ static void orc_forward_token(const orc_dims* dm, const orc_weights* w, const fl
   /* step 1: latent compression */
   orc_linear(w->w_down, L, d, xv, z);
   /* step 2: routing on the full-width x (not z) */
-  orc_route_token(d, R, k, x_t, w->w_router, w->expert_bias, ids_t, probs_t, NULL, NULL);
+  orc_route_token(d, R, k, dm->router, x_t, w->w_router, w->expert_bias, ids_t, probs_t, NULL,
+                  NULL);
   /* step 3: routed experts, slots in order */
   for (int32_t slot = 0; slot < k; ++slot) {
     const int64_t e = ids_t[slot];
@@ -301,7 +318,8 @@ void orc_forward_dense(const orc_dims* dm, const orc_weights* w, const float* x,
     double* probs = (double*)malloc(sizeof(double) * (size_t)k);
     for (int32_t i = 0; i < d; ++i) xv[i] = (double)x_t[i];
     orc_linear(w->w_down, L, d, xv, z);
-    orc_route_token(d, R, k, x_t, w->w_router, w->expert_bias, ids, probs, NULL, NULL);
+    orc_route_token(d, R, k, dm->router, x_t, w->w_router, w->expert_bias, ids, probs, NULL,
+                    NULL);
     for (int32_t e = 0; e < R; ++e)
       orc_situ(L, F, dm->beta1, dm->beta2, w->w_g + (int64_t)e * F * L,
                w->w_u + (int64_t)e * F * L, w->w_o + (int64_t)e * L * F, z,
@@ -333,4 +351,50 @@ void orc_forward_dense(const orc_dims* dm, const orc_weights* w, const float* x,
 void orc_rmsnorm_rows(int64_t N, int32_t n, const double* u, const float* w, double eps,
                       double* out) {
   for (int64_t t = 0; t < N; ++t) orc_rmsnorm(n, u + t * n, w, eps, out + t * n);
+}
+
+/* Router balancing losses ([diff] LatentMoE._balancing_losses; [tests]
+ * test_moe_aux_loss_penalizes_collapse), before their coefficients:
+ *   counts_e    = number of pairs routed to expert e        (bincount of ids)
+ *   frac_e      = counts_e / max(sum_e counts_e, 1)
+ *   prob_mean_e = mean over tokens of sigmoid(l_te)         (l = W_r x)
+ *   aux         = R * sum_e frac_e * prob_mean_e            (Switch/GShard form on sigmoid scores)
+ *   z           = mean over tokens of logsumexp_e(l_te)^2   (z-loss on the raw logits)
+ * out: [2 + 2R] = aux, z, frac[R], prob_mean[R].  logsumexp is formed as
+ * m + log(sum exp(l - m)) with m the row maximum. */
+void orc_router_losses(const orc_dims* dm, const float* x, const float* w_r, const int32_t* ids,
+                       double* out) {
+  const int64_t N = dm->n_tokens;
+  const int32_t d = dm->d, R = dm->n_routed, k = dm->top_k;
+  double* frac = out + 2;
+  double* pmean = out + 2 + R;
+  double* l = (double*)malloc(sizeof(double) * (size_t)R);
+  double* xv = (double*)malloc(sizeof(double) * (size_t)d);
+  double z = 0.0, total = 0.0;
+  for (int32_t e = 0; e < R; ++e) frac[e] = pmean[e] = 0.0;
+  for (int64_t i = 0; i < N * k; ++i) frac[ids[i]] += 1.0;
+  for (int32_t e = 0; e < R; ++e) total += frac[e];
+  if (total < 1.0) total = 1.0;
+  for (int32_t e = 0; e < R; ++e) frac[e] /= total;
+  for (int64_t t = 0; t < N; ++t) {
+    for (int32_t i = 0; i < d; ++i) xv[i] = (double)x[t * d + i];
+    orc_linear(w_r, R, d, xv, l);
+    double m = l[0], se = 0.0;
+    for (int32_t e = 1; e < R; ++e) m = l[e] > m ? l[e] : m;
+    for (int32_t e = 0; e < R; ++e) {
+      se += exp(l[e] - m);
+      pmean[e] += orc_sigmoid(l[e]);
+    }
+    const double lse = m + log(se);
+    z += lse * lse;
+  }
+  double aux = 0.0;
+  for (int32_t e = 0; e < R; ++e) {
+    pmean[e] = N > 0 ? pmean[e] / (double)N : 0.0;
+    aux += frac[e] * pmean[e];
+  }
+  out[0] = (double)R * aux;
+  out[1] = N > 0 ? z / (double)N : 0.0;
+  free(l);
+  free(xv);
 }

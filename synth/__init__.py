@@ -134,20 +134,22 @@ class Workload:
     beta1: float = 4.0
     beta2: float = 25.0
     rms_eps: float = 1e-6
+    router: int = 0               # 0: K3 sigmoid routing; 1: softmax over the top-k logits
     extra: dict = field(default_factory=dict, compare=False)
 
     def with_tokens(self, n: int) -> "Workload":
         return Workload(self.name, n, self.d, self.latent, self.n_routed, self.top_k,
                         self.ff_routed, self.n_shared, self.ff_shared, self.dtype, self.bias,
                         self.skew_experts, self.x_std, self.w_std, self.beta1, self.beta2,
-                        self.rms_eps)
+                        self.rms_eps, self.router)
 
     def replace(self, **kw) -> "Workload":
         fields = dict(name=self.name, n_tokens=self.n_tokens, d=self.d, latent=self.latent,
                       n_routed=self.n_routed, top_k=self.top_k, ff_routed=self.ff_routed,
                       n_shared=self.n_shared, ff_shared=self.ff_shared, dtype=self.dtype,
                       bias=self.bias, skew_experts=self.skew_experts, x_std=self.x_std,
-                      w_std=self.w_std, beta1=self.beta1, beta2=self.beta2, rms_eps=self.rms_eps)
+                      w_std=self.w_std, beta1=self.beta1, beta2=self.beta2, rms_eps=self.rms_eps,
+                      router=self.router)
         fields.update(kw)
         return Workload(**fields)
 

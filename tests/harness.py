@@ -17,7 +17,8 @@ P_ABS_TOL = 1e-6       # routing weights
 
 def odims(wl: synth.Workload, n=None) -> oracle.Dims:
     return oracle.Dims(wl.n_tokens if n is None else n, wl.d, wl.latent, wl.n_routed, wl.top_k,
-                       wl.n_shared, wl.ff_routed, wl.ff_shared, wl.beta1, wl.beta2, wl.rms_eps)
+                       wl.n_shared, wl.ff_routed, wl.ff_shared, wl.beta1, wl.beta2, wl.rms_eps,
+                       wl.router)
 
 
 def ldims(wl: synth.Workload, n=None):

@@ -399,3 +399,130 @@ def test_margin_conditioning_reaches_the_margin():
     _, _, keys, _ = oracle.route(dims, synth.to_f32(inp["x"]), synth.to_f32(inp["w_router"]),
                                  inp["expert_bias"])
     assert topk_gap(keys, wl.top_k).min() >= 1e-3
+
+
+# ------------------------------------------------- earlier router (softmax over top-k)
+
+def _prior(dims: oracle.Dims) -> oracle.Dims:
+    return oracle.Dims(dims.n_tokens, dims.d, dims.latent, dims.n_routed, dims.top_k,
+                       dims.n_shared, dims.ff_routed, dims.ff_shared, router=1)
+
+
+@pytest.mark.parametrize("R,k", [(6, 1), (6, 2), (8, 3), (9, 4), (7, 7)])
+def test_prior_router_selects_the_largest_logits(R, k):
+    """router = 1: T = TopK(l, k) on the raw logits, bias ignored; brute force over
+    all C(R,k) subsets and numpy's stable argsort of -l."""
+    dims = _prior(oracle.Dims(30, 10, 6, R, k, 1, 4, 4))
+    rng = np.random.default_rng(7 * R + k)
+    x = rng.standard_normal((30, 10)).astype(np.float32)
+    w_r = rng.standard_normal((R, 10)).astype(np.float32)
+    b = (5.0 * rng.standard_normal(R)).astype(np.float32)   # large, and must not matter
+    ids, probs, keys, _ = oracle.route(dims, x, w_r, b)
+    ids0, probs0, _, _ = oracle.route(dims, x, w_r, None)
+    np.testing.assert_array_equal(ids, ids0)
+    np.testing.assert_array_equal(probs, probs0)
+    for t in range(30):
+        l = w_r.astype(np.float64) @ x[t].astype(np.float64)
+        np.testing.assert_allclose(keys[t], l, rtol=1e-13)
+        best = max(itertools.combinations(range(R), k), key=lambda c: sum(l[list(c)]))
+        assert set(ids[t]) == set(best)
+        assert list(ids[t]) == list(np.argsort(-l, kind="stable")[:k])
+
+
+def test_prior_router_weights():
+    """Softmax over the selected logits: Σp = 1, p decreasing with the slot, k = 1
+    gives 1, and for k = 2 the first weight is the logistic of the logit gap."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((50, 16)).astype(np.float32)
+    w_r = rng.standard_normal((8, 16)).astype(np.float32)
+    for k in (1, 2, 4):
+        dims = _prior(oracle.Dims(50, 16, 8, 8, k, 1, 4, 4))
+        ids, probs, keys, _ = oracle.route(dims, x, w_r)
+        np.testing.assert_allclose(probs.sum(1), 1.0, rtol=0, atol=1e-15)
+        assert (np.diff(probs, axis=1) <= 0).all()
+        if k == 1:
+            np.testing.assert_array_equal(probs, 1.0)
+        if k == 2:
+            gap = keys[np.arange(50), ids[:, 0]] - keys[np.arange(50), ids[:, 1]]
+            np.testing.assert_allclose(probs[:, 0], 1.0 / (1.0 + np.exp(-gap)), rtol=1e-13)
+
+
+def test_prior_router_is_shift_invariant():
+    """Adding one constant to every logit (a constant input channel whose router
+    column is the constant) changes neither the selection nor the weights."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((40, 12)).astype(np.float32)
+    w_r = rng.standard_normal((8, 12)).astype(np.float32)
+    x[:, -1] = 1.0
+    w_r[:, -1] = 0.0
+    dims = _prior(oracle.Dims(40, 12, 6, 8, 3, 1, 4, 4))
+    ids0, p0, _, _ = oracle.route(dims, x, w_r)
+    w_r[:, -1] = 7.5
+    ids1, p1, _, _ = oracle.route(dims, x, w_r)
+    np.testing.assert_array_equal(ids0, ids1)
+    np.testing.assert_allclose(p0, p1, rtol=1e-12)
+
+
+# ------------------------------------------------------------ router balancing losses
+
+def test_router_losses_with_zero_router():
+    """W_r = 0: every logit is 0, every score 1/2, so prob_mean = 1/2, aux = R/2
+    (frac sums to 1) and z = (ln R)^2."""
+    for R, k in ((8, 2), (16, 4), (5, 5)):
+        dims = oracle.Dims(20, 10, 6, R, k, 1, 4, 4)
+        x = np.random.default_rng(R).standard_normal((20, 10)).astype(np.float32)
+        w_r = np.zeros((R, 10), np.float32)
+        ids, _, _, _ = oracle.route(dims, x, w_r)
+        out = oracle.router_losses(dims, x, w_r, ids)
+        np.testing.assert_allclose(out["prob_mean"], 0.5, rtol=1e-15)
+        assert out["frac"].sum() == pytest.approx(1.0, rel=1e-15)
+        assert out["aux"] == pytest.approx(R / 2.0, rel=1e-14)
+        assert out["z"] == pytest.approx(math.log(R) ** 2, rel=1e-13)
+
+
+def test_router_losses_collapsed_case_of_the_pages():
+    """The pages' collapse test: router rows 0 := 1, 1 := 0.5, x = 1.  Every token
+    picks {0, 1}, so frac = (1/2, 1/2, 0...), logits (32, 16, 0 x 6):
+    aux = R (sigma(32) + sigma(16)) / 2, z = (32 + ln(1 + e^-16 + 6 e^-32))^2.
+    The page asserts aux > 1.2, aux above the random-router value, and z > 0."""
+    with open(os.path.join(GOLDEN, "collapsed_router_losses.json")) as f:
+        g = json.load(f)
+    d, R, k = g["hidden_size"], g["n_routed"], g["top_k"]
+    n = int(np.prod(g["x_shape"][:-1]))
+    dims = oracle.Dims(n, d, 16, R, k, 1, 24, 24)
+    w_r = np.zeros((R, d), np.float32)
+    for row, val in g["router_rows"].items():
+        w_r[int(row)] = val
+    x = np.full((n, d), g["x_value"], np.float32)
+    ids, _, _, _ = oracle.route(dims, x, w_r)
+    out = oracle.router_losses(dims, x, w_r, ids)
+    np.testing.assert_allclose(out["frac"], [0.5, 0.5] + [0.0] * (R - 2), rtol=0, atol=0)
+    assert out["aux"] == pytest.approx(R * (_sig(32.0) + _sig(16.0)) / 2.0, rel=1e-14)
+    assert out["z"] == pytest.approx((32.0 + math.log1p(math.exp(-16.0) + 6 * math.exp(-32.0))) ** 2,
+                                     rel=1e-14)
+    assert out["aux"] > g["asserted"]["aux_collapsed_greater_than"]
+    assert out["z"] > g["asserted"]["z_greater_than"]
+    rng = np.random.default_rng(0)
+    xs = rng.standard_normal((n, d)).astype(np.float32)
+    ws = (rng.standard_normal((R, d)) / math.sqrt(d)).astype(np.float32)
+    ids_s, _, _, _ = oracle.route(dims, xs, ws)
+    assert out["aux"] > oracle.router_losses(dims, xs, ws, ids_s)["aux"]
+
+
+def test_router_losses_frac_is_the_routing_histogram_and_token_order_free():
+    """frac = counts / (N k) from the permutation's counts; aux and z do not depend
+    on the token order; aux <= R * max prob_mean."""
+    dims = oracle.Dims(64, 24, 12, 12, 3, 1, 8, 8)
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((64, 24)).astype(np.float32)
+    w_r = (rng.standard_normal((12, 24)) * 0.4).astype(np.float32)
+    ids, _, _, _ = oracle.route(dims, x, w_r)
+    out = oracle.router_losses(dims, x, w_r, ids)
+    counts, _, _, _ = oracle.permute(ids, 12)
+    np.testing.assert_allclose(out["frac"], counts / (64 * 3), rtol=1e-15)
+    perm = rng.permutation(64)
+    out2 = oracle.router_losses(dims, x[perm], w_r, ids[perm])
+    assert out2["aux"] == pytest.approx(out["aux"], rel=1e-13)
+    assert out2["z"] == pytest.approx(out["z"], rel=1e-13)
+    assert out["aux"] <= 12 * out["prob_mean"].max() + 1e-12
+    assert ((out["prob_mean"] > 0) & (out["prob_mean"] < 1)).all()
