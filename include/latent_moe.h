@@ -79,7 +79,17 @@ typedef struct {
   float beta2;      /* SiTU up cap (pages: 25)              */
   float rms_eps;    /* RMSNorm epsilon (1e-6)               */
   int32_t dtype;    /* lmoe_dtype                           */
+  int32_t router;   /* lmoe_router: which routing rule      */
 } lmoe_dims;
+
+/* Routing rules.  LMOE_ROUTER_K3 is the layer's (sec-07 K3 eq.13):
+ * s = sigmoid(l), T = TopK(s + b, k), p = s_T / max(sum s_T, 1e-9).
+ * LMOE_ROUTER_SOFTMAX_TOPK is the router that latent_moe.py had before it
+ * (the lines the compare view removes from LatentMoE.forward): T = TopK(l, k)
+ * on the raw logits, expert_bias unused, p = softmax over the k selected
+ * logits.  Either way the slots are in descending key order, a tie going to
+ * the lower expert index. */
+typedef enum { LMOE_ROUTER_K3 = 0, LMOE_ROUTER_SOFTMAX_TOPK = 1 } lmoe_router;
 
 /* Layer weights, device pointers in nn.Linear layout. */
 typedef struct {
@@ -103,12 +113,13 @@ LMOE_API size_t lmoe_workspace_size(const lmoe_dims* dims);
 /* Router (sec-07 compute flow step 2, K3 eq.13; latent_moe.py LatentMoE._route):
  * l = W_r x (fp32 accumulation), s = sigmoid(l), T = TopK(s + b, k) with the
  * slots in descending s + b (a tie goes to the lower expert index),
- * p_i = s_i / max(sum_T s, 1e-9).
+ * p_i = s_i / max(sum_T s, 1e-9).  dims->router selects the rule (lmoe_router).
  *   x        [N, d]      input rows
  *   w_router [R, d]
  *   expert_bias [R] fp32 or NULL
  *   ids      [N, k] int32 out;  probs [N, k] fp32 out.
- * Workspace: lmoe_workspace_size(dims) bytes. */
+ * Workspace: lmoe_workspace_size(dims) bytes; the logits l are left in it (see
+ * moe_router_losses). */
 LMOE_API lmoe_status moe_route(const lmoe_dims* dims, const void* x, const void* w_router,
                       const float* expert_bias, int32_t* ids, float* probs, void* ws,
                       size_t ws_bytes, lmoe_stream stream);
@@ -151,9 +162,27 @@ LMOE_API lmoe_status moe_combine(const lmoe_dims* dims, const void* expert_out, 
                         const float* probs, const float* rms_weight, void* u_normed,
                         lmoe_stream stream);
 
+/* Router balancing losses (latent_moe.py LatentMoE._balancing_losses; the
+ * pages' test_moe_aux_loss_penalizes_collapse), before their coefficients:
+ *   frac_e      = (pairs routed to e) / max(N*k, 1)
+ *   prob_mean_e = mean_t sigmoid(l_te)
+ *   aux         = R * sum_e frac_e * prob_mean_e
+ *   z           = mean_t (logsumexp_e l_te)^2
+ * The pages multiply them by aux_loss_coef and z_loss_coef.
+ *   logits [N, ld] fp32, or NULL for the logits that the last moe_route or
+ *          latent_moe_forward on this workspace left in it (ld is then ignored)
+ *   ids    [N, k] int32: the routing whose histogram gives frac
+ *   out    [2 + 2R] fp32 device memory out: aux, z, frac[R], prob_mean[R]
+ * Deterministic (fixed-order fp32 sums, integer histograms).  Workspace:
+ * lmoe_workspace_size(dims) bytes. */
+LMOE_API lmoe_status moe_router_losses(const lmoe_dims* dims, const float* logits, int64_t ld,
+                                       const int32_t* ids, float* out, void* ws, size_t ws_bytes,
+                                       lmoe_stream stream);
+
 /* The whole layer: y [N, d] = s_sh + W_up RMSNorm(u).  Optional outputs (NULL
  * to skip): ids_out [N, k], probs_out [N, k], counts_out [R].  All work is on
- * `stream`; no host synchronisation. */
+ * `stream`; no host synchronisation.  The router logits stay in the
+ * workspace for moe_router_losses. */
 LMOE_API lmoe_status latent_moe_forward(const lmoe_dims* dims, const lmoe_weights* weights, const void* x,
                                void* y, int32_t* ids_out, float* probs_out, int32_t* counts_out,
                                void* ws, size_t ws_bytes, lmoe_stream stream);

@@ -40,7 +40,8 @@ class Dims(ctypes.Structure):
                 ("n_routed", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("n_shared", ctypes.c_int32), ("ff_routed", ctypes.c_int32),
                 ("ff_shared", ctypes.c_int32), ("beta1", ctypes.c_float),
-                ("beta2", ctypes.c_float), ("rms_eps", ctypes.c_float), ("dtype", ctypes.c_int32)]
+                ("beta2", ctypes.c_float), ("rms_eps", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("router", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -63,6 +64,7 @@ _sigs = {
     "moe_dispatch_noalloc": (_S, [_DP, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn": (_S, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (_S, [_DP, _P, _P, _P, _P, _P, _P]),
+    "moe_router_losses": (_S, [_DP, _P, ctypes.c_int64, _P, _P, _P, ctypes.c_size_t, _P]),
     "latent_moe_forward": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, _P, _P, _P, _P,
                                 ctypes.c_size_t, _P]),
     "latent_moe_forward_host": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, _P, ctypes.c_size_t,
@@ -87,11 +89,15 @@ for _name, (_res, _args) in _sigs.items():
     _f.argtypes = _args
 
 
+ROUTER_K3, ROUTER_SOFTMAX_TOPK = 0, 1
+
+
 def make_dims(n_tokens, d, latent, n_routed, top_k, n_shared, ff_routed, ff_shared,
-              beta1=4.0, beta2=25.0, rms_eps=1e-6, dtype=torch.bfloat16) -> Dims:
+              beta1=4.0, beta2=25.0, rms_eps=1e-6, dtype=torch.bfloat16,
+              router=ROUTER_K3) -> Dims:
     code = {torch.bfloat16: BF16, torch.float32: F32}[dtype]
     return Dims(n_tokens, d, latent, n_routed, top_k, n_shared, ff_routed, ff_shared,
-                beta1, beta2, rms_eps, code)
+                beta1, beta2, rms_eps, code, router)
 
 
 def _ptr(t):
@@ -186,6 +192,13 @@ def moe_expert_ffn(dims, z, perm_token, offsets, w_g, w_u, w_o, expert_out, ws, 
 def moe_combine(dims, expert_out, inv_pair, probs, rms_weight, u_normed, stream=None):
     _check(_lib.moe_combine(ctypes.byref(dims), _ptr(expert_out), _ptr(inv_pair), _ptr(probs),
                             _ptr(rms_weight), _ptr(u_normed), _stream(stream)), "moe_combine")
+
+
+def moe_router_losses(dims, ids, out, ws, logits=None, ld=0, stream=None):
+    """out [2 + 2R] fp32 <- aux, z, frac[R], prob_mean[R] (logits=None: those left
+    in ``ws`` by the last moe_route / latent_moe_forward)."""
+    _check(_lib.moe_router_losses(ctypes.byref(dims), _ptr(logits), ld, _ptr(ids), _ptr(out),
+                                  _ptr(ws), ws.numel(), _stream(stream)), "moe_router_losses")
 
 
 def latent_moe_forward(dims, weights, x, y, ws, ids_out=None, probs_out=None, counts_out=None,

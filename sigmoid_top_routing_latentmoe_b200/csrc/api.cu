@@ -117,6 +117,8 @@ static lmoe_status check_dims(const lmoe_dims* d) {
     return fail(LMOE_EUNSUPPORTED, "n_tokens * top_k too large");
   if (!(d->beta1 > 0.0f) || !(d->beta2 > 0.0f) || !(d->rms_eps >= 0.0f))
     return fail(LMOE_EINVAL, "beta1, beta2 must be > 0 and rms_eps >= 0");
+  if (d->router != LMOE_ROUTER_K3 && d->router != LMOE_ROUTER_SOFTMAX_TOPK)
+    return fail(LMOE_EINVAL, "router %d", d->router);
   return LMOE_OK;
 }
 
@@ -131,7 +133,7 @@ static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
   size_t header, z, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, zp, h, eo,
-      hsh, uhat, x, y, total;
+      hsh, uhat, loss, x, y, total;
   int64_t logits_ld;
   int max_tiles;
 };
@@ -161,6 +163,8 @@ static Layout layout(const lmoe_dims* d, bool host_copies) {
   L.eo = take((size_t)P * d->latent * es);
   L.hsh = take((size_t)N * d->n_shared * (size_t)d->ff_shared * es);
   L.uhat = take((size_t)N * d->latent * es);
+  // scratch of moe_router_losses: per block of tokens, R sigmoid sums, R counts, one z sum
+  L.loss = take((size_t)loss_blocks(N) * (2 * (size_t)R + 1) * 4);
   if (host_copies) {
     L.x = take((size_t)N * d->d * es);
     L.y = take((size_t)N * d->d * es);
@@ -196,14 +200,14 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
   const Layout L = layout(d, false);
   const int64_t N = d->n_tokens;
   if (N == 0) return LMOE_OK;
+  float* logits = at<float>(ws, L.logits);
   if (d->n_routed <= 32) {
     ProfScope ps("route", st);
     LMOE_CUDA(launch_route_gemv<T>((const T*)x, (const T*)w_r, bias, N, d->d, d->n_routed,
-                                   d->top_k, ids, probs, st),
+                                   d->top_k, d->router, ids, probs, logits, L.logits_ld, st),
               "route_gemv");
     return LMOE_OK;
   }
-  float* logits = at<float>(ws, L.logits);
   ProfScope ps("route", st);
   if (std::is_same<T, __nv_bfloat16>::value) {
     XpassArgs a{};
@@ -218,7 +222,8 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
     g.mode = kStore;
     LMOE_CUDA(launch_simt_gemm<T>(g, st), "router logits");
   }
-  LMOE_CUDA(launch_route_topk(logits, L.logits_ld, bias, N, d->n_routed, d->top_k, ids, probs, st),
+  LMOE_CUDA(launch_route_topk(logits, L.logits_ld, bias, N, d->n_routed, d->top_k, d->router, ids,
+                              probs, st),
             "route_topk");
   return LMOE_OK;
 }
@@ -332,13 +337,14 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
     a.ws_g = (const T*)w->ws_g; a.ws_u = (const T*)w->ws_u; a.S = S; a.G = G;
     a.z = z; a.logits = logits; a.logits_ld = L.logits_ld;
     a.hsh = hsh; a.beta1 = d->beta1; a.beta2 = d->beta2;
-    a.bias = w->expert_bias; a.ids = ids; a.probs = probs; a.top_k = k;
+    a.bias = w->expert_bias; a.ids = ids; a.probs = probs; a.top_k = k; a.router = d->router;
     ProfScope ps("xpass", st);
     LMOE_CUDA(umma_xpass(a, status, st), "x-pass (tcgen05)");
   }
   if (R > 32) {
     ProfScope ps("route", st);
-    LMOE_CUDA(launch_route_topk(logits, L.logits_ld, w->expert_bias, N, R, k, ids, probs, st),
+    LMOE_CUDA(launch_route_topk(logits, L.logits_ld, w->expert_bias, N, R, k, d->router, ids,
+                                probs, st),
               "route_topk");
   }
   // step 3: dispatch, routed experts, combine + RMSNorm
@@ -521,6 +527,33 @@ lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const int32_t* 
   if (dims->dtype == LMOE_BF16)
     return run_expert_ffn<__nv_bfloat16>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
   return run_expert_ffn<float>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
+}
+
+lmoe_status moe_router_losses(const lmoe_dims* dims, const float* logits, int64_t ld,
+                              const int32_t* ids, float* out, void* ws, size_t ws_bytes,
+                              lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  LMOE_PTR(out, "out");
+  if (dims->n_tokens > 0) LMOE_PTR(ids, "ids");
+  LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
+  const Layout L = layout(dims, false);
+  if (logits == nullptr) {
+    logits = at<float>(ws, L.logits);
+    ld = L.logits_ld;
+  } else if (ld < dims->n_routed || (uintptr_t)logits % 4 != 0) {
+    return fail(LMOE_EINVAL, "logits: ld < n_routed or misaligned");
+  }
+  LMOE_TRY(check_device());
+  const int64_t nb = loss_blocks(dims->n_tokens);
+  float* part_s = at<float>(ws, L.loss);
+  int32_t* part_c = reinterpret_cast<int32_t*>(part_s + nb * dims->n_routed);
+  float* part_z = reinterpret_cast<float*>(part_c + nb * dims->n_routed);
+  ProfScope ps("router_losses", (cudaStream_t)stream);
+  LMOE_CUDA(launch_router_losses(logits, ld, ids, dims->n_tokens, dims->top_k, dims->n_routed,
+                                 part_s, part_c, part_z, &at<WsHeader>(ws, L.header)->status, out,
+                                 (cudaStream_t)stream),
+            "router losses");
+  return LMOE_OK;
 }
 
 lmoe_status moe_combine(const lmoe_dims* dims, const void* expert_out, const int32_t* inv_pair,

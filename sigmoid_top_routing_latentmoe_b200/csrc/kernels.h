@@ -10,11 +10,24 @@ namespace lmoe {
 // Warp-per-token router for small R (<= 32): fp32 GEMV over W_r, sigmoid,
 // biased top-k in registers, L1 normalisation.  T = float or bf16.
 template <typename T>
+// router: 0 K3 sigmoid rule, 1 softmax over the top-k logits.  logits_out
+// (row stride ld) receives the fp32 logits when not null.
 cudaError_t launch_route_gemv(const T* x, const T* w_r, const float* bias, int64_t n, int d, int R,
-                              int k, int32_t* ids, float* probs, cudaStream_t st);
+                              int k, int router, int32_t* ids, float* probs, float* logits_out,
+                              int64_t ld, cudaStream_t st);
 // Top-k + normalisation from precomputed fp32 logits [n, ld] (R valid columns).
 cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias, int64_t n, int R,
-                              int k, int32_t* ids, float* probs, cudaStream_t st);
+                              int k, int router, int32_t* ids, float* probs, cudaStream_t st);
+
+// ------------------------------------------------------ router balancing losses
+// Blocks of this many tokens each leave fixed-order partial sums.
+constexpr int kLossRows = 256;
+inline int loss_blocks(int64_t n) { return (int)((n + kLossRows - 1) / kLossRows); }
+// out [2 + 2R] = aux, z, frac[R], prob_mean[R]; part_s / part_c [blocks][R],
+// part_z [blocks] are scratch.
+cudaError_t launch_router_losses(const float* logits, int64_t ld, const int32_t* ids, int64_t n,
+                                 int k, int R, float* part_s, int32_t* part_c, float* part_z,
+                                 int32_t* status, float* out, cudaStream_t st);
 
 // ----------------------------------------------------------- permutation
 struct DispatchScratch {

@@ -1,8 +1,10 @@
 // Router kernels: K3 sigmoid routing (sec-07 compute flow step 2, K3 eq.13;
 // kda/layers/latent_moe.py LatentMoE._route):
 //   l = W_r x,  s = sigmoid(l),  T = TopK(s + b, k),  p_i = s_i / max(sum_T s, 1e-9).
-// The bias enters the selection only.  Slots are written in descending key
-// order; equal keys go to the lower expert index.
+// The bias enters the selection only.  router == 1 is the rule latent_moe.py
+// had before it: T = TopK(l, k), p = softmax over the k selected logits.
+// Slots are written in descending key order; equal keys go to the lower
+// expert index.
 #include "common.cuh"
 #include "kernels.h"
 #include "launch.h"
@@ -26,10 +28,13 @@ __device__ __forceinline__ void warp_argmax(float& key, int& idx) {
 }
 
 // Top-k over R <= 32 * VPL experts held VPL per lane (expert e = j*32 + lane),
-// then p = s / max(sum s, 1e-9).  Called by all 32 lanes of a warp.
+// then p = s / max(sum s, 1e-9); with softmax != 0, s holds the logits and
+// p = exp(s - s_first) / sum over the slots (slot 0 holds the largest).
+// Called by all 32 lanes of a warp.
 template <int VPL>
 __device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (&key_in)[VPL], int R,
-                                            int k, int32_t* ids_row, float* probs_row) {
+                                            int k, int32_t* ids_row, float* probs_row,
+                                            int softmax) {
   const int lane = threadIdx.x & 31;
   float key[VPL];
 #pragma unroll
@@ -37,6 +42,7 @@ __device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (
   float den = 0.0f;
   float sel_s = 0.0f;  // score of the slot this lane will write (lane == slot)
   int sel_id = 0;
+  float first = 0.0f;  // softmax: the largest selected logit
   for (int slot = 0; slot < k; ++slot) {
     float bk = -INFINITY;
     int bi = 0x7fffffff;
@@ -59,6 +65,10 @@ __device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (
       }
     }
     sc = __shfl_sync(0xffffffffu, sc, bi & 31);
+    if (softmax) {
+      if (slot == 0) first = sc;
+      sc = expf(sc - first);
+    }
     den += sc;
     if ((slot & 31) == lane) {
       sel_s = sc;
@@ -72,7 +82,7 @@ __device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (
       if (lane <= (slot & 31)) probs_row[base + lane] = sel_s;
     }
   }
-  den = fmaxf(den, 1e-9f);
+  if (!softmax) den = fmaxf(den, 1e-9f);
   __syncwarp();
   for (int slot = lane; slot < k; slot += 32) probs_row[slot] = probs_row[slot] / den;
 }
@@ -85,9 +95,11 @@ template <typename T, int RMAX>
 __global__ void __launch_bounds__(256) route_gemv_kernel(const T* __restrict__ x,
                                                          const T* __restrict__ w_r,
                                                          const float* __restrict__ bias, int64_t n,
-                                                         int d, int R, int k,
+                                                         int d, int R, int k, int router,
                                                          int32_t* __restrict__ ids,
-                                                         float* __restrict__ probs) {
+                                                         float* __restrict__ probs,
+                                                         float* __restrict__ logits_out,
+                                                         int64_t ld) {
   pdl_trigger();
   pdl_wait();
   constexpr int E = 16 / sizeof(T);  // elements per 16-byte vector
@@ -125,16 +137,21 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(const T* __restrict__ x
 #pragma unroll
   for (int e = 0; e < RMAX; ++e)
     if (e == lane) logit = acc[e];
+  if (logits_out != nullptr && lane < R) logits_out[t * ld + lane] = logit;
   float s[1], key[1];
-  s[0] = sigmoid_f(logit);
-  key[0] = s[0] + ((bias != nullptr && lane < R) ? bias[lane] : 0.0f);
-  select_topk<1>(s, key, R, k, ids + t * k, probs + t * k);
+  if (router) {
+    s[0] = key[0] = logit;
+  } else {
+    s[0] = sigmoid_f(logit);
+    key[0] = s[0] + ((bias != nullptr && lane < R) ? bias[lane] : 0.0f);
+  }
+  select_topk<1>(s, key, R, k, ids + t * k, probs + t * k, router);
 }
 
 template <int VPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
                                                          int64_t ld, const float* __restrict__ bias,
-                                                         int64_t n, int R, int k,
+                                                         int64_t n, int R, int k, int router,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ probs) {
   pdl_trigger();
@@ -148,38 +165,45 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   for (int j = 0; j < VPL; ++j) {
     int e = j * 32 + lane;
     float l = (e < R) ? lr[e] : 0.0f;
-    s[j] = sigmoid_f(l);
-    key[j] = s[j] + ((bias != nullptr && e < R) ? bias[e] : 0.0f);
+    if (router) {
+      s[j] = key[j] = l;
+    } else {
+      s[j] = sigmoid_f(l);
+      key[j] = s[j] + ((bias != nullptr && e < R) ? bias[e] : 0.0f);
+    }
   }
-  select_topk<VPL>(s, key, R, k, ids + t * k, probs + t * k);
+  select_topk<VPL>(s, key, R, k, ids + t * k, probs + t * k, router);
 }
 
 }  // namespace
 
 template <typename T>
 cudaError_t launch_route_gemv(const T* x, const T* w_r, const float* bias, int64_t n, int d, int R,
-                              int k, int32_t* ids, float* probs, cudaStream_t st) {
+                              int k, int router, int32_t* ids, float* probs, float* logits_out,
+                              int64_t ld, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int warps = 8;
   int64_t blocks = (n + warps - 1) / warps;
   cudaError_t e;
   if (R <= 16)
     e = launch_pdl(route_gemv_kernel<T, 16>, dim3((unsigned)blocks), dim3(warps * 32), 0, st, 1, x,
-                   w_r, bias, n, d, R, k, ids, probs);
+                   w_r, bias, n, d, R, k, router, ids, probs, logits_out, ld);
   else
     e = launch_pdl(route_gemv_kernel<T, 32>, dim3((unsigned)blocks), dim3(warps * 32), 0, st, 1, x,
-                   w_r, bias, n, d, R, k, ids, probs);
+                   w_r, bias, n, d, R, k, router, ids, probs, logits_out, ld);
   count_launch();
   return e;
 }
 template cudaError_t launch_route_gemv<float>(const float*, const float*, const float*, int64_t,
-                                              int, int, int, int32_t*, float*, cudaStream_t);
+                                              int, int, int, int, int32_t*, float*, float*,
+                                              int64_t, cudaStream_t);
 template cudaError_t launch_route_gemv<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
-                                                      const float*, int64_t, int, int, int,
-                                                      int32_t*, float*, cudaStream_t);
+                                                      const float*, int64_t, int, int, int, int,
+                                                      int32_t*, float*, float*, int64_t,
+                                                      cudaStream_t);
 
 cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias, int64_t n, int R,
-                              int k, int32_t* ids, float* probs, cudaStream_t st) {
+                              int k, int router, int32_t* ids, float* probs, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int warps = 8;
   unsigned blocks = (unsigned)((n + warps - 1) / warps);
@@ -188,7 +212,7 @@ cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias
   if (vpl <= V) {                                                                          \
     count_launch();                                                                        \
     return launch_pdl(route_topk_kernel<V>, dim3(blocks), dim3(warps * 32), 0, st, 1, logits, \
-                      ld, bias, n, R, k, ids, probs);                                     \
+                      ld, bias, n, R, k, router, ids, probs);                             \
   }
   LMOE_TOPK_CASE(1)
   LMOE_TOPK_CASE(2)

@@ -81,6 +81,7 @@ struct Params {
   int nz_sub, nr_sub, n_zr_tiles, g_blocks;
   int bn;                              // FINAL / ROUTED2 tile width: 128, 192 or 256
   int fuse_topk;                       // XPASS: top-k in the epilogue (R <= 32)
+  int router;                          // 0: K3 sigmoid rule; 1: softmax over the top-k logits
   int top_k;
   const float* bias;
   int32_t* ids;
@@ -682,18 +683,21 @@ __device__ __forceinline__ void pack_block(const float (&a)[32], const float (&b
   }
 }
 
-// K3 routing of one row from its fp32 logits (R <= 32, one TMEM chunk):
-// s = sigmoid(l), T = TopK(s + b, k) in descending key order (ties to the
-// lower expert), p = s_T / max(sum s_T, 1e-9).  Same operations, in the same
-// order, as the standalone top-k kernel.
+// Routing of one row from its fp32 logits (R <= 32, one TMEM chunk): the K3
+// rule s = sigmoid(l), T = TopK(s + b, k) in descending key order (ties to the
+// lower expert), p = s_T / max(sum s_T, 1e-9); or (router == 1) T = TopK(l, k),
+// p = softmax over the selected logits.  Same operations, in the same order,
+// as the standalone top-k kernel.
 __device__ __forceinline__ void route_row32(const Params& p, const float (&lg)[32], int64_t row) {
   float sc[32], key[32];
+  const bool soft = p.router == 1;
 #pragma unroll
   for (int e = 0; e < 32; ++e) {
-    sc[e] = 1.0f / (1.0f + expf(-lg[e]));
-    key[e] = (e < p.R) ? sc[e] + (p.bias != nullptr ? p.bias[e] : 0.0f) : -INFINITY;
+    sc[e] = soft ? lg[e] : 1.0f / (1.0f + expf(-lg[e]));
+    key[e] = (e < p.R) ? (soft ? lg[e] : sc[e] + (p.bias != nullptr ? p.bias[e] : 0.0f))
+                       : -INFINITY;
   }
-  float den = 0.0f;
+  float den = 0.0f, first = 0.0f;
   int32_t* ids = p.ids + row * p.top_k;
   float* probs = p.probs + row * p.top_k;
 #pragma unroll 1
@@ -713,11 +717,15 @@ __device__ __forceinline__ void route_row32(const Params& p, const float (&lg)[3
         sel = sc[e];
         key[e] = -INFINITY;
       }
+    if (soft) {
+      if (slot == 0) first = sel;
+      sel = expf(sel - first);
+    }
     ids[slot] = best;
     probs[slot] = sel;
     den += sel;
   }
-  den = fmaxf(den, 1e-9f);
+  if (!soft) den = fmaxf(den, 1e-9f);
 #pragma unroll 1
   for (int slot = 0; slot < p.top_k; ++slot) probs[slot] = probs[slot] / den;
 }
@@ -784,7 +792,15 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
             if (half == 0) {
               float lg[32];
               tc_ld32(tbase + tl.scol[s], lg);
-              if (lane < rows) route_row32(p, lg, grow0 + lane);
+              if (lane < rows) {
+                float* dst = static_cast<float*>(p.out1) + (grow0 + lane) * p.ld1;
+#pragma unroll
+                for (int g4 = 0; g4 < 8; ++g4)
+                  if (g4 * 4 < p.R)
+                    reinterpret_cast<float4*>(dst)[g4] =
+                        make_float4(lg[g4 * 4], lg[g4 * 4 + 1], lg[g4 * 4 + 2], lg[g4 * 4 + 3]);
+                route_row32(p, lg, grow0 + lane);
+              }
             }
             continue;
           }
@@ -1065,6 +1081,7 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   p.inv_beta2 = 1.0f / a.beta2;
   p.beta12 = a.beta1 * a.beta2;
   p.fuse_topk = (a.ids != nullptr && a.R <= 32) ? 1 : 0;
+  p.router = a.router;
   p.top_k = a.top_k;
   p.bias = a.bias;
   p.ids = a.ids;

@@ -28,7 +28,9 @@ struct XpassArgs {
   __nv_bfloat16* hsh;
   float beta1, beta2;
   // When R <= 32 and ids != nullptr the epilogue also routes each row (K3 top-k
-  // + L1 normalisation with bias b) and writes ids/probs instead of logits.
+  // + L1 normalisation with bias b, or router == 1: top-k of the logits +
+  // softmax) and writes ids/probs; the logits are written either way.
+  int router;
   const float* bias;
   int32_t* ids;
   float* probs;

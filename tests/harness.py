@@ -25,7 +25,7 @@ def ldims(wl: synth.Workload, n=None):
     import sigmoid_top_routing_latentmoe_b200 as lm
     return lm.make_dims(wl.n_tokens if n is None else n, wl.d, wl.latent, wl.n_routed, wl.top_k,
                         wl.n_shared, wl.ff_routed, wl.ff_shared, wl.beta1, wl.beta2, wl.rms_eps,
-                        torch.bfloat16 if wl.dtype == "bf16" else torch.float32)
+                        torch.bfloat16 if wl.dtype == "bf16" else torch.float32, wl.router)
 
 
 def prepare(wl: synth.Workload, seed: int = 0, margin_rows=None, margin: float = MARGIN) -> dict:

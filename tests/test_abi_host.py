@@ -46,6 +46,13 @@ def test_workspace_size_and_validation(lm):
         lm.workspace_size(bad)
     bad = lm.make_dims(4096, 770, 384, 16, 2, 2, 768, 1536)    # d not a multiple of 8
     assert lm._lib.lmoe_workspace_size(ctypes.byref(bad)) == 0
+    bad = lm.make_dims(4096, 768, 384, 16, 2, 2, 768, 1536, router=2)   # no such routing rule
+    assert lm._lib.lmoe_workspace_size(ctypes.byref(bad)) == 0
+    ok = lm.make_dims(4096, 768, 384, 16, 2, 2, 768, 1536, router=lm.ROUTER_SOFTMAX_TOPK)
+    assert lm.workspace_size(ok) == n
+    out_ws = 1 << 20                                # never dereferenced: checks fail first
+    st = lm._lib.moe_router_losses(ctypes.byref(d), None, 0, None, None, out_ws, 0, None)
+    assert st == lm.EINVAL
     # argument errors are reported before anything touches a device
     st = lm._lib.moe_dispatch(ctypes.byref(d), None, None, None, None, None, None, 0, None)
     assert st == lm.EINVAL
