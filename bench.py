@@ -468,7 +468,12 @@ def main():
                 "peak_source": peaks["source"] + (" sustained" if bound == "tensor" else "")}
     else:
         roof = None
-    roof_s = max(wl.flops() / (peaks["bf16_tflops"] * 1e12), wl.compulsory_bytes() / (peaks["hbm_gbs"] * 1e9))
+    # bytes the layer must read: the weights of the experts this input routes to
+    counts = torch.zeros(wl.n_routed, dtype=torch.int32, device=dev)
+    lm.latent_moe_forward(dims, wstruct, x, y, ws, counts_out=counts)
+    used = int((counts > 0).sum().item())
+    cbytes = wl.compulsory_bytes(used)
+    roof_s = max(wl.flops() / (peaks["bf16_tflops"] * 1e12), cbytes / (peaks["hbm_gbs"] * 1e9))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -479,7 +484,7 @@ def main():
                    "n_shared": wl.n_shared, "ff_shared": wl.ff_shared,
                    "parallelism": f"replicas{world}", "l2": "flushed (256 MiB write) between steps",
                    "launch": "eager" if args.eager else "cuda graph replay"},
-        "layer_roofline": {"flops": wl.flops(), "compulsory_bytes": wl.compulsory_bytes(),
+        "layer_roofline": {"flops": wl.flops(), "compulsory_bytes": cbytes, "experts_used": used,
                            "roof_us": roof_s * 1e6, "frac": roof_s / (ms_per_step / 1e3),
                            "peak_source": peaks["source"] + " burst"},
         "roofline": roof,

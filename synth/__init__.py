@@ -160,12 +160,15 @@ class Workload:
         per_tok = 2 * d * L + 2 * d * R + 6 * k * L * F + 6 * S * d * G + 2 * L * d
         return float(per_tok) * self.n_tokens
 
-    def compulsory_bytes(self) -> float:
-        """Every weight once + x + y (intermediates are implementation traffic)."""
+    def compulsory_bytes(self, experts_used=None) -> float:
+        """Every weight once + x + y (intermediates are implementation traffic).
+        experts_used: how many routed experts the routing selected at least once
+        (default all R); only their weights must be read."""
         es = 2 if self.dtype == "bf16" else 4
         d, L, R, F, S, G = (self.d, self.latent, self.n_routed, self.ff_routed, self.n_shared,
                             self.ff_shared)
-        weights = (L * d + R * d + d * L + 3 * R * F * L + 3 * S * G * d) * es + (L + R) * 4
+        used = R if experts_used is None else experts_used
+        weights = (L * d + R * d + d * L + 3 * used * F * L + 3 * S * G * d) * es + (L + R) * 4
         return float(weights + 2 * self.n_tokens * d * es)
 
 
@@ -177,6 +180,9 @@ WORKLOADS = {
     "mid": Workload("mid", 16384, 2048, 1024, 64, 8, 1024, 1, 4096, "bf16",
                     bias=("normal", 0.01)),
     "k3_width": Workload("k3_width", 8192, 7168, 3584, 896, 16, 512, 1, 2048, "bf16"),
+    # a decode-sized step of the K3-width layer: 64 tokens, ~1.1 pairs per expert,
+    # about 610 of the 896 experts selected: streaming their weights dominates
+    "k3_decode": Workload("k3_decode", 64, 7168, 3584, 896, 16, 512, 1, 2048, "bf16"),
 }
 
 

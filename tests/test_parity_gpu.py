@@ -72,7 +72,7 @@ def test_forward_parity_small(name, n):
 
 
 @pytest.mark.parametrize("name,sample", [("halfb_uniform", None), ("halfb_skewed", None),
-                                         ("mid", 192), ("k3_width", 48)])
+                                         ("mid", 192), ("k3_width", 48), ("k3_decode", None)])
 def test_forward_parity_full_size(name, sample):
     """The benchmark's workloads at full size.  Where the oracle cannot run every
     token in seconds, a fixed sample of tokens is compared (the margin is enforced
