@@ -79,8 +79,9 @@ def _load():
         _lib.orc_rmsnorm_rows.argtypes = [ctypes.c_int64, ctypes.c_int32, _P, _P,
                                           ctypes.c_double, _P]
         _lib.orc_router_losses.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, _P]
+        _lib.orc_backward.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Weights), _P, _P] + [_P] * 11
         for f in ("orc_situ", "orc_route", "orc_permute", "orc_forward", "orc_forward_dense",
-                  "orc_rmsnorm_rows", "orc_router_losses"):
+                  "orc_rmsnorm_rows", "orc_router_losses", "orc_backward"):
             getattr(_lib, f).restype = None
     return _lib
 
@@ -170,6 +171,32 @@ def router_losses(dims: Dims, x, w_router, ids):
     _load().orc_router_losses(ctypes.byref(c), _ptr(x), _ptr(w_router), _ptr(ids), _ptr(out))
     return {"aux": float(out[0]), "z": float(out[1]), "frac": out[2:2 + R].copy(),
             "prob_mean": out[2 + R:].copy()}
+
+
+GRAD_NAMES = ("x", "w_down", "w_router", "w_up", "rms_weight", "w_g", "w_u", "w_o",
+              "ws_g", "ws_u", "ws_o")
+
+
+def backward(dims: Dims, weights: dict, x, dy):
+    """Gradients of <dy, y> (y the layer's output) with respect to x and every
+    weight except expert_bias (which only selects): {name: float64 array}."""
+    cw, keep = _weights(weights)
+    x = _f32(x)
+    dy = _f32(dy)
+    N, d, L, R, F, S, G = (dims.n_tokens, dims.d, dims.latent, dims.n_routed, dims.ff_routed,
+                           dims.n_shared, dims.ff_shared)
+    assert x.shape == (N, d) and dy.shape == (N, d)
+    shapes = {"x": (N, d), "w_down": (L, d), "w_router": (R, d), "w_up": (d, L),
+              "rms_weight": (L,), "w_g": (R, F, L), "w_u": (R, F, L), "w_o": (R, L, F),
+              "ws_g": (max(S, 1), G, d), "ws_u": (max(S, 1), G, d), "ws_o": (max(S, 1), d, G)}
+    out = {n: np.zeros(shapes[n], np.float64) for n in GRAD_NAMES}
+    c = dims._c()
+    _load().orc_backward(ctypes.byref(c), ctypes.byref(cw), _ptr(x), _ptr(dy),
+                         *[_ptr(out[n]) for n in GRAD_NAMES])
+    if S == 0:
+        for n in ("ws_g", "ws_u", "ws_o"):
+            out[n] = out[n][:0]
+    return out
 
 
 def permute(ids, n_routed: int):

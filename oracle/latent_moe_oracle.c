@@ -398,3 +398,214 @@ void orc_router_losses(const orc_dims* dm, const float* x, const float* w_r, con
   free(l);
   free(xv);
 }
+
+/* ------------------------------------------------------------------ backward
+ * Gradients of the layer for an upstream gradient dy [N, d] (the pages' tests
+ * train the layer: test_moe_unselected_experts_have_zero_grad and the sparse
+ * == dense gradient checks of [tests]), by the chain rule through the five
+ * steps of the forward, token by token, in double:
+ *   y = s_sh + W_up uhat          dW_up += dy uhat^T,  duhat = W_up^T dy
+ *   uhat = u r w, r = (mean u^2 + eps)^(-1/2)
+ *                                 dw += duhat u r,  du = r w duhat - u r^3/l sum_j w_j duhat_j u_j
+ *   u = sum_i p_i E_i(z)          dp_i = <du, E_i(z)>,  dE_i = p_i du
+ *   E(v) = W_o h, h = g(a) up(c), a = W_g v, c = W_u v
+ *     g(a) = b1 tanh(a/b1) sigmoid(a),   g'(a) = sech^2(a/b1) sigmoid(a) + g(a) (1 - sigmoid(a))
+ *     up(c) = b2 tanh(c/b2),             up'(c) = sech^2(c/b2)
+ *                                 dW_o += dE h^T, dh = W_o^T dE, da = dh up g', dc = dh g up',
+ *                                 dW_g += da v^T, dW_u += dc v^T, dv += W_g^T da + W_u^T dc
+ *   routing (ids fixed: they are not differentiable; b enters no gradient):
+ *     K3: p_i = s_i / S, S = sum_T s (clamped at 1e-9), s = sigmoid(l):
+ *         ds_i = (dp_i - sum_j p_j dp_j) / S   (dp_i / 1e-9 when clamped),
+ *         dl_i = ds_i s_i (1 - s_i)
+ *     softmax over the top-k logits: dl_i = p_i (dp_i - sum_j p_j dp_j)
+ *                                 dW_r[e_i] += dl_i x,  dx += dl_i W_r[e_i]
+ *   z = W_down x                  dW_down += dz x^T,  dx += W_down^T dz
+ *   s_sh = sum_j E^sh_j(x)        E^sh backward with dE = dy and v = x
+ * Every output is overwritten.  Weight gradients of experts no token selected
+ * stay exactly 0. */
+static void orc_situ_backward(int32_t dim_in, int32_t ff, double beta1, double beta2,
+                              const float* w_g, const float* w_u, const float* w_o,
+                              const double* v, const double* dout, double* dv, double* dw_g,
+                              double* dw_u, double* dw_o, double* out) {
+  double* a = (double*)malloc(sizeof(double) * (size_t)ff);
+  double* c = (double*)malloc(sizeof(double) * (size_t)ff);
+  double* h = (double*)malloc(sizeof(double) * (size_t)ff);
+  double* dh = (double*)calloc((size_t)ff, sizeof(double));
+  orc_linear(w_g, ff, dim_in, v, a);
+  orc_linear(w_u, ff, dim_in, v, c);
+  for (int32_t f = 0; f < ff; ++f) {
+    const double tg = tanh(a[f] / beta1), sg = orc_sigmoid(a[f]), tu = tanh(c[f] / beta2);
+    h[f] = beta1 * tg * sg * beta2 * tu;
+  }
+  if (out) orc_linear(w_o, dim_in, ff, h, out);
+  for (int32_t i = 0; i < dim_in; ++i) {
+    const float* row = w_o + (int64_t)i * ff;
+    for (int32_t f = 0; f < ff; ++f) {
+      dh[f] += (double)row[f] * dout[i];
+      dw_o[(int64_t)i * ff + f] += dout[i] * h[f];
+    }
+  }
+  for (int32_t f = 0; f < ff; ++f) {
+    const double tg = tanh(a[f] / beta1), sg = orc_sigmoid(a[f]), tu = tanh(c[f] / beta2);
+    const double g = beta1 * tg * sg, up = beta2 * tu;
+    const double dg = (1.0 - tg * tg) * sg + g * (1.0 - sg);
+    const double du = 1.0 - tu * tu;
+    const double da = dh[f] * up * dg, dc = dh[f] * g * du;
+    const float* rg = w_g + (int64_t)f * dim_in;
+    const float* ru = w_u + (int64_t)f * dim_in;
+    double* gg = dw_g + (int64_t)f * dim_in;
+    double* gu = dw_u + (int64_t)f * dim_in;
+    for (int32_t j = 0; j < dim_in; ++j) {
+      gg[j] += da * v[j];
+      gu[j] += dc * v[j];
+      dv[j] += (double)rg[j] * da + (double)ru[j] * dc;
+    }
+  }
+  free(a);
+  free(c);
+  free(h);
+  free(dh);
+}
+
+void orc_backward(const orc_dims* dm, const orc_weights* w, const float* x, const float* dy,
+                  double* dx, double* dw_down, double* dw_router, double* dw_up, double* drms,
+                  double* dw_g, double* dw_u, double* dw_o, double* dws_g, double* dws_u,
+                  double* dws_o) {
+  const int64_t N = dm->n_tokens;
+  const int32_t d = dm->d, L = dm->latent, R = dm->n_routed, k = dm->top_k;
+  const int32_t F = dm->ff_routed, S = dm->n_shared, G = dm->ff_shared;
+  memset(dx, 0, sizeof(double) * (size_t)(N * d));
+  memset(dw_down, 0, sizeof(double) * (size_t)L * d);
+  memset(dw_router, 0, sizeof(double) * (size_t)R * d);
+  memset(dw_up, 0, sizeof(double) * (size_t)d * L);
+  memset(drms, 0, sizeof(double) * (size_t)L);
+  memset(dw_g, 0, sizeof(double) * (size_t)R * F * L);
+  memset(dw_u, 0, sizeof(double) * (size_t)R * F * L);
+  memset(dw_o, 0, sizeof(double) * (size_t)R * L * F);
+  if (S > 0) {
+    memset(dws_g, 0, sizeof(double) * (size_t)S * G * d);
+    memset(dws_u, 0, sizeof(double) * (size_t)S * G * d);
+    memset(dws_o, 0, sizeof(double) * (size_t)S * d * G);
+  }
+  double* xv = (double*)malloc(sizeof(double) * (size_t)d);
+  double* dyv = (double*)malloc(sizeof(double) * (size_t)d);
+  double* z = (double*)malloc(sizeof(double) * (size_t)L);
+  double* dz = (double*)malloc(sizeof(double) * (size_t)L);
+  double* eo = (double*)malloc(sizeof(double) * (size_t)k * L);
+  double* u = (double*)malloc(sizeof(double) * (size_t)L);
+  double* uhat = (double*)malloc(sizeof(double) * (size_t)L);
+  double* duhat = (double*)malloc(sizeof(double) * (size_t)L);
+  double* du = (double*)malloc(sizeof(double) * (size_t)L);
+  double* dE = (double*)malloc(sizeof(double) * (size_t)L);
+  double* l = (double*)malloc(sizeof(double) * (size_t)R);
+  double* dp = (double*)malloc(sizeof(double) * (size_t)k);
+  double* probs = (double*)malloc(sizeof(double) * (size_t)k);
+  int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+  for (int64_t t = 0; t < N; ++t) {
+    const float* x_t = x + t * d;
+    double* dx_t = dx + t * d;
+    for (int32_t i = 0; i < d; ++i) {
+      xv[i] = (double)x_t[i];
+      dyv[i] = (double)dy[t * d + i];
+    }
+    /* forward of this token */
+    orc_linear(w->w_down, L, d, xv, z);
+    orc_linear(w->w_router, R, d, xv, l);
+    orc_route_token(d, R, k, dm->router, x_t, w->w_router, w->expert_bias, ids, probs, NULL,
+                    NULL);
+    for (int32_t j = 0; j < L; ++j) u[j] = 0.0;
+    for (int32_t slot = 0; slot < k; ++slot) {
+      const int64_t e = ids[slot];
+      orc_situ(L, F, dm->beta1, dm->beta2, w->w_g + e * F * L, w->w_u + e * F * L,
+               w->w_o + e * L * F, z, eo + (int64_t)slot * L, NULL);
+      for (int32_t j = 0; j < L; ++j) u[j] += probs[slot] * eo[(int64_t)slot * L + j];
+    }
+    double ms = 0.0;
+    for (int32_t j = 0; j < L; ++j) ms += u[j] * u[j];
+    const double r = 1.0 / sqrt(ms / (double)L + dm->rms_eps);
+    for (int32_t j = 0; j < L; ++j) uhat[j] = u[j] * r * (double)w->rms_weight[j];
+    /* step 5: y = s_sh + W_up uhat */
+    for (int32_t j = 0; j < L; ++j) duhat[j] = 0.0;
+    for (int32_t i = 0; i < d; ++i) {
+      const float* row = w->w_up + (int64_t)i * L;
+      for (int32_t j = 0; j < L; ++j) {
+        dw_up[(int64_t)i * L + j] += dyv[i] * uhat[j];
+        duhat[j] += (double)row[j] * dyv[i];
+      }
+    }
+    /* RMSNorm */
+    double wdu = 0.0;
+    for (int32_t j = 0; j < L; ++j) {
+      drms[j] += duhat[j] * u[j] * r;
+      wdu += (double)w->rms_weight[j] * duhat[j] * u[j];
+    }
+    for (int32_t j = 0; j < L; ++j)
+      du[j] = r * (double)w->rms_weight[j] * duhat[j] - u[j] * r * r * r / (double)L * wdu;
+    /* routed experts and their weights p */
+    for (int32_t j = 0; j < L; ++j) dz[j] = 0.0;
+    for (int32_t slot = 0; slot < k; ++slot) {
+      const int64_t e = ids[slot];
+      double acc = 0.0;
+      for (int32_t j = 0; j < L; ++j) {
+        acc += du[j] * eo[(int64_t)slot * L + j];
+        dE[j] = probs[slot] * du[j];
+      }
+      dp[slot] = acc;
+      orc_situ_backward(L, F, dm->beta1, dm->beta2, w->w_g + e * F * L, w->w_u + e * F * L,
+                        w->w_o + e * L * F, z, dE, dz, dw_g + e * F * L, dw_u + e * F * L,
+                        dw_o + e * L * F, NULL);
+    }
+    /* router, through p only */
+    double pdp = 0.0, ssum = 0.0;
+    for (int32_t slot = 0; slot < k; ++slot) {
+      pdp += probs[slot] * dp[slot];
+      ssum += orc_sigmoid(l[ids[slot]]);
+    }
+    for (int32_t slot = 0; slot < k; ++slot) {
+      const int32_t e = ids[slot];
+      double dl;
+      if (dm->router == 1) {
+        dl = probs[slot] * (dp[slot] - pdp);
+      } else {
+        const double s = orc_sigmoid(l[e]);
+        const double ds = ssum >= 1e-9 ? (dp[slot] - pdp) / ssum : dp[slot] / 1e-9;
+        dl = ds * s * (1.0 - s);
+      }
+      const float* row = w->w_router + (int64_t)e * d;
+      double* grow = dw_router + (int64_t)e * d;
+      for (int32_t i = 0; i < d; ++i) {
+        grow[i] += dl * xv[i];
+        dx_t[i] += dl * (double)row[i];
+      }
+    }
+    /* step 1: z = W_down x */
+    for (int32_t j = 0; j < L; ++j) {
+      const float* row = w->w_down + (int64_t)j * d;
+      double* grow = dw_down + (int64_t)j * d;
+      for (int32_t i = 0; i < d; ++i) {
+        grow[i] += dz[j] * xv[i];
+        dx_t[i] += (double)row[i] * dz[j];
+      }
+    }
+    /* step 4: shared experts, dE = dy */
+    for (int32_t j = 0; j < S; ++j)
+      orc_situ_backward(d, G, dm->beta1, dm->beta2, w->ws_g + (int64_t)j * G * d,
+                        w->ws_u + (int64_t)j * G * d, w->ws_o + (int64_t)j * d * G, xv, dyv,
+                        dx_t, dws_g + (int64_t)j * G * d, dws_u + (int64_t)j * G * d,
+                        dws_o + (int64_t)j * d * G, NULL);
+  }
+  free(xv);
+  free(dyv);
+  free(z);
+  free(dz);
+  free(eo);
+  free(u);
+  free(uhat);
+  free(duhat);
+  free(du);
+  free(dE);
+  free(l);
+  free(dp);
+  free(probs);
+  free(ids);
+}

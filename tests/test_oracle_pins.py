@@ -526,3 +526,117 @@ def test_router_losses_frac_is_the_routing_histogram_and_token_order_free():
     assert out2["z"] == pytest.approx(out["z"], rel=1e-13)
     assert out["aux"] <= 12 * out["prob_mean"].max() + 1e-12
     assert ((out["prob_mean"] > 0) & (out["prob_mean"] < 1)).all()
+
+
+# ------------------------------------------------------------------ backward
+
+def _grid(rng, shape, scale, step=2.0 ** -8):
+    """Values on a coarse binary grid, so that +-2^-17 perturbations are exact in float32."""
+    return (np.round(rng.standard_normal(shape) * scale / step) * step).astype(np.float32)
+
+
+def _fd_case(router=0, S=1, clamp=False, seed=0):
+    dims = oracle.Dims(5, 16, 8, 6, 2, S, 12, 10, router=router)
+    rng = np.random.default_rng(seed)
+    d, L, R, F, G = dims.d, dims.latent, dims.n_routed, dims.ff_routed, dims.ff_shared
+    Sx = max(S, 1)
+    w = dict(w_down=_grid(rng, (L, d), 0.3), w_router=_grid(rng, (R, d), 0.5),
+             w_up=_grid(rng, (d, L), 0.3), rms_weight=(1.0 + _grid(rng, (L,), 0.2)),
+             expert_bias=_grid(rng, (R,), 0.1), w_g=_grid(rng, (R, F, L), 0.4),
+             w_u=_grid(rng, (R, F, L), 0.4), w_o=_grid(rng, (R, L, F), 0.3),
+             ws_g=_grid(rng, (Sx, G, d), 0.3), ws_u=_grid(rng, (Sx, G, d), 0.3),
+             ws_o=_grid(rng, (Sx, d, G), 0.3))
+    x = _grid(rng, (dims.n_tokens, d), 1.0)
+    if clamp:   # every logit near -30: the selected scores sum below 1e-9
+        x[:, -1] = 1.0
+        w["w_router"][:, -1] = -30.0
+    dy = _grid(rng, (dims.n_tokens, d), 1.0)
+    return dims, w, x, dy
+
+
+def _loss(dims, w, x, dy):
+    y = oracle.forward(dims, w, x)["y"]
+    return float((dy.astype(np.float64) * y).sum())
+
+
+@pytest.mark.parametrize("router,S,clamp", [(0, 1, False), (1, 2, False), (0, 0, False),
+                                            (0, 1, True)])
+def test_backward_matches_central_differences(router, S, clamp):
+    """Every gradient of <dy, y> against central differences of the forward
+    (h = 2^-17, exact in float32 on the inputs' grid, truncation error ~h^2;
+    routing unchanged by the perturbations).  Covers x, and sampled entries of every weight; the
+    K3 router (plain and with its 1e-9 clamp active) and the softmax router."""
+    dims, w, x, dy = _fd_case(router, S, clamp, seed=router * 10 + S + 3 * clamp)
+    ids0 = oracle.route(dims, x, w["w_router"], w["expert_bias"])[0]
+    g = oracle.backward(dims, w, x, dy)
+    h = 2.0 ** -17
+    rng = np.random.default_rng(42)
+
+    def fd(perturb):
+        plus, minus = perturb(h), perturb(-h)
+        return (_loss(dims, *plus, dy) - _loss(dims, *minus, dy)) / (2 * h)
+
+    checked = 0
+    # x: every entry
+    for t in range(dims.n_tokens):
+        for i in range(dims.d):
+            def px(eps, t=t, i=i):
+                xx = x.copy()
+                xx[t, i] += np.float32(eps)
+                assert (oracle.route(dims, xx, w["w_router"], w["expert_bias"])[0] == ids0).all()
+                return w, xx
+            got, want = g["x"][t, i], fd(px)
+            assert got == pytest.approx(want, rel=1e-6, abs=1e-8), ("x", t, i)
+            checked += 1
+    names = ["w_down", "w_router", "w_up", "rms_weight", "w_g", "w_u", "w_o"]
+    if S:
+        names += ["ws_g", "ws_u", "ws_o"]
+    for name in names:
+        arr = w[name]
+        picks = [tuple(rng.integers(0, n) for n in arr.shape) for _ in range(6)]
+        if name in ("w_g", "w_u", "w_o"):   # entries of a selected expert too
+            e = int(ids0[0, 0])
+            picks += [(e,) + tuple(rng.integers(0, n) for n in arr.shape[1:]) for _ in range(4)]
+        for idx in picks:
+            def pw(eps, name=name, idx=idx):
+                ww = dict(w)
+                ww[name] = w[name].copy()
+                ww[name][idx] += np.float32(eps)
+                return ww, x
+            got, want = g[name][idx], fd(pw)
+            assert got == pytest.approx(want, rel=1e-6, abs=1e-8), (name, idx)
+            checked += 1
+    assert checked > dims.n_tokens * dims.d
+
+
+def test_backward_unselected_experts_get_exactly_zero():
+    """The pages' test_moe_unselected_experts_have_zero_grad: experts no token
+    selects get gradients that are exactly 0; a selected one gets nonzero ones."""
+    dims, w, x, dy = _fd_case(seed=7)
+    ids = oracle.route(dims, x, w["w_router"], w["expert_bias"])[0]
+    g = oracle.backward(dims, w, x, dy)
+    used = set(ids.reshape(-1).tolist())
+    for e in range(dims.n_routed):
+        for name in ("w_g", "w_u", "w_o"):
+            if e in used:
+                assert np.abs(g[name][e]).sum() > 0
+            else:
+                assert (g[name][e] == 0).all()
+        if e not in used:
+            assert (g["w_router"][e] == 0).all()   # through p only: unselected rows get none
+
+
+def test_backward_with_zero_up_projection():
+    """W_up = 0 cuts the routed path: every routed, router, RMSNorm and W_down
+    gradient is 0, dW_up = dy^T RMSNorm(u), and dx is the shared experts' alone."""
+    dims, w, x, dy = _fd_case(seed=9)
+    w["w_up"] = np.zeros_like(w["w_up"])
+    g = oracle.backward(dims, w, x, dy)
+    for name in ("w_g", "w_u", "w_o", "w_router", "w_down", "rms_weight"):
+        assert (g[name] == 0).all(), name
+    uhat = oracle.forward(dims, w, x, want=("uhat",))["uhat"]
+    np.testing.assert_allclose(g["w_up"], dy.astype(np.float64).T @ uhat, rtol=1e-12, atol=1e-14)
+    w2 = dict(w)
+    w2["w_g"] = np.zeros_like(w["w_g"])
+    w2["w_down"] = np.zeros_like(w["w_down"])
+    np.testing.assert_allclose(oracle.backward(dims, w2, x, dy)["x"], g["x"], rtol=1e-13, atol=1e-15)
