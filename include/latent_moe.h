@@ -187,6 +187,37 @@ LMOE_API lmoe_status latent_moe_forward(const lmoe_dims* dims, const lmoe_weight
                                void* y, int32_t* ids_out, float* probs_out, int32_t* counts_out,
                                void* ws, size_t ws_bytes, lmoe_stream stream);
 
+/* Gradients of the layer (fp32 device buffers, caller-owned, every one
+ * fully overwritten; shapes as the weights). */
+typedef struct {
+  float* dx;          /* [N, d]                                          */
+  float* dw_down;     /* [l, d]                                          */
+  float* dw_router;   /* [R, d]                                          */
+  float* dw_up;       /* [d, l]                                          */
+  float* drms_weight; /* [l]                                             */
+  float* dw_g;        /* [R, F, l]                                       */
+  float* dw_u;        /* [R, F, l]                                       */
+  float* dw_o;        /* [R, l, F]                                       */
+  float* dws_g;       /* [S, G, d]   (unused when S = 0)                 */
+  float* dws_u;       /* [S, G, d]                                       */
+  float* dws_o;       /* [S, d, G]                                       */
+} lmoe_grads;
+
+/* Backward of the layer: the gradients of <dy, y> with respect to x and every
+ * weight, y = latent_moe_forward(x) (the pages train the layer; its tests check
+ * the gradients: unselected experts get exactly 0).  The routing ids are not
+ * differentiable and expert_bias only selects, so it gets no gradient; W_r gets
+ * its gradient through the routing weights p only.  The forward's internals
+ * are recomputed in fp32 from x (routing with the same kernels as the forward),
+ * so no forward state is needed; every sum runs in a fixed order
+ * (deterministic).  dy [N, d] in the activation dtype.  Workspace:
+ * lmoe_backward_workspace_size(dims) bytes, 256-byte aligned (its own layout,
+ * not the forward's). */
+LMOE_API size_t lmoe_backward_workspace_size(const lmoe_dims* dims);
+LMOE_API lmoe_status latent_moe_backward(const lmoe_dims* dims, const lmoe_weights* weights,
+                                         const void* x, const void* dy, const lmoe_grads* grads,
+                                         void* ws, size_t ws_bytes, lmoe_stream stream);
+
 /* The whole layer from HOST memory: copies x_host [N, d] (pinned or pageable)
  * to the device, runs latent_moe_forward, copies y back to y_host [N, d] and
  * waits for the stream.  Weights and workspace are device memory.  The

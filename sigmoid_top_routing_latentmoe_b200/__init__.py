@@ -54,6 +54,15 @@ class Weights(ctypes.Structure):
     _fields_ = [(n, _P) for n in WEIGHT_NAMES]
 
 
+GRAD_NAMES = ("dx", "dw_down", "dw_router", "dw_up", "drms_weight", "dw_g", "dw_u", "dw_o",
+              "dws_g", "dws_u", "dws_o")
+
+
+class Grads(ctypes.Structure):
+    """lmoe_grads."""
+    _fields_ = [(n, _P) for n in GRAD_NAMES]
+
+
 _S = ctypes.c_int
 _DP = ctypes.POINTER(Dims)
 _sigs = {
@@ -65,6 +74,9 @@ _sigs = {
     "moe_expert_ffn": (_S, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_combine": (_S, [_DP, _P, _P, _P, _P, _P, _P]),
     "moe_router_losses": (_S, [_DP, _P, ctypes.c_int64, _P, _P, _P, ctypes.c_size_t, _P]),
+    "lmoe_backward_workspace_size": (ctypes.c_size_t, [_DP]),
+    "latent_moe_backward": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, ctypes.POINTER(Grads), _P,
+                                 ctypes.c_size_t, _P]),
     "latent_moe_forward": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, _P, _P, _P, _P,
                                 ctypes.c_size_t, _P]),
     "latent_moe_forward_host": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, _P, ctypes.c_size_t,
@@ -207,6 +219,38 @@ def latent_moe_forward(dims, weights, x, y, ws, ids_out=None, probs_out=None, co
     _check(_lib.latent_moe_forward(ctypes.byref(dims), ctypes.byref(ws_struct), _ptr(x), _ptr(y),
                                    _ptr(ids_out), _ptr(probs_out), _ptr(counts_out), _ptr(ws),
                                    ws.numel(), _stream(stream)), "latent_moe_forward")
+
+
+def alloc_backward_workspace(dims: Dims, device="cuda") -> torch.Tensor:
+    """A 256-byte aligned byte tensor of lmoe_backward_workspace_size(dims)."""
+    n = _lib.lmoe_backward_workspace_size(ctypes.byref(dims))
+    if n == 0:
+        raise LmoeError("lmoe_backward_workspace_size: " + _lib.lmoe_last_error().decode())
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    return ws[off:off + n]
+
+
+def latent_moe_backward(dims, weights, x, dy, grads: dict, ws, stream=None):
+    """grads: {name in GRAD_NAMES: fp32 tensor} (dws_* may be absent when S = 0)."""
+    act = torch.bfloat16 if dims.dtype == BF16 else torch.float32
+    for name, t in (("x", x), ("dy", dy)):
+        if t.dtype != act or t.numel() != dims.n_tokens * dims.d or not t.is_contiguous():
+            raise LmoeError(f"{name}: expected a contiguous {act} tensor of {dims.n_tokens}x{dims.d}")
+    N, d, L, R, F, S, G = (dims.n_tokens, dims.d, dims.latent, dims.n_routed, dims.ff_routed,
+                           dims.n_shared, dims.ff_shared)
+    sizes = {"dx": N * d, "dw_down": L * d, "dw_router": R * d, "dw_up": d * L,
+             "drms_weight": L, "dw_g": R * F * L, "dw_u": R * F * L, "dw_o": R * L * F,
+             "dws_g": S * G * d, "dws_u": S * G * d, "dws_o": S * d * G}
+    for name, n in sizes.items():
+        t = grads.get(name)
+        if n and (t is None or t.dtype != torch.float32 or t.numel() != n or not t.is_contiguous()):
+            raise LmoeError(f"grads[{name}]: expected a contiguous float32 tensor of {n} elements")
+    ws_struct = weights if isinstance(weights, Weights) else weights_struct(weights)
+    g = Grads(*[_ptr(grads.get(n)) for n in GRAD_NAMES])
+    _check(_lib.latent_moe_backward(ctypes.byref(dims), ctypes.byref(ws_struct), _ptr(x), _ptr(dy),
+                                    ctypes.byref(g), _ptr(ws), ws.numel(), _stream(stream)),
+           "latent_moe_backward")
 
 
 def latent_moe_forward_host(dims, weights, x_host, y_host, ws, stream=None):

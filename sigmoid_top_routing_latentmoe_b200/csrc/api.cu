@@ -529,6 +529,90 @@ lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const int32_t* 
   return run_expert_ffn<float>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
 }
 
+static BwdDims bwd_dims(const lmoe_dims* d) {
+  BwdDims b;
+  b.N = d->n_tokens; b.d = d->d; b.L = d->latent; b.R = d->n_routed; b.k = d->top_k;
+  b.S = d->n_shared; b.F = d->ff_routed; b.G = d->n_shared > 0 ? d->ff_shared : 0;
+  b.beta1 = d->beta1; b.beta2 = d->beta2; b.rms_eps = d->rms_eps; b.router = d->router;
+  b.bf16 = d->dtype == LMOE_BF16 ? 1 : 0;
+  return b;
+}
+
+size_t lmoe_backward_workspace_size(const lmoe_dims* dims) {
+  if (check_dims(dims) != LMOE_OK) return 0;
+  return bwd_layout(bwd_dims(dims)).total;
+}
+
+lmoe_status latent_moe_backward(const lmoe_dims* dims, const lmoe_weights* w, const void* x,
+                                const void* dy, const lmoe_grads* g, void* ws, size_t ws_bytes,
+                                lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  if (w == nullptr || g == nullptr) return fail(LMOE_EINVAL, "weights or grads is NULL");
+  LMOE_PTR(w->w_down, "w_down");
+  LMOE_PTR(w->w_router, "w_router");
+  LMOE_PTR(w->w_up, "w_up");
+  LMOE_PTR(w->rms_weight, "rms_weight");
+  LMOE_PTR(w->w_g, "w_g");
+  LMOE_PTR(w->w_u, "w_u");
+  LMOE_PTR(w->w_o, "w_o");
+  LMOE_PTR(g->dw_down, "dw_down");
+  LMOE_PTR(g->dw_router, "dw_router");
+  LMOE_PTR(g->dw_up, "dw_up");
+  LMOE_PTR(g->drms_weight, "drms_weight");
+  LMOE_PTR(g->dw_g, "dw_g");
+  LMOE_PTR(g->dw_u, "dw_u");
+  LMOE_PTR(g->dw_o, "dw_o");
+  if (dims->n_shared > 0) {
+    LMOE_PTR(w->ws_g, "ws_g");
+    LMOE_PTR(w->ws_u, "ws_u");
+    LMOE_PTR(w->ws_o, "ws_o");
+    LMOE_PTR(g->dws_g, "dws_g");
+    LMOE_PTR(g->dws_u, "dws_u");
+    LMOE_PTR(g->dws_o, "dws_o");
+  }
+  if (dims->n_tokens > 0) {
+    LMOE_PTR(x, "x");
+    LMOE_PTR(dy, "dy");
+    LMOE_PTR(g->dx, "dx");
+  }
+  LMOE_PTR(ws, "ws");
+  if (((uintptr_t)ws & 255u) != 0) return fail(LMOE_EINVAL, "ws must be 256-byte aligned");
+  const BwdDims bd = bwd_dims(dims);
+  const size_t need = bwd_layout(bd).total;
+  if (ws_bytes < need)
+    return fail(LMOE_EWORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+  LMOE_TRY(check_device());
+  cudaStream_t st = (cudaStream_t)stream;
+  LMOE_CUDA(cudaMemsetAsync(ws, 0, 256, st), "clear the header");
+  if (dims->n_tokens == 0) {  // no tokens: every gradient is 0
+    const size_t L = dims->latent, d = dims->d, R = dims->n_routed, F = dims->ff_routed;
+    LMOE_CUDA(cudaMemsetAsync(g->dw_down, 0, L * d * 4, st), "memset");
+    LMOE_CUDA(cudaMemsetAsync(g->dw_router, 0, R * d * 4, st), "memset");
+    LMOE_CUDA(cudaMemsetAsync(g->dw_up, 0, d * L * 4, st), "memset");
+    LMOE_CUDA(cudaMemsetAsync(g->drms_weight, 0, L * 4, st), "memset");
+    LMOE_CUDA(cudaMemsetAsync(g->dw_g, 0, R * F * L * 4, st), "memset");
+    LMOE_CUDA(cudaMemsetAsync(g->dw_u, 0, R * F * L * 4, st), "memset");
+    LMOE_CUDA(cudaMemsetAsync(g->dw_o, 0, R * L * F * 4, st), "memset");
+    if (dims->n_shared > 0) {
+      const size_t SG = (size_t)dims->n_shared * dims->ff_shared;
+      LMOE_CUDA(cudaMemsetAsync(g->dws_g, 0, SG * d * 4, st), "memset");
+      LMOE_CUDA(cudaMemsetAsync(g->dws_u, 0, SG * d * 4, st), "memset");
+      LMOE_CUDA(cudaMemsetAsync(g->dws_o, 0, SG * d * 4, st), "memset");
+    }
+    return LMOE_OK;
+  }
+  BwdArgs a;
+  a.x = x; a.dy = dy; a.w_down = w->w_down; a.w_router = w->w_router; a.w_up = w->w_up;
+  a.w_g = w->w_g; a.w_u = w->w_u; a.w_o = w->w_o; a.ws_g = w->ws_g; a.ws_u = w->ws_u;
+  a.ws_o = w->ws_o; a.rms_weight = w->rms_weight; a.bias = w->expert_bias;
+  a.g.dx = g->dx; a.g.dw_down = g->dw_down; a.g.dw_router = g->dw_router; a.g.dw_up = g->dw_up;
+  a.g.drms = g->drms_weight; a.g.dw_g = g->dw_g; a.g.dw_u = g->dw_u; a.g.dw_o = g->dw_o;
+  a.g.dws_g = g->dws_g; a.g.dws_u = g->dws_u; a.g.dws_o = g->dws_o;
+  ProfScope ps("backward", st);
+  LMOE_CUDA(run_backward(bd, a, ws, st), "backward");
+  return LMOE_OK;
+}
+
 lmoe_status moe_router_losses(const lmoe_dims* dims, const float* logits, int64_t ld,
                               const int32_t* ids, float* out, void* ws, size_t ws_bytes,
                               lmoe_stream stream) {

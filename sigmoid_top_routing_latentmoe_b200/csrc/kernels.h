@@ -90,4 +90,29 @@ void count_launch(int n = 1);
 // Sets the per-thread message returned by lmoe_last_error (api.cu).
 void set_last_error(const char* msg);
 
+// ------------------------------------------------------------------ backward
+struct BwdDims {
+  int64_t N;
+  int d, L, R, k, S, F, G;
+  float beta1, beta2, rms_eps;
+  int router;
+  int bf16;  // x, dy and the weights are bf16 (else fp32); gradients are fp32
+};
+struct BwdGrads {
+  float *dx, *dw_down, *dw_router, *dw_up, *drms, *dw_g, *dw_u, *dw_o, *dws_g, *dws_u, *dws_o;
+};
+struct BwdArgs {
+  const void *x, *dy, *w_down, *w_router, *w_up, *w_g, *w_u, *w_o, *ws_g, *ws_u, *ws_o;
+  const float *rms_weight, *bias;
+  BwdGrads g;
+};
+struct BwdLayout {
+  size_t header, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, z, a, c, h,
+      dh, o, dE, u, uhat, duhat, du, rr, dp, dl, rms_part, ash, csh, hsh, dhsh, total;
+  int ld_logits, max_tiles;
+};
+BwdLayout bwd_layout(const BwdDims& d);
+// The workspace header (its first 256 bytes) must be zero on entry.
+cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStream_t st);
+
 }  // namespace lmoe
