@@ -289,6 +289,90 @@ def run_memory_kernels(args, wl):
         raise SystemExit("device status not OK")
 
 
+# fp32 FFMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (max SM clock)
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_backward_bench(args, wl):
+    """latent_moe_backward timed like the forward (CUDA graph replay, L2 flushed
+    between steps); one JSON line.  Algorithmic work: the gradient contractions,
+    2x the forward's FLOPs (the backward also recomputes the forward, 1x more),
+    on the CUDA cores in fp32."""
+    import torch
+    import sigmoid_top_routing_latentmoe_b200 as lm
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    inp = synth.make_inputs(wl, args.seed)
+
+    def todev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    w = {k: todev(inp[k]) for k in synth.WEIGHT_NAMES}
+    x = todev(inp["x"])
+    dy = todev(synth.normal(args.seed + 1, "dy", (wl.n_tokens, wl.d), 1.0,
+                            dtype="bf16" if wl.dtype == "bf16" else "f32"))
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    dims = lm.make_dims(wl.n_tokens, wl.d, wl.latent, wl.n_routed, wl.top_k, wl.n_shared,
+                        wl.ff_routed, wl.ff_shared, wl.beta1, wl.beta2, wl.rms_eps, dt)
+    ws = lm.alloc_backward_workspace(dims, device=dev)
+    N, d, L, R, F, S, G = (wl.n_tokens, wl.d, wl.latent, wl.n_routed, wl.ff_routed, wl.n_shared,
+                           wl.ff_shared)
+    shapes = {"dx": (N, d), "dw_down": (L, d), "dw_router": (R, d), "dw_up": (d, L),
+              "drms_weight": (L,), "dw_g": (R, F, L), "dw_u": (R, F, L), "dw_o": (R, L, F)}
+    if S:
+        shapes.update(dws_g=(S, G, d), dws_u=(S, G, d), dws_o=(S, d, G))
+    grads = {n: torch.empty(sh, dtype=torch.float32, device=dev) for n, sh in shapes.items()}
+    wstruct = lm.weights_struct(w)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        lm.latent_moe_backward(dims, wstruct, x, dy, grads, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if lm.get_device_status(ws) != lm.OK:
+        raise SystemExit("device status not OK after warm-up")
+    lm.launch_count(reset=True)
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.graph(graph, stream=cap):
+        step()
+    launches = lm.launch_count(reset=True)
+    graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    stream = torch.cuda.current_stream(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        graph.replay()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    work = 2.0 * wl.flops()
+    achieved = work / (ms / 1e3) / 1e12
+    print(json.dumps({
+        "metric": "LatentMoE layer bwd tokens/s on 1 B200 (gradients of x and every weight)",
+        "value": wl.n_tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (from %s inputs)" % wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "n_tokens": wl.n_tokens, "launch": "cuda graph replay",
+                   "l2": "flushed (256 MiB write) between steps"},
+        "roofline": {"kernel": "whole backward", "bound": "alu", "achieved": achieved,
+                     "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
+                     "frac": achieved / FP32_SIMT_TFLOPS, "traffic": None,
+                     "work": "2x forward FLOPs (the recomputed forward is not counted)"},
+        "clocks": clk, "gpu_launches": launches * args.steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -304,10 +388,14 @@ def main():
                     help="launch the kernels every step instead of replaying a CUDA graph")
     ap.add_argument("--memory-kernels", action="store_true",
                     help="time moe_route / moe_dispatch / moe_combine on their own instead")
+    ap.add_argument("--backward", action="store_true",
+                    help="time latent_moe_backward instead of the forward")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     if args.memory_kernels:
         return run_memory_kernels(args, wl)
+    if args.backward:
+        return run_backward_bench(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     if args.warmup < 3:
