@@ -34,9 +34,9 @@
 namespace lmoe {
 namespace {
 
-constexpr int GB = 64;   // output tile (rows and columns)
+constexpr int GB = 128;  // output tile (rows and columns)
 constexpr int GK = 16;   // K per smem stage
-constexpr int GT = 256;  // threads
+constexpr int GT = 256;  // threads: 16 x 16, each 8 x 8 outputs
 
 struct GemmDesc {
   const void* A;
@@ -52,12 +52,12 @@ struct GemmDesc {
   int M, N, K;
   int accumulate;           // C += result instead of C = result
   int form;                 // 0 plain; 1 grouped over routed tiles; 2 grouped along K per expert
-  const int4* tiles;        // form 1: (expert, first row, rows)
+  const int4* tiles;        // form 1: (expert, first row, rows), rows <= 128
   const int32_t* n_tiles;
   const int32_t* offsets;   // form 2: expert e sums rows [offsets[e], offsets[e+1])
   int64_t b_estride;        // form 1: B advances by this per expert
   int64_t c_estride;        // form 2: C advances by this per expert
-  int64_t a_estride;        // form 2: A advances by this per expert (0: rows index A directly)
+  int k_chunk;              // form 0 split along K: blockIdx.z takes [z k_chunk, (z+1) k_chunk)
 };
 
 __device__ __forceinline__ float ld_any(const void* p, int bf16, int64_t i) {
@@ -65,23 +65,26 @@ __device__ __forceinline__ float ld_any(const void* p, int bf16, int64_t i) {
               : static_cast<const float*>(p)[i];
 }
 
+// A 128 x 128 tile of C per CTA.  Each stage stages A [128 x 16] and B [16 x 128]
+// in smem as As[k][m], Bs[k][n] (the global reads run along whichever index is
+// contiguous); thread (tx, ty) then owns rows {4ty..4ty+3, 64+4ty..64+4ty+3}
+// and the same pattern of columns, read as float4 (conflict-free).
 __global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float As[GK][GB + 4];
-  __shared__ float Bs[GK][GB + 4];
+  __shared__ __align__(16) float As[GK][GB + 4];
+  __shared__ __align__(16) float Bs[GK][GB + 4];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   int m_lo, m_hi, k_lo, k_hi;
   const void* Bp = g.B;
   float* Cp = g.C;
   const int n0 = blockIdx.y * GB;
   if (g.form == 1) {
-    const int t = blockIdx.x >> 1;
+    const int t = blockIdx.x;
     if (t >= *g.n_tiles) return;
     const int4 tl = g.tiles[t];
-    m_lo = tl.y + (blockIdx.x & 1) * GB;
-    m_hi = min(tl.y + tl.z, m_lo + GB);
-    if (m_lo >= m_hi) return;
+    m_lo = tl.y;
+    m_hi = tl.y + tl.z;
     Bp = g.b_bf16 ? (const void*)(static_cast<const __nv_bfloat16*>(g.B) + tl.x * g.b_estride)
                   : (const void*)(static_cast<const float*>(g.B) + tl.x * g.b_estride);
     k_lo = 0;
@@ -96,20 +99,26 @@ __global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
       k_lo = g.offsets[e];
       k_hi = g.offsets[e + 1];
       Cp = g.C + e * g.c_estride;
+    } else if (g.k_chunk > 0) {  // one slice of K; C is this slice's partial block
+      k_lo = blockIdx.z * g.k_chunk;
+      k_hi = min(g.K, k_lo + g.k_chunk);
+      Cp = g.C + (int64_t)blockIdx.z * g.M * g.ldc;
     }
   }
-  float acc[4][4];
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-  for (int k0 = k_lo; k0 < k_hi; k0 += GK) {
-    // A tile [GB x GK] -> As[k][m]; coalesced along whichever index is contiguous
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  // global -> registers for the stage starting at k0 (the next stage's loads
+  // are in flight while the current one is multiplied out of smem)
+  float ra[8], rb[8];
+  auto fetch = [&](int k0) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 8; ++q) {
       int mi, ki;
       if (g.sak == 1) { mi = (tid >> 4) + 16 * q; ki = tid & 15; }
-      else { mi = tid & 63; ki = (tid >> 6) + 4 * q; }
+      else { mi = tid & 127; ki = (tid >> 7) + 2 * q; }
       const int m = m_lo + mi, k = k0 + ki;
       float v = 0.0f;
       if (m < m_hi && k < k_hi) {
@@ -117,13 +126,12 @@ __global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
         if (g.form != 2 && g.a_rows != nullptr) row = g.a_rows[m];
         v = ld_any(g.A, g.a_bf16, row * g.sam + (int64_t)k * g.sak);
       }
-      As[ki][mi] = v;
+      ra[q] = v;
     }
-    // B tile [GK x GB] -> Bs[k][n]
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 8; ++q) {
       int ki, ni;
-      if (g.sbn == 1) { ki = (tid >> 6) + 4 * q; ni = tid & 63; }
+      if (g.sbn == 1) { ki = (tid >> 7) + 2 * q; ni = tid & 127; }
       else { ki = tid & 15; ni = (tid >> 4) + 16 * q; }
       const int k = k0 + ki, n = n0 + ni;
       float v = 0.0f;
@@ -132,32 +140,45 @@ __global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
         if (g.form == 2 && g.b_rows != nullptr) krow = g.b_rows[k];
         v = ld_any(Bp, g.b_bf16, krow * g.sbk + (int64_t)n * g.sbn);
       }
-      Bs[ki][ni] = v;
+      rb[q] = v;
     }
+  };
+  auto stash = [&]() {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (g.sak == 1) As[tid & 15][(tid >> 4) + 16 * q] = ra[q];
+      else As[(tid >> 7) + 2 * q][tid & 127] = ra[q];
+      if (g.sbn == 1) Bs[(tid >> 7) + 2 * q][tid & 127] = rb[q];
+      else Bs[tid & 15][(tid >> 4) + 16 * q] = rb[q];
+    }
+  };
+  if (k_lo < k_hi) fetch(k_lo);
+  for (int k0 = k_lo; k0 < k_hi; k0 += GK) {
+    stash();
     __syncthreads();
+    if (k0 + GK < k_hi) fetch(k0 + GK);
 #pragma unroll
     for (int kk = 0; kk < GK; ++kk) {
-      float a[4], b[4];
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = As[kk][ty * 4 + i];
-        b[i] = Bs[kk][tx * 4 + i];
-      }
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
     }
     __syncthreads();
   }
-  // form 2: output rows are the GEMM's M rows (not the expert's pair rows)
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m_lo + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int m = m_lo + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
     if (m >= m_hi) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
       if (n >= g.N) continue;
       float* c = Cp + (int64_t)m * g.ldc + n;
       *c = g.accumulate ? *c + acc[i][j] : acc[i][j];
@@ -165,9 +186,58 @@ __global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
   }
 }
 
-cudaError_t gemm(const GemmDesc& g, int max_tiles, int R, cudaStream_t st) {
+// C (+)= the sum of the K slices' partial blocks, slices in order.
+__global__ void split_sum_kernel(const float* __restrict__ part, int splits, int M, int N,
+                                 float* __restrict__ C, int64_t ldc, int accumulate) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t total = (int64_t)M * N;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = i / N, n = i - m * N;
+    float v = accumulate ? C[m * ldc + n] : 0.0f;
+    for (int s = 0; s < splits; ++s) v += part[(int64_t)s * total + i];
+    C[m * ldc + n] = v;
+  }
+}
+
+// Scratch for the K slices of plain GEMMs with few output tiles (floats).
+constexpr int64_t kSplitScratch = (int64_t)16 << 20;
+
+cudaError_t gemm(const GemmDesc& g0, int max_tiles, int R, cudaStream_t st,
+                 float* split_scratch = nullptr) {
+  GemmDesc g = g0;
+  // A plain GEMM with fewer output tiles than SMs and a long K runs as
+  // K slices (a fixed number, summed in order by a second kernel).
+  if (g.form == 0 && split_scratch != nullptr) {
+    const int64_t tiles = (int64_t)((g.M + GB - 1) / GB) * ((g.N + GB - 1) / GB);
+    int splits = (int)std::min<int64_t>(16, (2 * 148 + tiles - 1) / tiles);
+    splits = std::min(splits, g.K / (8 * GK));
+    while (splits > 1 && (int64_t)splits * g.M * g.N > kSplitScratch) --splits;
+    if (tiles < 148 && splits > 1) {
+      const int chunk = ((g.K + splits - 1) / splits + GK - 1) / GK * GK;
+      splits = (g.K + chunk - 1) / chunk;
+      GemmDesc p = g;
+      p.C = split_scratch;
+      p.ldc = g.N;
+      p.accumulate = 0;
+      p.k_chunk = chunk;
+      count_launch();
+      cudaError_t e = launch_pdl(bwd_gemm_kernel,
+                                 dim3((unsigned)((g.M + GB - 1) / GB), (unsigned)((g.N + GB - 1) / GB),
+                                      (unsigned)splits),
+                                 dim3(GT), 0, st, 1, p);
+      if (e != cudaSuccess) return e;
+      const int64_t total = (int64_t)g.M * g.N;
+      count_launch();
+      return launch_pdl(split_sum_kernel,
+                        dim3((unsigned)std::min<int64_t>((total + 255) / 256, 148 * 16)), dim3(256),
+                        0, st, 1, (const float*)split_scratch, splits, g.M, g.N, g.C, g.ldc,
+                        g.accumulate);
+    }
+  }
   dim3 grid;
-  if (g.form == 1) grid = dim3((unsigned)(2 * max_tiles), (unsigned)((g.N + GB - 1) / GB), 1);
+  if (g.form == 1) grid = dim3((unsigned)max_tiles, (unsigned)((g.N + GB - 1) / GB), 1);
   else grid = dim3((unsigned)((g.M + GB - 1) / GB), (unsigned)((g.N + GB - 1) / GB),
                    g.form == 2 ? (unsigned)R : 1u);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
@@ -391,6 +461,7 @@ BwdLayout bwd_layout(const BwdDims& d) {
   L.csh = take((size_t)N * d.S * d.G * 4);
   L.hsh = take((size_t)N * d.S * d.G * 4);
   L.dhsh = take((size_t)N * d.S * d.G * 4);
+  L.split = take((size_t)kSplitScratch * 4);
   L.total = off;
   return L;
 }
@@ -417,13 +488,14 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   float *duhat = F32(L.duhat), *du = F32(L.du), *rr = F32(L.rr), *dp = F32(L.dp);
   float *dl = F32(L.dl), *rms_part = F32(L.rms_part);
   float *ash = F32(L.ash), *csh = F32(L.csh), *hsh = F32(L.hsh), *dhsh = F32(L.dhsh);
+  float* split = F32(L.split);
   const int64_t FL = (int64_t)F * Lt;
   cudaError_t e;
 #define LMOE_STEP(call) do { if ((e = (call)) != cudaSuccess) return e; } while (0)
   // ---- forward, recomputed in fp32
   // router logits, then the same top-k kernel as the forward
   LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.w_router, bf, 1, D, logits, L.ld_logits, (int)N, R, D), 0,
-                 R, st));
+                 R, st, split));
   LMOE_STEP(launch_route_topk(logits, L.ld_logits, a.bias, N, R, k, d.router, ids, probs, st));
   DispatchScratch ds;
   ds.block_counts = I32(L.block_counts);
@@ -432,7 +504,7 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   ds.tiles = tiles;
   LMOE_STEP(launch_dispatch(ids, N, k, R, I32(L.counts), offsets, perm, inv, ds, st));
   // z = x W_down^T
-  LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.w_down, bf, 1, D, z, Lt, (int)N, Lt, D), 0, R, st));
+  LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.w_down, bf, 1, D, z, Lt, (int)N, Lt, D), 0, R, st, split));
   // a, c = z[perm] W_g,e^T, z[perm] W_u,e^T on the routed tiles
   {
     GemmDesc g = desc(z, 0, Lt, 1, a.w_g, bf, 1, Lt, pa, F, 0, F, Lt);
@@ -456,8 +528,8 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
                        (const float*)o, (const int32_t*)inv, (const float*)probs, a.rms_weight, N,
                        k, Lt, d.rms_eps, u, uhat, rr));
   // ---- step 5: y = s_sh + W_up uhat
-  LMOE_STEP(gemm(desc(a.dy, bf, D, 1, a.w_up, bf, Lt, 1, duhat, Lt, (int)N, Lt, D), 0, R, st));
-  LMOE_STEP(gemm(desc(a.dy, bf, 1, D, uhat, 0, Lt, 1, a.g.dw_up, Lt, D, Lt, (int)N), 0, R, st));
+  LMOE_STEP(gemm(desc(a.dy, bf, D, 1, a.w_up, bf, Lt, 1, duhat, Lt, (int)N, Lt, D), 0, R, st, split));
+  LMOE_STEP(gemm(desc(a.dy, bf, 1, D, uhat, 0, Lt, 1, a.g.dw_up, Lt, D, Lt, (int)N), 0, R, st, split));
   // ---- RMSNorm, and the routing weights' and experts' output gradients
   count_launch();
   LMOE_STEP(launch_pdl(rms_dp_kernel, dim3(warps_grid), dim3(256), 0, st, 1, (const float*)u,
@@ -479,7 +551,7 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   {  // dW_o,e = dE^T h over expert e's rows
     GemmDesc g = desc(dE, 0, 1, Lt, h, 0, F, 1, a.g.dw_o, F, Lt, F, 0);
     g.form = 2; g.offsets = offsets; g.c_estride = FL;
-    LMOE_STEP(gemm(g, 0, R, st));
+    LMOE_STEP(gemm(g, 0, R, st, split));
   }
   count_launch();
   LMOE_STEP(launch_pdl(situ_bwd_kernel, dim3(grid_for(P * F, 256)), dim3(256), 0, st, 1, pa, pc,
@@ -487,9 +559,9 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   {  // dW_g,e = da^T z[perm], dW_u,e = dc^T z[perm]
     GemmDesc g = desc(pa, 0, 1, F, z, 0, Lt, 1, a.g.dw_g, Lt, F, Lt, 0);
     g.form = 2; g.offsets = offsets; g.c_estride = FL; g.b_rows = perm;
-    LMOE_STEP(gemm(g, 0, R, st));
+    LMOE_STEP(gemm(g, 0, R, st, split));
     g.A = pc; g.C = a.g.dw_u;
-    LMOE_STEP(gemm(g, 0, R, st));
+    LMOE_STEP(gemm(g, 0, R, st, split));
   }
   {  // dzp = da W_g,e + dc W_u,e (written over o)
     GemmDesc g = desc(pa, 0, F, 1, a.w_g, bf, Lt, 1, o, Lt, 0, Lt, F);
@@ -506,16 +578,16 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   LMOE_STEP(launch_pdl(router_bwd_kernel, dim3(warps_grid), dim3(256), 0, st, 1,
                        (const float*)logits, (int64_t)L.ld_logits, (const int32_t*)ids,
                        (const float*)probs, (const float*)dp, N, k, R, d.router, dl));
-  LMOE_STEP(gemm(desc(dl, 0, 1, R, a.x, bf, D, 1, a.g.dw_router, D, R, D, (int)N), 0, R, st));
+  LMOE_STEP(gemm(desc(dl, 0, 1, R, a.x, bf, D, 1, a.g.dw_router, D, R, D, (int)N), 0, R, st, split));
   // ---- step 1
-  LMOE_STEP(gemm(desc(du, 0, 1, Lt, a.x, bf, D, 1, a.g.dw_down, D, Lt, D, (int)N), 0, R, st));
-  LMOE_STEP(gemm(desc(du, 0, Lt, 1, a.w_down, bf, D, 1, a.g.dx, D, (int)N, D, Lt), 0, R, st));
-  LMOE_STEP(gemm(desc(dl, 0, R, 1, a.w_router, bf, D, 1, a.g.dx, D, (int)N, D, R, 1), 0, R, st));
+  LMOE_STEP(gemm(desc(du, 0, 1, Lt, a.x, bf, D, 1, a.g.dw_down, D, Lt, D, (int)N), 0, R, st, split));
+  LMOE_STEP(gemm(desc(du, 0, Lt, 1, a.w_down, bf, D, 1, a.g.dx, D, (int)N, D, Lt), 0, R, st, split));
+  LMOE_STEP(gemm(desc(dl, 0, R, 1, a.w_router, bf, D, 1, a.g.dx, D, (int)N, D, R, 1), 0, R, st, split));
   // ---- step 4: shared experts, dE = dy
   if (S > 0) {
     const int SG = S * G;
-    LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.ws_g, bf, 1, D, ash, SG, (int)N, SG, D), 0, R, st));
-    LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.ws_u, bf, 1, D, csh, SG, (int)N, SG, D), 0, R, st));
+    LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.ws_g, bf, 1, D, ash, SG, (int)N, SG, D), 0, R, st, split));
+    LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.ws_u, bf, 1, D, csh, SG, (int)N, SG, D), 0, R, st, split));
     count_launch();
     LMOE_STEP(launch_pdl(situ_fwd_kernel, dim3(grid_for(N * SG, 256)), dim3(256), 0, st, 1,
                          (const float*)ash, (const float*)csh, N * SG, d.beta1, d.beta2, hsh));
@@ -525,18 +597,18 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
                           : (const void*)(static_cast<const float*>(a.ws_o) + (int64_t)j * D * G);
       // dh_sh,j = dy W_o,sh,j ;  dW_o,sh,j = dy^T h_sh,j
       LMOE_STEP(gemm(desc(a.dy, bf, D, 1, wo, bf, G, 1, dhsh + (int64_t)j * G, SG, (int)N, G, D),
-                     0, R, st));
+                     0, R, st, split));
       LMOE_STEP(gemm(desc(a.dy, bf, 1, D, hsh + (int64_t)j * G, 0, SG, 1,
                           a.g.dws_o + (int64_t)j * D * G, G, D, G, (int)N),
-                     0, R, st));
+                     0, R, st, split));
     }
     count_launch();
     LMOE_STEP(launch_pdl(situ_bwd_kernel, dim3(grid_for(N * SG, 256)), dim3(256), 0, st, 1, ash,
                          csh, (const float*)dhsh, N * SG, d.beta1, d.beta2));
-    LMOE_STEP(gemm(desc(ash, 0, 1, SG, a.x, bf, D, 1, a.g.dws_g, D, SG, D, (int)N), 0, R, st));
-    LMOE_STEP(gemm(desc(csh, 0, 1, SG, a.x, bf, D, 1, a.g.dws_u, D, SG, D, (int)N), 0, R, st));
-    LMOE_STEP(gemm(desc(ash, 0, SG, 1, a.ws_g, bf, D, 1, a.g.dx, D, (int)N, D, SG, 1), 0, R, st));
-    LMOE_STEP(gemm(desc(csh, 0, SG, 1, a.ws_u, bf, D, 1, a.g.dx, D, (int)N, D, SG, 1), 0, R, st));
+    LMOE_STEP(gemm(desc(ash, 0, 1, SG, a.x, bf, D, 1, a.g.dws_g, D, SG, D, (int)N), 0, R, st, split));
+    LMOE_STEP(gemm(desc(csh, 0, 1, SG, a.x, bf, D, 1, a.g.dws_u, D, SG, D, (int)N), 0, R, st, split));
+    LMOE_STEP(gemm(desc(ash, 0, SG, 1, a.ws_g, bf, D, 1, a.g.dx, D, (int)N, D, SG, 1), 0, R, st, split));
+    LMOE_STEP(gemm(desc(csh, 0, SG, 1, a.ws_u, bf, D, 1, a.g.dx, D, (int)N, D, SG, 1), 0, R, st, split));
   }
 #undef LMOE_STEP
   return cudaGetLastError();

@@ -183,13 +183,13 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
         first = chunk_counts[(int64_t)cb * R + e];
         tot = counts[e];
       } else {
-        for (int c0 = 0; c0 < C; c0 += 16) {
-          int32_t v[16];
+        for (int c0 = 0; c0 < C; c0 += 32) {  // up to 32 loads in flight
+          int32_t v[32];
 #pragma unroll
-          for (int u = 0; u < 16; ++u)
+          for (int u = 0; u < 32; ++u)
             v[u] = c0 + u < C ? chunk_counts[(int64_t)(c0 + u) * R + e] : 0;
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
+          for (int u = 0; u < 32; ++u) {
             first += c0 + u < cb ? v[u] : 0;
             tot += v[u];
           }

@@ -108,7 +108,7 @@ struct BwdArgs {
 };
 struct BwdLayout {
   size_t header, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, z, a, c, h,
-      dh, o, dE, u, uhat, duhat, du, rr, dp, dl, rms_part, ash, csh, hsh, dhsh, total;
+      dh, o, dE, u, uhat, duhat, du, rr, dp, dl, rms_part, ash, csh, hsh, dhsh, split, total;
   int ld_logits, max_tiles;
 };
 BwdLayout bwd_layout(const BwdDims& d);
