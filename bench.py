@@ -184,6 +184,13 @@ def cpu_baseline(wl: synth.Workload, seed: int, budget_s: float = 12.0) -> dict:
                       f"{t:.1f} s"}
 
 
+def workload_config(wl: synth.Workload, world: int) -> dict:
+    """The layer's sizes, shared by both arms' JSON lines."""
+    return {"workload": wl.name, "n_tokens": wl.n_tokens, "d": wl.d, "latent": wl.latent,
+            "n_routed": wl.n_routed, "top_k": wl.top_k, "ff_routed": wl.ff_routed,
+            "n_shared": wl.n_shared, "ff_shared": wl.ff_shared, "parallelism": f"replicas{world}"}
+
+
 def run_reference(args, wl):
     world, rank, _ = _dist()
     if rank != 0:
@@ -216,7 +223,7 @@ def run_reference(args, wl):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "tokens_per_step": n_step, "n_tokens": wl.n_tokens},
+            "config": workload_config(wl, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"{n_step} of {wl.n_tokens} tokens per step"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -567,11 +574,8 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": wl.name, "n_tokens": wl.n_tokens, "d": wl.d, "latent": wl.latent,
-                   "n_routed": wl.n_routed, "top_k": wl.top_k, "ff_routed": wl.ff_routed,
-                   "n_shared": wl.n_shared, "ff_shared": wl.ff_shared,
-                   "parallelism": f"replicas{world}", "l2": "flushed (256 MiB write) between steps",
-                   "launch": "eager" if args.eager else "cuda graph replay"},
+        "config": dict(workload_config(wl, world), l2="flushed (256 MiB write) between steps",
+                       launch="eager" if args.eager else "cuda graph replay"),
         "layer_roofline": {"flops": wl.flops(), "compulsory_bytes": cbytes, "experts_used": used,
                            "roof_us": roof_s * 1e6, "frac": roof_s / (ms_per_step / 1e3),
                            "peak_source": peaks["source"] + " burst"},
