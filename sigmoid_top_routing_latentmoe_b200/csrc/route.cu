@@ -31,10 +31,9 @@ __device__ __forceinline__ void warp_argmax(float& key, int& idx) {
 // then p = s / max(sum s, 1e-9); with softmax != 0, s holds the logits and
 // p = exp(s - s_first) / sum over the slots (slot 0 holds the largest).
 // Called by all 32 lanes of a warp.
-template <int VPL>
+template <int VPL, bool SOFTMAX>
 __device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (&key_in)[VPL], int R,
-                                            int k, int32_t* ids_row, float* probs_row,
-                                            int softmax) {
+                                            int k, int32_t* ids_row, float* probs_row) {
   const int lane = threadIdx.x & 31;
   float key[VPL];
 #pragma unroll
@@ -65,7 +64,7 @@ __device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (
       }
     }
     sc = __shfl_sync(0xffffffffu, sc, bi & 31);
-    if (softmax) {
+    if (SOFTMAX) {
       if (slot == 0) first = sc;
       sc = expf(sc - first);
     }
@@ -82,7 +81,7 @@ __device__ __forceinline__ void select_topk(const float (&s)[VPL], const float (
       if (lane <= (slot & 31)) probs_row[base + lane] = sel_s;
     }
   }
-  if (!softmax) den = fmaxf(den, 1e-9f);
+  if (!SOFTMAX) den = fmaxf(den, 1e-9f);
   __syncwarp();
   for (int slot = lane; slot < k; slot += 32) probs_row[slot] = probs_row[slot] / den;
 }
@@ -145,13 +144,14 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(const T* __restrict__ x
     s[0] = sigmoid_f(logit);
     key[0] = s[0] + ((bias != nullptr && lane < R) ? bias[lane] : 0.0f);
   }
-  select_topk<1>(s, key, R, k, ids + t * k, probs + t * k, router);
+  if (router) select_topk<1, true>(s, key, R, k, ids + t * k, probs + t * k);
+  else select_topk<1, false>(s, key, R, k, ids + t * k, probs + t * k);
 }
 
-template <int VPL>
+template <int VPL, bool SOFTMAX>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
                                                          int64_t ld, const float* __restrict__ bias,
-                                                         int64_t n, int R, int k, int router,
+                                                         int64_t n, int R, int k,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ probs) {
   pdl_trigger();
@@ -165,14 +165,14 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   for (int j = 0; j < VPL; ++j) {
     int e = j * 32 + lane;
     float l = (e < R) ? lr[e] : 0.0f;
-    if (router) {
+    if (SOFTMAX) {
       s[j] = key[j] = l;
     } else {
       s[j] = sigmoid_f(l);
       key[j] = s[j] + ((bias != nullptr && e < R) ? bias[e] : 0.0f);
     }
   }
-  select_topk<VPL>(s, key, R, k, ids + t * k, probs + t * k, router);
+  select_topk<VPL, SOFTMAX>(s, key, R, k, ids + t * k, probs + t * k);
 }
 
 }  // namespace
@@ -211,8 +211,10 @@ cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias
 #define LMOE_TOPK_CASE(V)                                                                  \
   if (vpl <= V) {                                                                          \
     count_launch();                                                                        \
-    return launch_pdl(route_topk_kernel<V>, dim3(blocks), dim3(warps * 32), 0, st, 1, logits, \
-                      ld, bias, n, R, k, router, ids, probs);                             \
+    return router ? launch_pdl(route_topk_kernel<V, true>, dim3(blocks), dim3(warps * 32), 0, st, \
+                               1, logits, ld, bias, n, R, k, ids, probs)                  \
+                  : launch_pdl(route_topk_kernel<V, false>, dim3(blocks), dim3(warps * 32), 0,    \
+                               st, 1, logits, ld, bias, n, R, k, ids, probs);             \
   }
   LMOE_TOPK_CASE(1)
   LMOE_TOPK_CASE(2)
