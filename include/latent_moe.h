@@ -138,6 +138,20 @@ LMOE_API lmoe_status moe_dispatch(const lmoe_dims* dims, const int32_t* ids, int
                          int32_t* offsets, int32_t* perm_token, int32_t* inv_pair, void* ws,
                          size_t ws_bytes, lmoe_stream stream);
 
+/* Consistency check of a permutation (what moe_dispatch promises, verified on
+ * the device; the pages' stable argsort + bincount + cumsum define it):
+ * every id in [0, R); counts summing to N*k; offsets[0] = 0 and offsets[e+1] -
+ * offsets[e] = counts[e]; inv_pair a bijection onto the N*k sorted slots
+ * (every slot taken exactly once); perm_token[inv_pair[t, i]] = t; the slot of
+ * (t, i) inside its expert's range; tokens ascending inside an expert.  A
+ * violation sets LMOE_EDEVICE in the workspace status word (read it with
+ * lmoe_get_device_status); nothing is written otherwise.  Workspace:
+ * lmoe_workspace_size(dims) bytes. */
+LMOE_API lmoe_status lmoe_check_dispatch(const lmoe_dims* dims, const int32_t* ids,
+                                         const int32_t* counts, const int32_t* offsets,
+                                         const int32_t* perm_token, const int32_t* inv_pair,
+                                         void* ws, size_t ws_bytes, lmoe_stream stream);
+
 /* Routed experts on the sorted pairs (sec-07 compute flow step 3 and the
  * sparse-dispatch subsection; latent_moe.py _routed_u, without padding to
  * the capacity C): for each expert e and sorted row r in

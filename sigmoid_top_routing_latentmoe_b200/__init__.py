@@ -75,6 +75,7 @@ _sigs = {
     "moe_combine": (_S, [_DP, _P, _P, _P, _P, _P, _P]),
     "moe_router_losses": (_S, [_DP, _P, ctypes.c_int64, _P, _P, _P, ctypes.c_size_t, _P]),
     "lmoe_backward_workspace_size": (ctypes.c_size_t, [_DP]),
+    "lmoe_check_dispatch": (_S, [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "latent_moe_backward": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, ctypes.POINTER(Grads), _P,
                                  ctypes.c_size_t, _P]),
     "latent_moe_forward": (_S, [_DP, ctypes.POINTER(Weights), _P, _P, _P, _P, _P, _P,
@@ -185,6 +186,14 @@ def moe_dispatch(dims, ids, counts, offsets, perm_token, inv_pair, ws, stream=No
     _check(_lib.moe_dispatch(ctypes.byref(dims), _ptr(ids), _ptr(counts), _ptr(offsets),
                              _ptr(perm_token), _ptr(inv_pair), _ptr(ws), ws.numel(),
                              _stream(stream)), "moe_dispatch")
+
+
+def check_dispatch(dims, ids, counts, offsets, perm_token, inv_pair, ws, stream=None):
+    """Device-side consistency check of a permutation; a violation sets EDEVICE
+    in the workspace status word (lmoe_get_device_status)."""
+    _check(_lib.lmoe_check_dispatch(ctypes.byref(dims), _ptr(ids), _ptr(counts), _ptr(offsets),
+                                    _ptr(perm_token), _ptr(inv_pair), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "lmoe_check_dispatch")
 
 
 def moe_dispatch_noalloc(dims, ids, counts, offsets, perm_token, inv_pair, stream=None):

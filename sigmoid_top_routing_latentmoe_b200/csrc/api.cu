@@ -529,6 +529,30 @@ lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const int32_t* 
   return run_expert_ffn<float>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
 }
 
+lmoe_status lmoe_check_dispatch(const lmoe_dims* dims, const int32_t* ids, const int32_t* counts,
+                                const int32_t* offsets, const int32_t* perm_token,
+                                const int32_t* inv_pair, void* ws, size_t ws_bytes,
+                                lmoe_stream stream) {
+  LMOE_TRY(check_dims(dims));
+  LMOE_PTR(counts, "counts");
+  LMOE_PTR(offsets, "offsets");
+  if (dims->n_tokens > 0) {
+    LMOE_PTR(ids, "ids");
+    LMOE_PTR(perm_token, "perm_token");
+    LMOE_PTR(inv_pair, "inv_pair");
+  }
+  LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
+  LMOE_TRY(check_device());
+  const Layout L = layout(dims, false);
+  // the bitmap lives in the sorted-row area of the workspace (N*k*l elements >= N*k/32 words)
+  uint32_t* bitmap = at<uint32_t>(ws, L.eo);
+  LMOE_CUDA(launch_check_dispatch(ids, dims->n_tokens, dims->top_k, dims->n_routed, counts, offsets,
+                                  perm_token, inv_pair, bitmap, &at<WsHeader>(ws, L.header)->status,
+                                  (cudaStream_t)stream),
+            "check dispatch");
+  return LMOE_OK;
+}
+
 static BwdDims bwd_dims(const lmoe_dims* d) {
   BwdDims b;
   b.N = d->n_tokens; b.d = d->d; b.L = d->latent; b.R = d->n_routed; b.k = d->top_k;

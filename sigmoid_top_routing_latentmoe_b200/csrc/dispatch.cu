@@ -278,6 +278,63 @@ __global__ void gather_rows_kernel(const T* __restrict__ z, const int32_t* __res
   for (int i = lane; i < width / vec; i += 32) d[i] = s[i];
 }
 
+// Consistency check of a permutation: ids in range, counts summing to N k,
+// offsets the exclusive sum of counts, inv_pair a bijection onto the sorted
+// slots (a bitmap, every slot set exactly once), perm_token[inv_pair[t, i]] = t,
+// slots of expert e inside [offsets[e], offsets[e+1]) and tokens ascending
+// inside an expert.  A violation sets kStatusDevice in the status word.
+__global__ void check_counts_kernel(const int32_t* __restrict__ counts,
+                                    const int32_t* __restrict__ offsets, int R, int64_t n_pairs,
+                                    int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
+  if (threadIdx.x != 0) return;
+  int64_t run = 0;
+  bool bad = offsets[0] != 0;
+  for (int e = 0; e < R; ++e) {
+    if (counts[e] < 0 || offsets[e + 1] - offsets[e] != counts[e]) bad = true;
+    run += counts[e];
+  }
+  if (run != n_pairs || offsets[R] != n_pairs) bad = true;
+  if (bad) record_status(status, kStatusDevice);
+}
+__global__ void check_pairs_kernel(const int32_t* __restrict__ ids,
+                                   const int32_t* __restrict__ offsets,
+                                   const int32_t* __restrict__ perm_token,
+                                   const int32_t* __restrict__ inv_pair, int64_t n_pairs, int k,
+                                   int R, uint32_t* __restrict__ bitmap,
+                                   int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
+  for (int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; p < n_pairs;
+       p += (int64_t)gridDim.x * blockDim.x) {
+    const int e = ids[p];
+    const int64_t slot = inv_pair[p];
+    const int32_t t = (int32_t)(p / k);
+    bool bad = (unsigned)e >= (unsigned)R || slot < 0 || slot >= n_pairs;
+    if (!bad) {
+      bad = perm_token[slot] != t || slot < offsets[e] || slot >= offsets[e + 1];
+      // tokens ascend inside an expert: the next slot of the same expert holds a later token
+      if (!bad && slot + 1 < offsets[e + 1] && slot + 1 < n_pairs && perm_token[slot + 1] <= t)
+        bad = true;
+      const uint32_t bit = 1u << (slot & 31);
+      if (!bad && (atomicOr(&bitmap[slot >> 5], bit) & bit)) bad = true;  // slot taken twice
+    }
+    if (bad) record_status(status, kStatusDevice);
+  }
+}
+__global__ void check_bitmap_kernel(const uint32_t* __restrict__ bitmap, int64_t n_pairs,
+                                    int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < (n_pairs + 31) / 32;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t left = n_pairs - w * 32;
+    const uint32_t want = left >= 32 ? 0xffffffffu : ((1u << left) - 1u);
+    if (bitmap[w] != want) record_status(status, kStatusDevice);  // a slot nobody maps to
+  }
+}
+
 // Tile list from offsets alone (for moe_expert_ffn called on its own).  One
 // warp: each lane scans a contiguous run of experts.
 __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int R,
@@ -352,6 +409,27 @@ cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t
   return cudaGetLastError();
 }
 
+
+cudaError_t launch_check_dispatch(const int32_t* ids, int64_t n, int k, int R,
+                                  const int32_t* counts, const int32_t* offsets,
+                                  const int32_t* perm_token, const int32_t* inv_pair,
+                                  uint32_t* bitmap, int32_t* status, cudaStream_t st) {
+  const int64_t n_pairs = n * k;
+  cudaError_t e = cudaMemsetAsync(bitmap, 0, (size_t)((n_pairs + 31) / 32) * 4, st);
+  if (e != cudaSuccess) return e;
+  count_launch();
+  e = launch_pdl(check_counts_kernel, dim3(1), dim3(32), 0, st, 1, counts, offsets, R, n_pairs,
+                 status);
+  if (e != cudaSuccess || n_pairs == 0) return e;
+  const unsigned blocks = (unsigned)std::min<int64_t>((n_pairs + 255) / 256, 148 * 8);
+  count_launch();
+  e = launch_pdl(check_pairs_kernel, dim3(blocks), dim3(256), 0, st, 1, ids, offsets, perm_token,
+                 inv_pair, n_pairs, k, R, bitmap, status);
+  if (e != cudaSuccess) return e;
+  count_launch();
+  return launch_pdl(check_bitmap_kernel, dim3(blocks), dim3(256), 0, st, 1, (const uint32_t*)bitmap,
+                    n_pairs, status);
+}
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
                                cudaStream_t st) {

@@ -42,6 +42,11 @@ cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t
                             const DispatchScratch& s, cudaStream_t st);
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
                                cudaStream_t st);
+// Consistency check of a permutation (bitmap: (N k + 31) / 32 words of scratch).
+cudaError_t launch_check_dispatch(const int32_t* ids, int64_t n, int k, int R,
+                                  const int32_t* counts, const int32_t* offsets,
+                                  const int32_t* perm_token, const int32_t* inv_pair,
+                                  uint32_t* bitmap, int32_t* status, cudaStream_t st);
 // zp[r, :] = z[perm_token[r], :]
 template <typename T>
 cudaError_t launch_gather_rows(const T* z, const int32_t* perm_token, int64_t n_rows, int width,

@@ -314,3 +314,61 @@ def test_capped_wait_reports_timeout():
     # the context is still usable afterwards
     t = torch.ones(4, device="cuda") * 2
     assert float(t.sum()) == 8.0
+
+
+# ------------------------------------------------ device-side consistency check
+
+def _dispatch(N, k, R, seed, skew=False):
+    dims = lm.make_dims(N, 64, 32, R, k, 0, 64, 64)
+    ws = lm.alloc_workspace(dims)
+    ids = torch.from_numpy(_random_ids(N, k, R, seed=seed, skew=skew)).cuda()
+    counts = torch.empty(R, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(R + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(N * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(N * k, dtype=torch.int32, device="cuda")
+    lm.moe_dispatch(dims, ids, counts, offsets, perm, inv, ws)
+    return dims, ws, ids, counts, offsets, perm, inv
+
+
+@pytest.mark.parametrize("N,k,R,skew", [(300, 2, 16, False), (4096, 2, 16, True),
+                                        (1000, 16, 896, False), (1, 1, 4, False)])
+def test_check_dispatch_accepts_the_permutation(N, k, R, skew):
+    dims, ws, ids, counts, offsets, perm, inv = _dispatch(N, k, R, seed=N + R, skew=skew)
+    lm.check_dispatch(dims, ids, counts, offsets, perm, inv, ws)
+    torch.cuda.synchronize()
+    assert lm.get_device_status(ws) == lm.OK
+
+
+def test_check_dispatch_flags_corruptions():
+    """Each corruption (in-range values only) sets EDEVICE: two pairs swapped
+    across experts, a wrong token in perm_token, a count moved between experts,
+    two pairs on one slot."""
+    N, k, R = 512, 2, 16
+    dims, ws, ids, counts, offsets, perm, inv = _dispatch(N, k, R, seed=5)
+    h_ids = host(ids).reshape(-1)
+    a = 0
+    b = int(np.nonzero(h_ids != h_ids[0])[0][0])
+
+    def flagged(**bad):
+        lm.workspace_init(ws)
+        args = dict(ids=ids, counts=counts, offsets=offsets, perm=perm, inv=inv)
+        args.update(bad)
+        lm.check_dispatch(dims, args["ids"], args["counts"], args["offsets"], args["perm"],
+                          args["inv"], ws)
+        torch.cuda.synchronize()
+        return lm.get_device_status(ws) == lm.EDEVICE
+
+    assert not flagged()
+    inv2 = inv.clone()
+    inv2[a], inv2[b] = inv[b], inv[a]
+    assert flagged(inv=inv2)
+    perm2 = perm.clone()
+    perm2[0] = (perm[0] + 1) % N
+    assert flagged(perm=perm2)
+    counts2 = counts.clone()
+    counts2[0] += 1
+    counts2[1] -= 1
+    assert flagged(counts=counts2)
+    inv3 = inv.clone()
+    inv3[1] = inv[0]
+    assert flagged(inv=inv3)
