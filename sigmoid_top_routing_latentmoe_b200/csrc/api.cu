@@ -228,9 +228,11 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
   return LMOE_OK;
 }
 
+// z != nullptr: the scatter also writes the sorted rows of z to the workspace
+// (the A operand of the routed GEMMs).
 static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t* counts,
                                 int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
-                                cudaStream_t st) {
+                                cudaStream_t st, const void* z = nullptr) {
   const Layout L = layout(d, false);
   DispatchScratch s;
   s.block_counts = at<int32_t>(ws, L.block_counts);
@@ -238,19 +240,22 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
   s.n_mtiles = &at<WsHeader>(ws, L.header)->n_mtiles;
   s.tiles = at<int4>(ws, L.tiles);
   ProfScope ps("dispatch", st);
+  const int es = d->dtype == LMOE_BF16 ? 2 : 4;
   LMOE_CUDA(launch_dispatch(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm, inv,
-                            s, st),
+                            s, st, z, z != nullptr ? at<char>(ws, L.zp) : nullptr,
+                            d->latent * es),
             "dispatch");
   return LMOE_OK;
 }
 
 // Routed experts on sorted pairs; the tile list must already be in the workspace.
 // perm holds the token of each sorted pair: its rows of z are first copied in
-// sorted order, the A operand of GEMM1.
+// sorted order, the A operand of GEMM1, unless the dispatch already did
+// (rows_sorted).
 template <typename T>
 static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32_t* perm,
                                   const void* w_g, const void* w_u, const void* w_o, void* eo,
-                                  void* ws, cudaStream_t st) {
+                                  void* ws, cudaStream_t st, bool rows_sorted = false) {
   const Layout L = layout(d, false);
   const int64_t P = d->n_tokens * d->top_k;
   if (P == 0) return LMOE_OK;
@@ -260,7 +265,7 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   const int4* tiles = at<int4>(ws, L.tiles);
   const int32_t* n_tiles = &at<WsHeader>(ws, L.header)->n_mtiles;
   const bool tc = std::is_same<T, __nv_bfloat16>::value;
-  {
+  if (!rows_sorted) {
     ProfScope ps("gather", st);
     LMOE_CUDA(launch_gather_rows<T>((const T*)z, perm, P, Lt, zp, st), "gather");
   }
@@ -348,8 +353,11 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
               "route_topk");
   }
   // step 3: dispatch, routed experts, combine + RMSNorm
-  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st));
-  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st));
+  // Small sorted copies of z (up to 16 MiB) are made by the scatter itself, saving a
+  // launch; larger ones by the gather kernel, which has more memory parallelism.
+  const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * sizeof(T) <= (16u << 20);
+  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
+  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
   {
     ProfScope ps("combine", st);
     LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, k, Lt, d->rms_eps, uhat, st),
@@ -408,8 +416,11 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
   // step 2: routing
   LMOE_TRY(run_route<T>(d, x, w->w_router, w->expert_bias, ids, probs, ws, st));
   // step 3: dispatch, routed experts, combine + RMSNorm
-  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st));
-  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st));
+  // Small sorted copies of z (up to 16 MiB) are made by the scatter itself, saving a
+  // launch; larger ones by the gather kernel, which has more memory parallelism.
+  const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * sizeof(T) <= (16u << 20);
+  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
+  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
   {
     ProfScope ps("combine", st);
     LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, d->top_k, Lt, d->rms_eps, uhat,

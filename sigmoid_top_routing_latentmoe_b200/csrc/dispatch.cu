@@ -157,11 +157,17 @@ __global__ void empty_scan_kernel(int R, int32_t* __restrict__ counts, int32_t* 
 // expert e in earlier chunks -- from the chunk counts: summed here when
 // `prefixed` is 0, or read as the column scan left them.  CTA 0 also writes
 // counts (unless prefixed), offsets and the routed row-tile list.
+// With z != nullptr each chunk has `subs` CTAs: all of them rank the chunk's
+// pairs (cheap), sub-CTA 0 writes perm_token / inv_pair, and sub-CTA s copies
+// the z rows of the pairs whose index is s modulo subs to their sorted slots in
+// zp (row_vecs 16-byte vectors per row), a warp's rows copied together so that
+// many loads are in flight.
 __global__ void __launch_bounds__(kThreads) scatter_kernel(
     const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int k, int R, int C,
     const int32_t* __restrict__ chunk_counts, int prefixed, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ n_mtiles, int4* __restrict__ tiles,
-    int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair) {
+    int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair, int subs,
+    const uint4* __restrict__ z, uint4* __restrict__ zp, int row_vecs) {
   pdl_trigger();
   pdl_wait();
   // [kWarps][R] per-warp counts, then first slots; [R] this chunk's first slot
@@ -170,8 +176,9 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t totals[2];
   __shared__ int32_t carry[2];
+  __shared__ int32_t row_slot[kWarps][32], row_tok[kWarps][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int cb = blockIdx.x;
+  const int cb = blockIdx.x / subs, sub = blockIdx.x - cb * subs;
   for (int i = threadIdx.x; i < kWarps * R; i += kThreads) wcnt[i] = 0;
   if (threadIdx.x == 0) carry[0] = carry[1] = 0;
   __syncthreads();
@@ -201,7 +208,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
     const int32_t ex_t = block_exclusive_scan(nt, warp_sums, &totals[1]) + carry[1];
     if (e < R) {
       base[e] = ex_c + first;
-      if (cb == 0) {
+      if (cb == 0 && sub == 0) {
         if (!prefixed) counts[e] = tot;
         offsets[e] = ex_c;
         for (int t = 0; t * kTileM < tot; ++t)
@@ -215,7 +222,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
     }
     __syncthreads();
   }
-  if (cb == 0 && threadIdx.x == 0) {
+  if (cb == 0 && sub == 0 && threadIdx.x == 0) {
     offsets[R] = carry[0];
     *n_mtiles = carry[1];
   }
@@ -255,9 +262,41 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
     if (valid && lower == 0) my[e] += __popc(same);
     __syncwarp();
     const int32_t tok = (int32_t)((uint32_t)p / (uint32_t)k);  // pairs < 2^31
-    if (valid) {
+    if (valid && sub == 0) {
       perm_token[slot] = tok;
       inv_pair[p] = slot;
+    }
+    if (z != nullptr) {
+      // this sub-CTA's rows of the step: pairs p with p mod subs == sub
+      const bool mine = valid && (int)(p % subs) == sub;
+      const unsigned sel = __ballot_sync(0xffffffffu, mine);
+      const int at = __popc(sel & ((1u << lane) - 1u));
+      if (mine) {
+        row_slot[warp][at] = slot;
+        row_tok[warp][at] = tok;
+      }
+      __syncwarp();
+      const int n_vec = __popc(sel) * row_vecs;
+      for (int i0 = 0; i0 < n_vec; i0 += 32 * 8) {  // 8 loads in flight per lane
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * 32 + lane;
+          if (i < n_vec) {
+            const int r = i / row_vecs, c = i - r * row_vecs;
+            v[u] = z[(int64_t)row_tok[warp][r] * row_vecs + c];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * 32 + lane;
+          if (i < n_vec) {
+            const int r = i / row_vecs, c = i - r * row_vecs;
+            zp[(int64_t)row_slot[warp][r] * row_vecs + c] = v[u];
+          }
+        }
+      }
+      __syncwarp();
     }
   }
 }
@@ -376,7 +415,8 @@ int dispatch_blocks(int64_t n_pairs) {
 
 cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
-                            const DispatchScratch& s, cudaStream_t st) {
+                            const DispatchScratch& s, cudaStream_t st, const void* z, void* zp,
+                            int row_bytes) {
   const int64_t n_pairs = n * k;
   const int64_t chunk = chunk_pairs(n_pairs);
   const int nb = dispatch_blocks(n_pairs);
@@ -401,10 +441,13 @@ cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t
   const size_t smem = (size_t)(kWarps + 1) * R * sizeof(int32_t);
   e = set_smem(scatter_kernel, smem);
   if (e != cudaSuccess) return e;
+  // with the row copy: enough CTAs per chunk to cover the SMs twice (at most 16)
+  const int subs = z != nullptr ? std::max(1, std::min(16, (2 * 148 + nb - 1) / nb)) : 1;
   count_launch();
-  e = launch_pdl(scatter_kernel, dim3(nb), dim3(kThreads), smem, st, 1, ids, n_pairs, chunk, k, R,
-                 nb, (const int32_t*)s.block_counts, prefixed, counts, offsets, s.n_mtiles,
-                 s.tiles, perm_token, inv_pair);
+  e = launch_pdl(scatter_kernel, dim3((unsigned)(nb * subs)), dim3(kThreads), smem, st, 1, ids,
+                 n_pairs, chunk, k, R, nb, (const int32_t*)s.block_counts, prefixed, counts,
+                 offsets, s.n_mtiles, s.tiles, perm_token, inv_pair, subs,
+                 static_cast<const uint4*>(z), static_cast<uint4*>(zp), row_bytes / 16);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -37,9 +37,12 @@ struct DispatchScratch {
   int4* tiles;            // out: [max_tiles] (expert, row0, rows, 0)
 };
 int dispatch_blocks(int64_t n_pairs);
+// With z != nullptr the scatter also copies each pair's z row (row_bytes, a
+// multiple of 16) to its sorted slot in zp.
 cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
-                            const DispatchScratch& s, cudaStream_t st);
+                            const DispatchScratch& s, cudaStream_t st, const void* z = nullptr,
+                            void* zp = nullptr, int row_bytes = 0);
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
                                cudaStream_t st);
 // Consistency check of a permutation (bitmap: (N k + 31) / 32 words of scratch).
