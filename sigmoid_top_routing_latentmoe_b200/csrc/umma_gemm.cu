@@ -74,6 +74,7 @@ constexpr int kPadMap = 5;
 struct Params {
   CUtensorMap tmA0, tmA1;              // A operands (FINAL: h_sh, uhat)
   CUtensorMap tmB0, tmB1, tmB2, tmB3;  // B operands (see decode_tile)
+  int map_mask;                        // encoded maps: bit 0 A0, 1 A1, 2 B0, 3 B1, 4 B2, 5 B3
   int M;                               // dense rows
   int n_tiles;                         // tiles along the output columns
   int kb0, kb1;                        // K blocks (FINAL: per shared expert, then uhat)
@@ -889,6 +890,14 @@ __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_cons
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (threadIdx.x == 32) {  // fetch the encoded tensor maps while the previous kernel finishes
+    const CUtensorMap* maps[6] = {&p.tmA0, &p.tmA1, &p.tmB0, &p.tmB1, &p.tmB2, &p.tmB3};
+#pragma unroll
+    for (int i = 0; i < 6; ++i)
+      if (p.map_mask & (1 << i))
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(maps[i]))
+                     : "memory");
+  }
   if (warp == 1) {
     if (CG == 1) {
       asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -1057,6 +1066,7 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
     ok = ok && make_map3(&p.tmB2, a.ws_g, a.d, a.G, a.S, SUB) &&
          make_map3(&p.tmB3, a.ws_u, a.d, a.G, a.S, SUB);
   if (!ok) return cudaErrorInvalidValue;
+  p.map_mask = 1 | (a.L > 0 ? 4 : 0) | (a.R > 0 ? 8 : 0) | (a.S > 0 ? 16 | 32 : 0);
   p.M = (int)a.N;
   p.kb0 = (a.d + BK - 1) / BK;
   p.L = a.L;
@@ -1105,6 +1115,7 @@ cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
          make_map3(&p.tmB0, a.ws_o, a.G, a.d, a.S, hb) &&
          make_map3(&p.tmB2, a.ws_o, a.G, a.d, a.S, hb);
   if (!ok) return cudaErrorInvalidValue;
+  p.map_mask = 2 | 8 | 32 | (a.S > 0 ? 1 | 4 | 16 : 0);
   p.M = (int)a.N;
   p.S = a.S;
   p.G = a.G;
@@ -1125,6 +1136,7 @@ cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   bool ok = make_map(&p.tmA0, a.a, a.L, a.P, 1, BM) && make_map3(&p.tmB0, a.w0, a.L, a.F, a.R, SUB) &&
             make_map3(&p.tmB1, a.w1, a.L, a.F, a.R, SUB);
   if (!ok) return cudaErrorInvalidValue;
+  p.map_mask = 1 | 4 | 8;
   p.kb0 = (a.L + BK - 1) / BK;
   p.L = a.L;
   p.F = a.F;
@@ -1152,6 +1164,7 @@ cudaError_t umma_routed2(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   bool ok = make_map(&p.tmA0, a.a, a.F, a.P, 1, BM) && make_map3(&p.tmB0, a.w0, a.F, a.L, a.R, SUB) &&
             (p.bn == SUB || make_map3(&p.tmB1, a.w0, a.F, a.L, a.R, p.bn - SUB));
   if (!ok) return cudaErrorInvalidValue;
+  p.map_mask = 1 | 4 | (p.bn == SUB ? 0 : 8);
   p.kb0 = (a.F + BK - 1) / BK;
   p.L = a.L;
   p.F = a.F;
