@@ -16,7 +16,8 @@
 //                            softmax over the top-k logits: dl_i = p_i (dp_i - <p, dp>)
 //   z = W_down x             dW_down = dz^T x, dx = dz W_down + dl W_r + (shared terms)
 // Every contraction runs through one CUDA-core fp32 GEMM kernel with generic
-// strides (any operand layout, bf16 or fp32 operands), in three forms: plain;
+// strides (any operand layout; bf16 or fp32 operands, a template parameter
+// each), in three forms: plain;
 // grouped over the routed row tiles (one expert's weights per tile); grouped
 // along K per expert (weight gradients: a sum over that expert's rows).  No
 // atomics: every result is a fixed-order sum, so the gradients are
@@ -35,18 +36,19 @@ namespace lmoe {
 namespace {
 
 constexpr int GB = 128;  // output tile (rows and columns)
-constexpr int GK = 16;   // K per smem stage
+constexpr int GK = 8;    // K per smem stage
 constexpr int GT = 256;  // threads: 16 x 16, each 8 x 8 outputs
+constexpr int GE = GB * GK / GT;  // elements of each operand a thread loads per stage
+constexpr int kRmsRows = 32;  // tokens per partial sum of the RMSNorm weight gradient
+int rms_blocks(int64_t n) { return (int)((n + kRmsRows - 1) / kRmsRows); }
 
 struct GemmDesc {
   const void* A;
   int a_bf16;
   int64_t sam, sak;         // A(m, k) = A[m * sam + k * sak]
-  const int32_t* a_rows;    // optional row map of A (forms 0 and 1): A row = a_rows[m]
   const void* B;
   int b_bf16;
   int64_t sbk, sbn;         // B(k, n) = B[k * sbk + n * sbn]
-  const int32_t* b_rows;    // optional row map of B's K index (form 2)
   float* C;
   int64_t ldc;
   int M, N, K;
@@ -60,20 +62,31 @@ struct GemmDesc {
   int k_chunk;              // form 0 split along K: blockIdx.z takes [z k_chunk, (z+1) k_chunk)
 };
 
-__device__ __forceinline__ float ld_any(const void* p, int bf16, int64_t i) {
-  return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i])
-              : static_cast<const float*>(p)[i];
+// Operand loads keep the raw bits (a bf16 zero-extended to 32 bits) so that no
+// instruction waits on a load until the stage is written to smem, one stage
+// later: the loads stay in flight behind the current stage's FMAs.
+template <int BF>
+__device__ __forceinline__ uint32_t ld_raw(const void* p, int64_t i) {
+  if (BF) return (uint32_t)__ldg(static_cast<const unsigned short*>(p) + i);
+  return __float_as_uint(__ldg(static_cast<const float*>(p) + i));
+}
+template <int BF>
+__device__ __forceinline__ float from_raw(uint32_t r) {
+  return BF ? __uint_as_float(r << 16) : __uint_as_float(r);
 }
 
-// A 128 x 128 tile of C per CTA.  Each stage stages A [128 x 16] and B [16 x 128]
-// in smem as As[k][m], Bs[k][n] (the global reads run along whichever index is
-// contiguous); thread (tx, ty) then owns rows {4ty..4ty+3, 64+4ty..64+4ty+3}
+// A 128 x 128 tile of C per CTA (two CTAs per SM).  Each stage stages A
+// [128 x GK] and B [GK x 128] in smem as As[k][m], Bs[k][n] (the global reads
+// run along whichever index is contiguous), double-buffered so that one barrier
+// per stage suffices; thread (tx, ty) owns rows {4ty..4ty+3, 64+4ty..64+4ty+3}
 // and the same pattern of columns, read as float4 (conflict-free).
-__global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
+// ABF / BBF: A / B hold bf16 (else fp32).
+template <int ABF, int BBF>
+__global__ void __launch_bounds__(GT, 2) bwd_gemm_kernel(const GemmDesc g) {
   pdl_trigger();
   pdl_wait();
-  __shared__ __align__(16) float As[GK][GB + 4];
-  __shared__ __align__(16) float Bs[GK][GB + 4];
+  __shared__ __align__(16) float As[2][GK][GB + 4];
+  __shared__ __align__(16) float Bs[2][GK][GB + 4];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   int m_lo, m_hi, k_lo, k_hi;
   const void* Bp = g.B;
@@ -85,8 +98,8 @@ __global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
     const int4 tl = g.tiles[t];
     m_lo = tl.y;
     m_hi = tl.y + tl.z;
-    Bp = g.b_bf16 ? (const void*)(static_cast<const __nv_bfloat16*>(g.B) + tl.x * g.b_estride)
-                  : (const void*)(static_cast<const float*>(g.B) + tl.x * g.b_estride);
+    Bp = BBF ? (const void*)(static_cast<const __nv_bfloat16*>(g.B) + tl.x * g.b_estride)
+             : (const void*)(static_cast<const float*>(g.B) + tl.x * g.b_estride);
     k_lo = 0;
     k_hi = g.K;
   } else {
@@ -110,59 +123,52 @@ __global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-  // global -> registers for the stage starting at k0 (the next stage's loads
-  // are in flight while the current one is multiplied out of smem)
-  float ra[8], rb[8];
+  const bool a_kc = g.sak == 1, b_nc = g.sbn == 1;
+  uint32_t ra[GE], rb[GE];
+  // a K-contiguous operand is read as GK consecutive elements per row, else as
+  // 128 consecutive rows per k
   auto fetch = [&](int k0) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      int mi, ki;
-      if (g.sak == 1) { mi = (tid >> 4) + 16 * q; ki = tid & 15; }
-      else { mi = tid & 127; ki = (tid >> 7) + 2 * q; }
+    for (int q = 0; q < GE; ++q) {
+      const int mi = a_kc ? tid / GK + (GT / GK) * q : tid & 127;
+      const int ki = a_kc ? tid % GK : (tid >> 7) + 2 * q;
       const int m = m_lo + mi, k = k0 + ki;
-      float v = 0.0f;
-      if (m < m_hi && k < k_hi) {
-        int64_t row = m;
-        if (g.form != 2 && g.a_rows != nullptr) row = g.a_rows[m];
-        v = ld_any(g.A, g.a_bf16, row * g.sam + (int64_t)k * g.sak);
-      }
-      ra[q] = v;
+      ra[q] = (m < m_hi && k < k_hi) ? ld_raw<ABF>(g.A, (int64_t)m * g.sam + (int64_t)k * g.sak)
+                                     : 0u;
     }
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      int ki, ni;
-      if (g.sbn == 1) { ki = (tid >> 7) + 2 * q; ni = tid & 127; }
-      else { ki = tid & 15; ni = (tid >> 4) + 16 * q; }
+    for (int q = 0; q < GE; ++q) {
+      const int ki = b_nc ? (tid >> 7) + 2 * q : tid % GK;
+      const int ni = b_nc ? tid & 127 : tid / GK + (GT / GK) * q;
       const int k = k0 + ki, n = n0 + ni;
-      float v = 0.0f;
-      if (k < k_hi && n < g.N) {
-        int64_t krow = k;
-        if (g.form == 2 && g.b_rows != nullptr) krow = g.b_rows[k];
-        v = ld_any(Bp, g.b_bf16, krow * g.sbk + (int64_t)n * g.sbn);
-      }
-      rb[q] = v;
+      rb[q] = (k < k_hi && n < g.N) ? ld_raw<BBF>(Bp, (int64_t)k * g.sbk + (int64_t)n * g.sbn)
+                                    : 0u;
     }
   };
-  auto stash = [&]() {
+  auto stash = [&](int buf) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (g.sak == 1) As[tid & 15][(tid >> 4) + 16 * q] = ra[q];
-      else As[(tid >> 7) + 2 * q][tid & 127] = ra[q];
-      if (g.sbn == 1) Bs[(tid >> 7) + 2 * q][tid & 127] = rb[q];
-      else Bs[tid & 15][(tid >> 4) + 16 * q] = rb[q];
+    for (int q = 0; q < GE; ++q) {
+      if (a_kc) As[buf][tid % GK][tid / GK + (GT / GK) * q] = from_raw<ABF>(ra[q]);
+      else As[buf][(tid >> 7) + 2 * q][tid & 127] = from_raw<ABF>(ra[q]);
+      if (b_nc) Bs[buf][(tid >> 7) + 2 * q][tid & 127] = from_raw<BBF>(rb[q]);
+      else Bs[buf][tid % GK][tid / GK + (GT / GK) * q] = from_raw<BBF>(rb[q]);
     }
   };
-  if (k_lo < k_hi) fetch(k_lo);
+  if (k_lo < k_hi) {
+    fetch(k_lo);
+    stash(0);
+  }
+  __syncthreads();
+  int buf = 0;
   for (int k0 = k_lo; k0 < k_hi; k0 += GK) {
-    stash();
-    __syncthreads();
-    if (k0 + GK < k_hi) fetch(k0 + GK);
+    const bool more = k0 + GK < k_hi;
+    if (more) fetch(k0 + GK);  // in flight while this stage is multiplied out
 #pragma unroll
     for (int kk = 0; kk < GK; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -170,7 +176,10 @@ __global__ void __launch_bounds__(GT) bwd_gemm_kernel(const GemmDesc g) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
     }
+    // the other buffer was last read before the previous barrier
+    if (more) stash(buf ^ 1);
     __syncthreads();
+    buf ^= 1;
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -204,17 +213,55 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, int
 // Scratch for the K slices of plain GEMMs with few output tiles (floats).
 constexpr int64_t kSplitScratch = (int64_t)16 << 20;
 
+using GemmKernel = void (*)(GemmDesc);
+GemmKernel gemm_kernel(const GemmDesc& g) {
+  if (g.a_bf16) return g.b_bf16 ? bwd_gemm_kernel<1, 1> : bwd_gemm_kernel<1, 0>;
+  return g.b_bf16 ? bwd_gemm_kernel<0, 1> : bwd_gemm_kernel<0, 0>;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n = v > 0 ? v : 148;
+  }
+  return n;
+}
+
+// Number of K slices of a plain GEMM with `tiles` output tiles: the one that
+// best fills whole waves of resident CTAs (two per SM), each extra slice costing
+// a little (its partial block is written and summed once more).
+int choose_splits(int64_t tiles, int64_t MN, int K) {
+  const int64_t resident = 2 * (int64_t)sm_count();
+  if (tiles >= resident) return 1;
+  const int max_s = std::min(16, K / 128);  // slices of at least 128
+  int best = 1;
+  double best_score = (double)tiles / (double)resident;
+  for (int s = 2; s <= max_s; ++s) {
+    if ((int64_t)s * MN > kSplitScratch) break;
+    const int64_t ctas = tiles * s;
+    const int64_t waves = (ctas + resident - 1) / resident;
+    const double score = (double)ctas / (double)(waves * resident) - 0.03 * (s - 1);
+    if (score > best_score + 1e-9) {
+      best = s;
+      best_score = score;
+    }
+  }
+  return best;
+}
+
 cudaError_t gemm(const GemmDesc& g0, int max_tiles, int R, cudaStream_t st,
                  float* split_scratch = nullptr) {
   GemmDesc g = g0;
-  // A plain GEMM with fewer output tiles than SMs and a long K runs as
-  // K slices (a fixed number, summed in order by a second kernel).
+  const GemmKernel kern = gemm_kernel(g);
+  // A plain GEMM with too few output tiles to fill the GPU runs as K slices
+  // (a fixed number, summed in order by a second kernel).
   if (g.form == 0 && split_scratch != nullptr) {
     const int64_t tiles = (int64_t)((g.M + GB - 1) / GB) * ((g.N + GB - 1) / GB);
-    int splits = (int)std::min<int64_t>(16, (2 * 148 + tiles - 1) / tiles);
-    splits = std::min(splits, g.K / (8 * GK));
-    while (splits > 1 && (int64_t)splits * g.M * g.N > kSplitScratch) --splits;
-    if (tiles < 148 && splits > 1) {
+    int splits = choose_splits(tiles, (int64_t)g.M * g.N, g.K);
+    if (splits > 1) {
       const int chunk = ((g.K + splits - 1) / splits + GK - 1) / GK * GK;
       splits = (g.K + chunk - 1) / chunk;
       GemmDesc p = g;
@@ -223,7 +270,7 @@ cudaError_t gemm(const GemmDesc& g0, int max_tiles, int R, cudaStream_t st,
       p.accumulate = 0;
       p.k_chunk = chunk;
       count_launch();
-      cudaError_t e = launch_pdl(bwd_gemm_kernel,
+      cudaError_t e = launch_pdl(kern,
                                  dim3((unsigned)((g.M + GB - 1) / GB), (unsigned)((g.N + GB - 1) / GB),
                                       (unsigned)splits),
                                  dim3(GT), 0, st, 1, p);
@@ -242,7 +289,7 @@ cudaError_t gemm(const GemmDesc& g0, int max_tiles, int R, cudaStream_t st,
                    g.form == 2 ? (unsigned)R : 1u);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
   count_launch();
-  return launch_pdl(bwd_gemm_kernel, grid, dim3(GT), 0, st, 1, g);
+  return launch_pdl(kern, grid, dim3(GT), 0, st, 1, g);
 }
 
 __device__ __forceinline__ float sigmoid_b(float v) { return 1.0f / (1.0f + expf(-v)); }
@@ -333,15 +380,15 @@ __global__ void rms_dp_kernel(const float* __restrict__ u, const float* __restri
   }
 }
 
-// RMSNorm weight gradient: part[b][j] = sum over block b's tokens of duhat u r
-// (tokens in order), then drms[j] = sum_b part[b][j] (blocks in order).
+// RMSNorm weight gradient: part[b][j] = sum over block b's kRmsRows tokens of
+// duhat u r (tokens in order), then drms[j] = sum_b part[b][j] (blocks in order).
 __global__ void rms_dw_part_kernel(const float* __restrict__ u, const float* __restrict__ duhat,
                                    const float* __restrict__ rr, int64_t n, int L,
                                    float* __restrict__ part) {
   pdl_trigger();
   pdl_wait();
-  const int64_t t0 = (int64_t)blockIdx.x * kLossRows;
-  const int64_t t1 = min(n, t0 + kLossRows);
+  const int64_t t0 = (int64_t)blockIdx.x * kRmsRows;
+  const int64_t t1 = min(n, t0 + kRmsRows);
   for (int j = threadIdx.x; j < L; j += blockDim.x) {
     float acc = 0.0f;
     for (int64_t t = t0; t < t1; ++t) acc = fmaf(duhat[t * L + j] * u[t * L + j], rr[t], acc);
@@ -443,6 +490,7 @@ BwdLayout bwd_layout(const BwdDims& d) {
   L.block_counts = take((size_t)dispatch_blocks(P) * d.R * 4);
   L.tiles = take((size_t)L.max_tiles * 16);
   L.z = take((size_t)N * d.L * 4);
+  L.zp = take((size_t)P * d.L * 4);
   L.a = take((size_t)P * d.F * 4);
   L.c = take((size_t)P * d.F * 4);
   L.h = take((size_t)P * d.F * 4);
@@ -456,7 +504,7 @@ BwdLayout bwd_layout(const BwdDims& d) {
   L.rr = take((size_t)N * 4);
   L.dp = take((size_t)P * 4);
   L.dl = take((size_t)N * d.R * 4);
-  L.rms_part = take((size_t)loss_blocks(N) * d.L * 4);
+  L.rms_part = take((size_t)rms_blocks(N) * d.L * 4);
   L.ash = take((size_t)N * d.S * d.G * 4);
   L.csh = take((size_t)N * d.S * d.G * 4);
   L.hsh = take((size_t)N * d.S * d.G * 4);
@@ -483,7 +531,7 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   int32_t* perm = I32(L.perm);
   int32_t* inv = I32(L.inv);
   int4* tiles = reinterpret_cast<int4*>(base + L.tiles);
-  float *z = F32(L.z), *pa = F32(L.a), *pc = F32(L.c), *h = F32(L.h), *dh = F32(L.dh);
+  float *z = F32(L.z), *zp = F32(L.zp), *pa = F32(L.a), *pc = F32(L.c), *h = F32(L.h), *dh = F32(L.dh);
   float *o = F32(L.o), *dE = F32(L.dE), *u = F32(L.u), *uhat = F32(L.uhat);
   float *duhat = F32(L.duhat), *du = F32(L.du), *rr = F32(L.rr), *dp = F32(L.dp);
   float *dl = F32(L.dl), *rms_part = F32(L.rms_part);
@@ -505,10 +553,11 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   LMOE_STEP(launch_dispatch(ids, N, k, R, I32(L.counts), offsets, perm, inv, ds, st));
   // z = x W_down^T
   LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.w_down, bf, 1, D, z, Lt, (int)N, Lt, D), 0, R, st, split));
-  // a, c = z[perm] W_g,e^T, z[perm] W_u,e^T on the routed tiles
+  // zp = z[perm], the sorted rows; a, c = zp W_g,e^T, zp W_u,e^T on the routed tiles
+  LMOE_STEP(launch_gather_rows<float>(z, perm, P, Lt, zp, st));
   {
-    GemmDesc g = desc(z, 0, Lt, 1, a.w_g, bf, 1, Lt, pa, F, 0, F, Lt);
-    g.a_rows = perm; g.form = 1; g.tiles = tiles; g.n_tiles = n_mtiles; g.b_estride = FL;
+    GemmDesc g = desc(zp, 0, Lt, 1, a.w_g, bf, 1, Lt, pa, F, 0, F, Lt);
+    g.form = 1; g.tiles = tiles; g.n_tiles = n_mtiles; g.b_estride = FL;
     LMOE_STEP(gemm(g, L.max_tiles, R, st));
     g.B = a.w_u; g.C = pc;
     LMOE_STEP(gemm(g, L.max_tiles, R, st));
@@ -535,7 +584,7 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   LMOE_STEP(launch_pdl(rms_dp_kernel, dim3(warps_grid), dim3(256), 0, st, 1, (const float*)u,
                        (const float*)duhat, (const float*)rr, a.rms_weight, (const float*)o,
                        (const int32_t*)inv, (const float*)probs, N, k, Lt, du, dp, dE));
-  const int rb = loss_blocks(N);
+  const int rb = rms_blocks(N);
   count_launch();
   LMOE_STEP(launch_pdl(rms_dw_part_kernel, dim3(rb), dim3(256), 0, st, 1, (const float*)u,
                        (const float*)duhat, (const float*)rr, N, Lt, rms_part));
@@ -556,9 +605,9 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   count_launch();
   LMOE_STEP(launch_pdl(situ_bwd_kernel, dim3(grid_for(P * F, 256)), dim3(256), 0, st, 1, pa, pc,
                        (const float*)dh, P * F, d.beta1, d.beta2));
-  {  // dW_g,e = da^T z[perm], dW_u,e = dc^T z[perm]
-    GemmDesc g = desc(pa, 0, 1, F, z, 0, Lt, 1, a.g.dw_g, Lt, F, Lt, 0);
-    g.form = 2; g.offsets = offsets; g.c_estride = FL; g.b_rows = perm;
+  {  // dW_g,e = da^T zp, dW_u,e = dc^T zp
+    GemmDesc g = desc(pa, 0, 1, F, zp, 0, Lt, 1, a.g.dw_g, Lt, F, Lt, 0);
+    g.form = 2; g.offsets = offsets; g.c_estride = FL;
     LMOE_STEP(gemm(g, 0, R, st, split));
     g.A = pc; g.C = a.g.dw_u;
     LMOE_STEP(gemm(g, 0, R, st, split));

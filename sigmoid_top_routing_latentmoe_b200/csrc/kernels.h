@@ -115,7 +115,7 @@ struct BwdArgs {
   BwdGrads g;
 };
 struct BwdLayout {
-  size_t header, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, z, a, c, h,
+  size_t header, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, z, zp, a, c, h,
       dh, o, dE, u, uhat, duhat, du, rr, dp, dl, rms_part, ash, csh, hsh, dhsh, split, total;
   int ld_logits, max_tiles;
 };
