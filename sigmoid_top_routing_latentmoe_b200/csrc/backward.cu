@@ -230,23 +230,27 @@ int sm_count() {
   return n;
 }
 
-// Number of K slices of a plain GEMM with `tiles` output tiles: the one that
-// best fills whole waves of resident CTAs (two per SM), each extra slice costing
-// a little (its partial block is written and summed once more).
+// Number of K slices of a plain GEMM with `tiles` output tiles: the one with the
+// least estimated time, taken as the K steps of the busiest SM (its CTAs times
+// the slice length; a CTA alone on its SM runs at about 0.7 of the rate of two
+// sharing one, which hide each other's latencies) with 3 % more per extra slice
+// (its partial block is written and summed once more).
 int choose_splits(int64_t tiles, int64_t MN, int K) {
-  const int64_t resident = 2 * (int64_t)sm_count();
-  if (tiles >= resident) return 1;
+  const int64_t sms = sm_count();
+  if (tiles >= 2 * sms) return 1;
   const int max_s = std::min(16, K / 128);  // slices of at least 128
+  auto load = [&](int64_t ctas) {
+    const int64_t per_sm = (ctas + sms - 1) / sms;
+    return per_sm == 1 ? 1.43 : (double)per_sm;
+  };
   int best = 1;
-  double best_score = (double)tiles / (double)resident;
+  double best_cost = load(tiles) * K;
   for (int s = 2; s <= max_s; ++s) {
     if ((int64_t)s * MN > kSplitScratch) break;
-    const int64_t ctas = tiles * s;
-    const int64_t waves = (ctas + resident - 1) / resident;
-    const double score = (double)ctas / (double)(waves * resident) - 0.03 * (s - 1);
-    if (score > best_score + 1e-9) {
+    const double cost = load(tiles * s) * ((double)K / s) * (1.0 + 0.03 * (s - 1));
+    if (cost < best_cost * (1.0 - 1e-9)) {
       best = s;
-      best_score = score;
+      best_cost = cost;
     }
   }
   return best;
