@@ -42,8 +42,10 @@ def _run(wl, dev, dy):
     return g
 
 
+# The last two token counts make the weight-gradient contractions (K = tokens)
+# run as K slices with a shorter last slice, in the fp32 and the bf16 kernels.
 CASES = [("toy_fp32", 128, 0), ("halfb_uniform", 64, 0), ("halfb_skewed", 48, 0),
-         ("halfb_uniform", 40, 1), ("mid", 16, 0)]
+         ("halfb_uniform", 40, 1), ("mid", 16, 0), ("toy_fp32", 1000, 0), ("halfb_uniform", 300, 0)]
 
 
 @pytest.mark.parametrize("name,n,router", CASES)
