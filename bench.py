@@ -236,7 +236,7 @@ def run_memory_kernels(args, wl):
     """Routing, dispatch and combine called on their own through the C ABI at the
     workload's shapes (synthetic activations; no expert weights), each timed with
     CUDA events over --steps calls with L2 flushed in between.  Prints one JSON
-    line per entry point: algorithmic bytes per call (the survey's definitions),
+    line per entry point: algorithmic bytes per call (what the entry point must read and write),
     time, and the fraction of the roof max(bytes / HBM, FLOPs / bf16 peak)."""
     import torch
     import sigmoid_top_routing_latentmoe_b200 as lm

@@ -81,18 +81,18 @@ static lmoe_status cuda_fail(cudaError_t e, const char* where) {
 // ------------------------------------------------------------- device check
 static lmoe_status check_device() {
   static std::mutex mu;
-  static int verdict[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  static int arch_ok[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
   int dev = 0;
   LMOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(LMOE_EUNSUPPORTED, "device index %d", dev);
   std::lock_guard<std::mutex> lk(mu);
-  if (verdict[dev] == 0) {
+  if (arch_ok[dev] == 0) {
     int major = 0, minor = 0;
     LMOE_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "attr");
     LMOE_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "attr");
-    verdict[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    arch_ok[dev] = (major == 10 && minor == 0) ? 1 : 2;
   }
-  if (verdict[dev] != 1) return fail(LMOE_EUNSUPPORTED, "device %d is not sm_100 (B200)", dev);
+  if (arch_ok[dev] != 1) return fail(LMOE_EUNSUPPORTED, "device %d is not sm_100 (B200)", dev);
   return LMOE_OK;
 }
 

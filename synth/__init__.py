@@ -187,8 +187,8 @@ WORKLOADS = {
 
 
 def make_x_rows(wl: Workload, seed: int, rows, redraw_round: int = 0) -> np.ndarray:
-    """x rows for the given token indices.  Round 0 is the base draw; round r > 0
-    is an independent redraw of the same rows (stream "x.redraw.<r>")."""
+    """x rows for the given token indices.  Redraw 0 is the base draw; redraw r > 0
+    is an independent draw of the same rows (stream "x.redraw.<r>")."""
     rows = np.asarray(rows, dtype=np.int64)
     tag = "x" if redraw_round == 0 else f"x.redraw.{redraw_round}"
     out = np.empty((len(rows), wl.d), np.uint16 if wl.dtype == "bf16" else np.float32)
