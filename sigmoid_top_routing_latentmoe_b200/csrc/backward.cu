@@ -31,6 +31,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "launch.h"
+#include "umma_gemm.h"
 
 namespace lmoe {
 namespace {
@@ -545,10 +546,45 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   cudaError_t e;
 #define LMOE_STEP(call) do { if ((e = (call)) != cudaSuccess) return e; } while (0)
   // ---- forward, recomputed in fp32
-  // router logits, then the same top-k kernel as the forward
-  LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.w_router, bf, 1, D, logits, L.ld_logits, (int)N, R, D), 0,
-                 R, st, split));
-  LMOE_STEP(launch_route_topk(logits, L.ld_logits, a.bias, N, R, k, d.router, ids, probs, st));
+  // bf16 operands: the contractions with x (z, the router logits and the shared
+  // experts' gate / up pre-activations) are one tensor-core pass over x, exact
+  // products with fp32 sums, that also routes as the forward does (the same
+  // epilogue for R <= 32, else the same top-k kernel); fp32 operands: CUDA-core GEMMs
+  const int SG = S * G;
+  if (bf) {
+    XpassArgs xa{};
+    xa.x = static_cast<const __nv_bfloat16*>(a.x);
+    xa.N = N;
+    xa.d = D;
+    xa.w_down = static_cast<const __nv_bfloat16*>(a.w_down);
+    xa.L = Lt;
+    xa.w_router = static_cast<const __nv_bfloat16*>(a.w_router);
+    xa.R = R;
+    xa.ws_g = static_cast<const __nv_bfloat16*>(a.ws_g);
+    xa.ws_u = static_cast<const __nv_bfloat16*>(a.ws_u);
+    xa.S = S;
+    xa.G = G;
+    xa.z32 = z;
+    xa.logits = logits;
+    xa.logits_ld = L.ld_logits;
+    xa.a_sh = ash;
+    xa.c_sh = csh;
+    xa.beta1 = d.beta1;
+    xa.beta2 = d.beta2;
+    xa.router = d.router;
+    xa.bias = a.bias;
+    xa.ids = R <= 32 ? ids : nullptr;
+    xa.probs = probs;
+    xa.top_k = k;
+    LMOE_STEP(umma_xpass(xa, status, st));
+    if (R > 32)
+      LMOE_STEP(launch_route_topk(logits, L.ld_logits, a.bias, N, R, k, d.router, ids, probs, st));
+  } else {
+    // router logits, then the same top-k kernel as the forward
+    LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.w_router, bf, 1, D, logits, L.ld_logits, (int)N, R, D),
+                   0, R, st, split));
+    LMOE_STEP(launch_route_topk(logits, L.ld_logits, a.bias, N, R, k, d.router, ids, probs, st));
+  }
   DispatchScratch ds;
   ds.block_counts = I32(L.block_counts);
   ds.status = status;
@@ -556,7 +592,8 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   ds.tiles = tiles;
   LMOE_STEP(launch_dispatch(ids, N, k, R, I32(L.counts), offsets, perm, inv, ds, st));
   // z = x W_down^T
-  LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.w_down, bf, 1, D, z, Lt, (int)N, Lt, D), 0, R, st, split));
+  if (!bf)
+    LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.w_down, bf, 1, D, z, Lt, (int)N, Lt, D), 0, R, st, split));
   // zp = z[perm], the sorted rows; a, c = zp W_g,e^T, zp W_u,e^T on the routed tiles
   LMOE_STEP(launch_gather_rows<float>(z, perm, P, Lt, zp, st));
   {
@@ -638,9 +675,10 @@ cudaError_t run_backward(const BwdDims& d, const BwdArgs& a, void* ws, cudaStrea
   LMOE_STEP(gemm(desc(dl, 0, R, 1, a.w_router, bf, D, 1, a.g.dx, D, (int)N, D, R, 1), 0, R, st, split));
   // ---- step 4: shared experts, dE = dy
   if (S > 0) {
-    const int SG = S * G;
-    LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.ws_g, bf, 1, D, ash, SG, (int)N, SG, D), 0, R, st, split));
-    LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.ws_u, bf, 1, D, csh, SG, (int)N, SG, D), 0, R, st, split));
+    if (!bf) {
+      LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.ws_g, bf, 1, D, ash, SG, (int)N, SG, D), 0, R, st, split));
+      LMOE_STEP(gemm(desc(a.x, bf, D, 1, a.ws_u, bf, 1, D, csh, SG, (int)N, SG, D), 0, R, st, split));
+    }
     count_launch();
     LMOE_STEP(launch_pdl(situ_fwd_kernel, dim3(grid_for(N * SG, 256)), dim3(256), 0, st, 1,
                          (const float*)ash, (const float*)csh, N * SG, d.beta1, d.beta2, hsh));

@@ -65,7 +65,10 @@ struct Cfg {
   static constexpr int MT = BM * CG;                     // tile rows
 };
 
-enum Mode { XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3 };
+// XPASS_F32: the x-pass with fp32 z and shared gate / up pre-activations (no SiTU)
+enum Mode { XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3, XPASS_F32 = 4 };
+template <int MODE>
+constexpr bool is_xpass() { return MODE == XPASS || MODE == XPASS_F32; }
 enum Epi { EPI_Z = 1, EPI_SITU = 3, EPI_STORE = 4 };
 // B sub-tile sources of the x-pass: 0 W_down, 1 W_r, 2 W_g,sh, 3 W_u,sh,
 // 5 zero padding (a box outside W_r: loads zeros, stores nothing).
@@ -90,6 +93,7 @@ struct Params {
   void* out0;
   void* out1;
   void* out2;
+  void* out3;                          // XPASS_F32: up pre-activations (row stride ld2)
   int64_t ld0, ld1, ld2;
   const int4* tiles;
   const int32_t* n_mtiles;
@@ -365,7 +369,7 @@ __device__ __forceinline__ uint32_t instr_desc_cg(int n) {
 // ---------------------------------------------------------- tile decoding
 template <int MODE, int CG>
 __device__ __forceinline__ int total_tiles(const Params& p) {
-  if (MODE == XPASS || MODE == FINAL) return ((p.M + Cfg<CG>::MT - 1) / Cfg<CG>::MT) * p.n_tiles;
+  if (is_xpass<MODE>() || MODE == FINAL) return ((p.M + Cfg<CG>::MT - 1) / Cfg<CG>::MT) * p.n_tiles;
   return (*p.n_mtiles) * p.n_tiles;
 }
 
@@ -376,7 +380,7 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
   tl.srows[0] = tl.srows[1] = SUB;
   tl.scol[0] = 0;
   tl.scol[1] = SUB;
-  if (MODE == XPASS || MODE == FINAL) {
+  if (is_xpass<MODE>() || MODE == FINAL) {
     constexpr int MT = Cfg<CG>::MT;
     const int m_tiles = (p.M + MT - 1) / MT;
     const int mt = t % m_tiles, n = t / m_tiles;
@@ -545,9 +549,9 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
         else tma2_load_2d(a_dst, &p.tmA0, bar, kk, arow);
         for (int s = s0; s < s1; ++s) {
           int m = tl.bmap[s];
-          const bool pad = (MODE == XPASS && m == kPadMap);
+          const bool pad = (is_xpass<MODE>() && m == kPadMap);
           if (pad) m = 1;
-          const bool three_d = !(MODE == XPASS && m < 2);
+          const bool three_d = !(is_xpass<MODE>() && m < 2);
           load_b<CG>(b_dst + (CG == 1 ? s * SUB * BK * 2 : 0), bmap_ptr(p, m), three_d, bar, kk,
                      tl.brow[s], tl.bz[s]);
         }
@@ -674,6 +678,15 @@ __device__ __forceinline__ void warp_store_bf16(uint32_t stage, const uint32_t (
   warp_store_block(stage, w, reinterpret_cast<char*>(base), ld * 2, rows, cols * 2);
 }
 
+// 32 fp32 accumulator columns of the warp's rows (lane = row), cols <= 32 of them.
+__device__ __forceinline__ void warp_store_f32(uint32_t stage, const float (&v)[32], float* base,
+                                               int64_t ld, int rows, int cols) {
+  uint32_t w[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+  warp_store_block(stage, w, reinterpret_cast<char*>(base), ld * 4, rows, cols * 4);
+}
+
 // 64 fp32 accumulator columns -> 32 packed bf16x2 words.
 __device__ __forceinline__ void pack_block(const float (&a)[32], const float (&b)[32],
                                            uint32_t (&w)[32]) {
@@ -758,7 +771,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
       int width;
       __nv_bfloat16* out;
       int64_t ld;
-      if (MODE == XPASS) {
+      if (is_xpass<MODE>()) {
         width = p.G - (tl.ocol - (tl.ocol / p.G) * p.G);  // hidden units left in this expert
         out = static_cast<__nv_bfloat16*>(p.out2);
         ld = p.ld2;
@@ -768,7 +781,23 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         ld = p.ld0;
       }
       const int cols = min(64, width - half * 64);
-      if (cols > 0) {
+      if (MODE == XPASS_F32) {
+        if (cols > 0) {  // the pre-activations themselves, fp32
+          float g0[32], u0[32], g1[32], u1[32];
+          const uint32_t c0 = half * 64;
+          tc_ld32x4(tbase + c0, g0, tbase + SUB + c0, u0, tbase + c0 + 32, g1,
+                    tbase + SUB + c0 + 32, u1);
+          const int64_t at = grow0 * p.ld2 + tl.ocol + half * 64;
+          float* ga = static_cast<float*>(p.out2) + at;
+          float* ua = static_cast<float*>(p.out3) + at;
+          warp_store_f32(stage, g0, ga, p.ld2, rows, min(32, cols));
+          warp_store_f32(stage, u0, ua, p.ld2, rows, min(32, cols));
+          if (cols > 32) {
+            warp_store_f32(stage, g1, ga + 32, p.ld2, rows, cols - 32);
+            warp_store_f32(stage, u1, ua + 32, p.ld2, rows, cols - 32);
+          }
+        }
+      } else if (cols > 0) {
         uint32_t w[32];
         {
           float g0[32], u0[32], g1[32], u1[32];
@@ -783,7 +812,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         }
         warp_store_bf16(stage, w, out + grow0 * ld + tl.ocol + half * 64, ld, rows, cols);
       }
-    } else if (MODE == XPASS) {
+    } else if (is_xpass<MODE>()) {
 #pragma unroll 1
       for (int s = 0; s < tl.n_sub; ++s) {
         if (tl.bmap[s] == kPadMap) continue;
@@ -826,6 +855,12 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         if (cols <= 0) continue;
         float a[32], b[32];
         tc_ld32x2(tbase + tl.scol[s] + half * 64, a, tbase + tl.scol[s] + half * 64 + 32, b);
+        if (MODE == XPASS_F32) {
+          float* zf = static_cast<float*>(p.out0) + grow0 * p.ld0 + col;
+          warp_store_f32(stage, a, zf, p.ld0, rows, min(32, cols));
+          if (cols > 32) warp_store_f32(stage, b, zf + 32, p.ld0, rows, cols - 32);
+          continue;
+        }
         uint32_t w[32];
         pack_block(a, b, w);
         warp_store_bf16(stage, w, static_cast<__nv_bfloat16*>(p.out0) + grow0 * p.ld0 + col,
@@ -1079,11 +1114,13 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   p.n_zr_tiles = (p.nz_sub + p.nr_sub + 1) / 2;
   p.g_blocks = a.S > 0 ? (a.G + SUB - 1) / SUB : 0;
   p.n_tiles = p.n_zr_tiles + a.S * p.g_blocks;
-  p.out0 = a.z;
+  const bool f32 = a.z32 != nullptr;
+  p.out0 = f32 ? (void*)a.z32 : (void*)a.z;
   p.ld0 = a.L;
   p.out1 = a.logits;
   p.ld1 = a.logits_ld;
-  p.out2 = a.hsh;
+  p.out2 = f32 ? (void*)a.a_sh : (void*)a.hsh;
+  p.out3 = a.c_sh;
   p.ld2 = (int64_t)a.S * a.G;
   p.beta1 = a.beta1;
   p.beta2 = a.beta2;
@@ -1098,7 +1135,8 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   p.probs = a.probs;
   const int total = (int)((a.N + 2 * BM - 1) / (2 * BM)) * p.n_tiles;
   const int units = a.max_units > 0 ? std::min(a.max_units, num_sms() / 2) : num_sms() / 2;
-  return launch<XPASS, 2>(p, std::min(total, units), st);
+  return f32 ? launch<XPASS_F32, 2>(p, std::min(total, units), st)
+             : launch<XPASS, 2>(p, std::min(total, units), st);
 }
 
 cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {

@@ -26,6 +26,12 @@ struct XpassArgs {
   float* logits;
   int64_t logits_ld;
   __nv_bfloat16* hsh;
+  // z32 != nullptr: fp32 pre-activations instead (for the backward's recompute):
+  // z32 [N, L] = x W_down^T, a_sh / c_sh [N, S*G] = x W_g,sh^T / x W_u,sh^T, and
+  // no SiTU; z and hsh are not written.
+  float* z32;
+  float* a_sh;
+  float* c_sh;
   float beta1, beta2;
   // When R <= 32 and ids != nullptr the epilogue also routes each row (K3 top-k
   // + L1 normalisation with bias b, or router == 1: top-k of the logits +
