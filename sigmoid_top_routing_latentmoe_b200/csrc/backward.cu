@@ -220,14 +220,14 @@ GemmKernel gemm_kernel(const GemmDesc& g) {
   return g.b_bf16 ? bwd_gemm_kernel<0, 1> : bwd_gemm_kernel<0, 0>;
 }
 
+// SMs of the device current at the first call (B200: 148); thread-safe init.
 int sm_count() {
-  static int n = 0;
-  if (n == 0) {
+  static const int n = [] {
     int dev = 0, v = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    n = v > 0 ? v : 148;
-  }
+    return v > 0 ? v : 148;
+  }();
   return n;
 }
 
