@@ -15,6 +15,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import sys
@@ -86,15 +87,17 @@ def kernel_work(wl: synth.Workload, tag: str):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+    """Samples the SM clock and the clock-event (throttle) reasons with NVML
+    while a region runs, as fast as NVML answers (a sample every ~0.2 ms)."""
 
     REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
                "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
                "display_clock_setting": 0x100}
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, period_s: float = 2e-4):
         self.index = index
+        self.period_s = period_s
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
@@ -111,18 +114,22 @@ class ClockSampler:
         except Exception:
             self.ok = False
 
-    def _run(self):
+    def _sample(self):
         nv = self._nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-            except Exception:
-                pass
-            time.sleep(0.01)
+            self._sample()
+            time.sleep(self.period_s)
 
     def start(self):
         if self.ok:
+            self._sample()                       # at least one sample, taken at the start
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
 
@@ -130,9 +137,23 @@ class ClockSampler:
         if self._t is not None:
             self._stop.set()
             self._t.join()
+            self._sample()                       # and one at the end
         names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def pick_tensor_peak(peaks: dict, region_s: float, clk: dict):
+    """Denominator for a tensor-core kernel: the burst peak (cuBLAS timed alone)
+    when the timed region is short (< 1 s) or the SM clock stayed within 2 % of
+    its maximum; the sustained (power-capped) peak only for long regions that
+    ran at a lower clock."""
+    mhz, mx = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    at_max = mhz is not None and mx and mhz >= 0.98 * mx
+    if region_s < 1.0 or at_max:
+        why = "timed region %.3f s" % region_s if region_s < 1.0 else "SM clock within 2%% of max"
+        return peaks["bf16_tflops"], f"{peaks['source']} burst ({why})"
+    return peaks["bf16_tflops_sustained"], f"{peaks['source']} sustained (region {region_s:.1f} s)"
 
 
 def _dist():
@@ -158,6 +179,18 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first 'model name' line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(wl: synth.Workload, seed: int, budget_s: float = 12.0) -> dict:
     """The oracle as it stands on the host cores, on a bounded sample of the
     workload's tokens: first a small probe, then a sample sized to ~budget_s."""
@@ -179,7 +212,7 @@ def cpu_baseline(wl: synth.Workload, seed: int, budget_s: float = 12.0) -> dict:
     n = int(min(wl.n_tokens, max(probe_n, probe_n * budget_s / max(t_probe, 1e-6))))
     t = run(n)
     return {"value": n / t, "unit": "tokens/s", "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{n} of {wl.n_tokens} tokens of {wl.name}, fp64 C oracle, OpenMP over tokens, "
                       f"{t:.1f} s"}
 
@@ -225,6 +258,7 @@ def run_reference(args, wl):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(wl, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "cpu_model": cpu_model(),
                              "sample": f"{n_step} of {wl.n_tokens} tokens per step"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -482,7 +516,10 @@ def main():
     torch.cuda.synchronize()
     lm.launch_count(reset=True)
     k_ms, k_n = 0.0, 0
+    region0 = torch.cuda.Event(enable_timing=True)
+    region1 = torch.cuda.Event(enable_timing=True)
     clocks.start()
+    region0.record(stream)
     for i in range(args.steps):
         flush.zero_()                        # L2 flushed between timed steps (outside the events)
         starts[i].record(stream)
@@ -495,10 +532,12 @@ def main():
             ms_i, n_i = lm.profile_peek(prof_tag)
             k_ms += ms_i
             k_n += n_i
+    region1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
+    region_s = region0.elapsed_time(region1) / 1e3
     if graph is not None:
         launches = launches_per_step * args.steps
         lm.profile_read()
@@ -512,6 +551,33 @@ def main():
     value = world * wl.n_tokens / (ms_per_step / 1e3)
     if lm.get_device_status(ws) != lm.OK:
         raise SystemExit("device status not OK after the timed region")
+
+    # hot: the same K steps back to back, L2 not flushed (weights and x stay cached)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    h0.record(stream)
+    for _ in range(args.steps):
+        graph.replay() if graph is not None else step()
+    h1.record(stream)
+    torch.cuda.synchronize()
+    hot_ms = max_over_ranks(h0.elapsed_time(h1) / args.steps, dev)
+    # sustained clocks: >= 1 s of back-to-back replays, sampled like the timed region
+    n_sus = max(1, int(math.ceil(1.0 / max(ms_per_step / 1e3, 1e-6))))
+    sus = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sus.start()
+    s0.record(stream)
+    for _ in range(n_sus):
+        graph.replay() if graph is not None else step()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    clk_sus = sus.stop()
+    clk_sus["seconds"] = s0.elapsed_time(s1) / 1e3
+    clk_sus["steps"] = n_sus
+    clk_sus["ms_per_step"] = s0.elapsed_time(s1) / n_sus
 
     # per-kernel breakdown (a separate pass with every kernel bracketed by events)
     lm.profile_enable("*")
@@ -551,16 +617,15 @@ def main():
         k_avg_s = k_ms / k_n / 1e3
         if bound == "tensor":
             achieved = work / k_avg_s / 1e12
-            peak = peaks["bf16_tflops_sustained"]
+            peak, peak_source = pick_tensor_peak(peaks, region_s, clk)
             unit = "TFLOP/s"
         else:
             achieved = work / k_avg_s / 1e9
-            peak = peaks["hbm_gbs"]
+            peak, peak_source = peaks["hbm_gbs"], peaks["source"]
             unit = "GB/s"
         roof = {"kernel": prof_tag, "bound": bound, "achieved": achieved, "peak": peak,
                 "unit": unit, "frac": achieved / peak, "traffic": measured_traffic(wl, prof_tag),
-                "launch_us": k_avg_s * 1e6, "launches": k_n,
-                "peak_source": peaks["source"] + (" sustained" if bound == "tensor" else "")}
+                "launch_us": k_avg_s * 1e6, "launches": k_n, "peak_source": peak_source}
     else:
         roof = None
     # bytes the layer must read: the weights of the experts this input routes to
@@ -580,7 +645,10 @@ def main():
                            "roof_us": roof_s * 1e6, "frac": roof_s / (ms_per_step / 1e3),
                            "peak_source": peaks["source"] + " burst"},
         "roofline": roof,
-        "clocks": clk,
+        "clocks": dict(clk, region_s=region_s),
+        "clocks_sustained": clk_sus,
+        "hot": {"value": world * wl.n_tokens / (hot_ms / 1e3), "unit": "tokens/s",
+                "ms_per_step": hot_ms, "l2": "not flushed (back-to-back steps)"},
         "e2e": {"value": world * wl.n_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
         "gpu_launches": launches,

@@ -133,7 +133,8 @@ LMOE_API lmoe_status moe_route(const lmoe_dims* dims, const void* x, const void*
  *   perm_token [N*k]  int32 out: token of each sorted pair (expert-major,
  *                     tokens ascending inside an expert)
  *   inv_pair   [N, k] int32 out: sorted position of pair (t, slot)
- * Out-of-range ids set LMOE_EDEVICE in the status word (the pair is dropped). */
+ * An out-of-range id sets LMOE_EDEVICE in the status word; its pair is
+ * dropped (counted nowhere, no sorted slot) and its inv_pair entry is -1. */
 LMOE_API lmoe_status moe_dispatch(const lmoe_dims* dims, const int32_t* ids, int32_t* counts,
                          int32_t* offsets, int32_t* perm_token, int32_t* inv_pair, void* ws,
                          size_t ws_bytes, lmoe_stream stream);
@@ -171,7 +172,9 @@ LMOE_API lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const 
  * step 3 sum and step 5 RMSNorm): for each token t, in slot order,
  *   u_t = sum_i probs[t, i] * expert_out[inv_pair[t, i]]   (fp32, no atomics)
  *   u_normed_t = u_t / sqrt(mean(u_t^2) + eps) * rms_weight
- *   u_normed [N, l] out. */
+ *   u_normed [N, l] out.
+ * Slots whose inv_pair entry is negative (pairs the dispatch dropped) add
+ * nothing to u_t. */
 LMOE_API lmoe_status moe_combine(const lmoe_dims* dims, const void* expert_out, const int32_t* inv_pair,
                         const float* probs, const float* rms_weight, void* u_normed,
                         lmoe_stream stream);
@@ -246,7 +249,9 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
  * inspection after latent_moe_forward: offsets[0..6] = z [N,l], router logits
  * [N, ld] fp32, shared hidden units [N, S*G], RMSNorm(u) [N,l], routed expert
  * outputs [N*k, l], routed hidden units [N*k, F], sorted z rows [N*k, l];
- * offsets[7] = ld, the row stride (elements) of the logits. */
+ * offsets[7] = ld, the row stride (elements) of the logits.  With n >= 11
+ * also offsets[8..10] = the permutation the forward built: expert offsets
+ * [R+1], perm_token [N*k] and inv_pair [N,k], all int32.  n < 8 is EINVAL. */
 LMOE_API lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offsets, int32_t n);
 
 /* moe_dispatch without a workspace: the same permutation, bit for bit, for
@@ -264,7 +269,8 @@ LMOE_API lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offset
  *   The first call on a device looks the array's address up (make it before
  *   any stream capture).  All calls share the array and it keeps the last
  *   call's contents, so calls that overlap on the GPU race: serialise them.
- *   Out-of-range ids are dropped as in moe_dispatch but not reported.
+ *   Out-of-range ids are dropped as in moe_dispatch (inv_pair -1 for their
+ *   pairs) but not reported: the status word is private to this call.
  * Arguments and outputs as in moe_dispatch. */
 LMOE_API lmoe_status moe_dispatch_noalloc(const lmoe_dims* dims, const int32_t* ids,
                                           int32_t* counts, int32_t* offsets, int32_t* perm_token,

@@ -151,8 +151,8 @@ def alloc_workspace(dims: Dims, device="cuda", host: bool = False, stream=None) 
 
 def workspace_views(dims: Dims, ws: torch.Tensor) -> dict:
     """Views of the forward's intermediates inside ``ws`` (for inspection)."""
-    off = (ctypes.c_size_t * 8)()
-    _check(_lib.lmoe_workspace_layout(ctypes.byref(dims), off, 8), "lmoe_workspace_layout")
+    off = (ctypes.c_size_t * 11)()
+    _check(_lib.lmoe_workspace_layout(ctypes.byref(dims), off, 11), "lmoe_workspace_layout")
     act = torch.bfloat16 if dims.dtype == BF16 else torch.float32
     es = 2 if dims.dtype == BF16 else 4
     N, L, k, F = dims.n_tokens, dims.latent, dims.top_k, dims.ff_routed
@@ -165,7 +165,10 @@ def workspace_views(dims: Dims, ws: torch.Tensor) -> dict:
             "logits": view(off[1], N, off[7], torch.float32, 4)[:, :dims.n_routed],
             "hsh": view(off[2], N, SG, act, es), "uhat": view(off[3], N, L, act, es),
             "eo": view(off[4], N * k, L, act, es), "h": view(off[5], N * k, F, act, es),
-            "zp": view(off[6], N * k, L, act, es)}
+            "zp": view(off[6], N * k, L, act, es),
+            "offsets": view(off[8], 1, dims.n_routed + 1, torch.int32, 4)[0],
+            "perm": view(off[9], 1, N * k, torch.int32, 4)[0],
+            "inv": view(off[10], N, k, torch.int32, 4)}
 
 
 def workspace_init(ws: torch.Tensor, stream=None):

@@ -752,8 +752,9 @@ lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offsets, int32_
   LMOE_TRY(check_dims(dims));
   if (offsets == nullptr || n < 8) return fail(LMOE_EINVAL, "offsets needs 8 entries");
   const Layout L = layout(dims, false);
-  const size_t v[8] = {L.z, L.logits, L.hsh, L.uhat, L.eo, L.h, L.zp, (size_t)L.logits_ld};
-  for (int i = 0; i < 8; ++i) offsets[i] = v[i];
+  const size_t v[11] = {L.z,  L.logits, L.hsh, L.uhat,    L.eo,  L.h,
+                        L.zp, (size_t)L.logits_ld, L.offsets, L.perm, L.inv};
+  for (int i = 0; i < (n >= 11 ? 11 : 8); ++i) offsets[i] = v[i];
   return LMOE_OK;
 }
 

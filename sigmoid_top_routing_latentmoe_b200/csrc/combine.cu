@@ -32,6 +32,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ eo,
     for (int e = 0; e < E; ++e) u[v][e] = 0.0f;
   for (int i = 0; i < k; ++i) {
     const int64_t r = inv_pair[t * k + i];
+    if (r < 0) continue;  // a pair the dispatch dropped (out-of-range id)
     const float p = probs[t * k + i];
     const uint4* row = reinterpret_cast<const uint4*>(eo + r * L);
 #pragma unroll
@@ -96,8 +97,8 @@ __global__ void __launch_bounds__(128) combine_block_kernel(const T* __restrict_
     for (int j = 0; j < UNROLL; ++j) {
       const int i = i0 + j;
       pw[j] = 0.0f;
-      if (i < k) {
-        const int64_t r = inv_pair[t * k + i];
+      const int64_t r = i < k ? inv_pair[t * k + i] : -1;
+      if (r >= 0) {  // r < 0: a pair the dispatch dropped (out-of-range id)
         pw[j] = probs[t * k + i];
         const uint4* row = reinterpret_cast<const uint4*>(eo + r * L);
 #pragma unroll
@@ -105,11 +106,14 @@ __global__ void __launch_bounds__(128) combine_block_kernel(const T* __restrict_
           const int vi = v * 128 + threadIdx.x;
           raw[j][v] = vi < nvec ? row[vi] : make_uint4(0, 0, 0, 0);
         }
+      } else {
+#pragma unroll
+        for (int v = 0; v < VPT; ++v) raw[j][v] = make_uint4(0, 0, 0, 0);
       }
     }
 #pragma unroll
     for (int j = 0; j < UNROLL; ++j) {
-      if (i0 + j < k) {
+      if (i0 + j < k && pw[j] != 0.0f) {
 #pragma unroll
         for (int v = 0; v < VPT; ++v) {
           const T* el = reinterpret_cast<const T*>(&raw[j][v]);

@@ -265,6 +265,8 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
     if (valid && sub == 0) {
       perm_token[slot] = tok;
       inv_pair[p] = slot;
+    } else if (!valid && p < p1 && sub == 0) {
+      inv_pair[p] = -1;  // an out-of-range id: the pair takes no slot
     }
     if (z != nullptr) {
       // this sub-CTA's rows of the step: pairs p with p mod subs == sub

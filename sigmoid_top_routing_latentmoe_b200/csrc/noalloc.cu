@@ -19,8 +19,9 @@
 //   - All calls share the one array and it keeps the last call's contents.
 //     Two calls whose work overlaps on the GPU (different streams, or
 //     different host threads) race on it: serialise them.
-//   - Out-of-range ids are dropped, as in moe_dispatch, but they are not
-//     reported: the status word is private to this variant.
+//   - Out-of-range ids are dropped, as in moe_dispatch (their inv_pair
+//     entries are -1), but they are not reported: the status word is
+//     private to this variant.
 //   - Sizes whose scratch does not fit the array are rejected with
 //     LMOE_EUNSUPPORTED before anything is launched.
 #include <cstdarg>

@@ -31,6 +31,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -1036,27 +1037,44 @@ static bool make_map3(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+// Per-device launch state: the SM count, and whether each kernel instance has
+// had its dynamic shared-memory limit raised on that device (the attribute is
+// per device).  Guarded by one mutex; read once per device.
+constexpr int kMaxDevices = 64;
+static std::mutex g_dev_mu;
+static int g_sms[kMaxDevices] = {0};
+
+static int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  return dev;
+}
+
 static int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_sms[dev] == 0) {
+    int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+    g_sms[dev] = n > 0 ? n : 148;
   }
-  return n;
+  return g_sms[dev];
 }
 
 // grid: CTAs (CG = 1) or CTA pairs (CG = 2).
 template <int MODE, int CG>
 static cudaError_t launch(const Params& p, int grid, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(umma_gemm_kernel<MODE, CG>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg<CG>::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr = true;
+  static bool attr[kMaxDevices] = {false};
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!attr[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(umma_gemm_kernel<MODE, CG>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           Cfg<CG>::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      attr[dev] = true;
+    }
   }
   if (grid <= 0) return cudaSuccess;
   count_launch();

@@ -88,6 +88,10 @@ def test_forward_parity_full_size(name, sample):
     assert (np.sort(h_ids, axis=1)[:, 1:] != np.sort(h_ids, axis=1)[:, :-1]).all()
     np.testing.assert_allclose(host(probs).sum(1), 1.0, atol=1e-5)
     np.testing.assert_array_equal(host(counts), np.bincount(h_ids.reshape(-1), minlength=wl.n_routed))
+    # the permutation the forward built (in its workspace), on every pair
+    v = lm.workspace_views(ldims(wl), ws)
+    check_permutation_properties(h_ids, host(counts), host(v["offsets"]), host(v["perm"]),
+                                 host(v["inv"]), wl.n_routed)
     # deterministic: a second run is bit-identical
     y2, ids2, _, _, _ = _run_forward(wl, dev, ws)
     assert torch.equal(y, y2) and torch.equal(ids, ids2)

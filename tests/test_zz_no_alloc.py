@@ -58,3 +58,33 @@ def test_noalloc_rejects_sizes_beyond_its_array():
     st = lm._lib.moe_dispatch_noalloc(ctypes.byref(d), None, None, None, None, None, None)
     assert st == lm.EUNSUPPORTED
     assert "fixed array" in lm._lib.lmoe_last_error().decode()
+
+
+def test_noalloc_out_of_range_id_is_dropped_with_inv_pair_minus_one():
+    """A pair whose id is outside [0, R) takes no sorted slot: counts and offsets
+    cover the valid pairs only, its inv_pair entry is -1, and the valid pairs
+    are permuted as if it were absent (bit for bit against a stable argsort)."""
+    N, k, R = 300, 2, 16
+    ids_np = _ids(N, k, R, 3)
+    ids_np[17, 1] = R + 5                      # one out-of-range id
+    flat = ids_np.reshape(-1)
+    valid = (flat >= 0) & (flat < R)
+    counts_ref = np.bincount(flat[valid], minlength=R).astype(np.int32)
+    offsets_ref = np.concatenate([[0], np.cumsum(counts_ref)]).astype(np.int32)
+    order = np.flatnonzero(valid)[np.argsort(flat[valid], kind="stable")]
+    inv_ref = np.full(N * k, -1, dtype=np.int32)
+    inv_ref[order] = np.arange(order.size, dtype=np.int32)
+    perm_ref = (order // k).astype(np.int32)
+
+    ids = torch.from_numpy(ids_np).cuda()
+    dims = lm.make_dims(N, 64, 32, R, k, 0, 64, 64)
+    got = _outputs(N, k, R)
+    for t in got:
+        t.fill_(-7)
+    lm.moe_dispatch_noalloc(dims, ids, *got)
+    torch.cuda.synchronize()
+    counts, offsets, perm, inv = (t.cpu().numpy() for t in got)
+    np.testing.assert_array_equal(counts, counts_ref)
+    np.testing.assert_array_equal(offsets, offsets_ref)
+    np.testing.assert_array_equal(inv.reshape(-1), inv_ref)
+    np.testing.assert_array_equal(perm[:order.size], perm_ref)
