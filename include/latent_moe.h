@@ -239,7 +239,17 @@ LMOE_API lmoe_status latent_moe_backward(const lmoe_dims* dims, const lmoe_weigh
  * to the device, runs latent_moe_forward, copies y back to y_host [N, d] and
  * waits for the stream.  Weights and workspace are device memory.  The
  * workspace must be lmoe_workspace_size_host(dims) bytes (it also holds the
- * device copies of x and y). */
+ * device copies of x and y).
+ * The tokens may be processed in up to 8 chunks (tokens are independent, so y
+ * is bit-identical to one latent_moe_forward over all N): x chunks are copied
+ * in on a library-owned stream, each chunk's forward runs on `stream` once its
+ * x has landed, and its y is copied out on a second library-owned stream while
+ * the next chunk computes.  The chunk count comes from a cost model of copy
+ * time against forward time (one chunk when streaming the expert weights
+ * dominates).  The copy streams and their events are created on the first
+ * call on each device and kept until the process exits; the copies wait for
+ * work queued on `stream` before the call, and the call returns after all of
+ * it has finished.  Pinned host buffers are needed for the copies to overlap. */
 LMOE_API size_t lmoe_workspace_size_host(const lmoe_dims* dims);
 LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_weights* weights,
                                     const void* x_host, void* y_host, void* ws, size_t ws_bytes,

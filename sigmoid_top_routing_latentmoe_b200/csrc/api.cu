@@ -1,5 +1,7 @@
 // C ABI of the LatentMoE forward library: argument checks, workspace layout
 // and the launch sequence of each entry point.  See include/latent_moe.h.
+#include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -228,6 +230,18 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
   return LMOE_OK;
 }
 
+// The bf16 routed GEMMs run on CTA pairs over 256-row tiles when experts get
+// at least 64 sorted pairs on average (one tile then covers an expert's rows
+// with at most one pass over its weights per pair), and on single CTAs over
+// 128-row tiles for decode-like loads of a few rows per expert, where a
+// 256-row MMA would mostly multiply empty rows.
+static bool routed_pairs(const lmoe_dims* d) {
+  return d->dtype == LMOE_BF16 && d->n_tokens * (int64_t)d->top_k >= 64 * (int64_t)d->n_routed;
+}
+static int routed_tile_m(const lmoe_dims* d) {
+  return routed_pairs(d) ? kRoutedPairTileM : kTileM;
+}
+
 // z != nullptr: the scatter also writes the sorted rows of z to the workspace
 // (the A operand of the routed GEMMs).
 static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t* counts,
@@ -243,7 +257,7 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
   const int es = d->dtype == LMOE_BF16 ? 2 : 4;
   LMOE_CUDA(launch_dispatch(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm, inv,
                             s, st, z, z != nullptr ? at<char>(ws, L.zp) : nullptr,
-                            d->latent * es),
+                            d->latent * es, routed_tile_m(d)),
             "dispatch");
   return LMOE_OK;
 }
@@ -278,6 +292,7 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   RoutedArgs ra{};
   ra.P = P; ra.L = Lt; ra.F = F; ra.R = d->n_routed; ra.tiles = tiles; ra.n_mtiles = n_tiles;
   ra.max_tiles = L.max_tiles; ra.beta1 = d->beta1; ra.beta2 = d->beta2;
+  ra.pairs = routed_pairs(d) ? 1 : 0;
   {
     ProfScope ps("expert_gemm1", st);
     if (tc) {
@@ -462,6 +477,77 @@ static lmoe_status check_weights(const lmoe_dims* d, const lmoe_weights* w) {
   return LMOE_OK;
 }
 
+// ------------------------------------------------------ host entry point
+// latent_moe_forward_host pipelines chunks of tokens: the x chunks go to the
+// device on one copy stream, each chunk's forward runs on the caller's stream
+// as soon as its x has landed, and its y returns on a second copy stream while
+// the next chunk computes.  The two copy streams and the events are created
+// once per device and kept for the life of the process.
+constexpr int kMaxHostChunks = 8;
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t in_done[kMaxHostChunks] = {}, fwd_done[kMaxHostChunks] = {};
+};
+
+static lmoe_status host_pipe(HostPipe** out) {
+  static std::mutex mu;
+  static HostPipe pipes[64];
+  static bool ready[64] = {false};
+  int dev = 0;
+  LMOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LMOE_EUNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  HostPipe& p = pipes[dev];
+  if (!ready[dev]) {
+    const unsigned ef = cudaEventDisableTiming;
+    LMOE_CUDA(cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking), "copy stream");
+    LMOE_CUDA(cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking), "copy stream");
+    LMOE_CUDA(cudaEventCreateWithFlags(&p.start, ef), "event");
+    LMOE_CUDA(cudaEventCreateWithFlags(&p.done, ef), "event");
+    for (int c = 0; c < kMaxHostChunks; ++c) {
+      LMOE_CUDA(cudaEventCreateWithFlags(&p.in_done[c], ef), "event");
+      LMOE_CUDA(cudaEventCreateWithFlags(&p.fwd_done[c], ef), "event");
+    }
+    ready[dev] = true;
+  }
+  *out = &p;
+  return LMOE_OK;
+}
+
+// Number of token chunks for the host entry point, from a rough cost model:
+// per chunk of n tokens, the copies take n*d*es / 50 GB/s each way and the
+// forward max(FLOPs / 1 PFLOP/s, bytes / 6 TB/s) + 15 us of launch latency,
+// where every chunk streams the weights of the experts it selects again.  The
+// pipeline costs copy_in(first) + sum over chunks of the slowest stage +
+// copy_out(last); the count with the least estimate wins (1 when streaming the
+// weights dominates, as at widths where they are gigabytes).
+static int host_chunks(const lmoe_dims* d) {
+  const double N = (double)d->n_tokens, es = d->dtype == LMOE_BF16 ? 2.0 : 4.0;
+  const double D = d->d, L = d->latent, R = d->n_routed, k = d->top_k, F = d->ff_routed;
+  const double SG = (double)d->n_shared * (d->n_shared > 0 ? d->ff_shared : 0);
+  const double flops_tok = 2 * D * L + 2 * D * R + 6 * k * L * F + 6 * SG * D + 2 * L * D;
+  const double w_dense = (2 * D * L + D * R + 3 * SG * D) * es, w_expert = 3 * F * L * es;
+  const double copy_bw = 50e9, flop_rate = d->dtype == LMOE_BF16 ? 1.0e15 : 2.0e13,
+               hbm = 6.0e12, launch = 15e-6;
+  double best = 0.0;
+  int best_c = 1;
+  for (int c = 1; c <= kMaxHostChunks; ++c) {
+    const double n = std::ceil(N / c);
+    if (c > 1 && n < 256) break;
+    const double used = R * (1.0 - std::pow(1.0 - k / R, n));  // experts a chunk selects
+    const double t_copy = n * D * es / copy_bw;
+    const double t_fwd = std::max(n * flops_tok / flop_rate,
+                                  (w_dense + used * w_expert + 6 * n * D * es) / hbm) + launch;
+    const double t = 2 * t_copy + c * std::max(t_copy, t_fwd);
+    if (c == 1 || t < best) {
+      best = t;
+      best_c = c;
+    }
+  }
+  return best_c;
+}
+
 }  // namespace lmoe
 
 using namespace lmoe;
@@ -533,7 +619,7 @@ lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const int32_t* 
   cudaStream_t st = (cudaStream_t)stream;
   const Layout L = layout(dims, false);
   LMOE_CUDA(launch_build_tiles(offsets, dims->n_routed, &at<WsHeader>(ws, L.header)->n_mtiles,
-                               at<int4>(ws, L.tiles), st),
+                               at<int4>(ws, L.tiles), st, routed_tile_m(dims)),
             "build_tiles");
   if (dims->dtype == LMOE_BF16)
     return run_expert_ffn<__nv_bfloat16>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
@@ -733,17 +819,53 @@ lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_weights* w
   LMOE_TRY(check_device());
   cudaStream_t st = (cudaStream_t)stream;
   const Layout L = layout(dims, true);
-  const size_t bytes = (size_t)dims->n_tokens * dims->d * (dims->dtype == LMOE_BF16 ? 2 : 4);
-  void* xd = at<char>(ws, L.x);
-  void* yd = at<char>(ws, L.y);
-  if (bytes) LMOE_CUDA(cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st), "H2D x");
-  lmoe_status s;
-  if (dims->dtype == LMOE_BF16)
-    s = run_forward_tc(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st);
-  else
-    s = run_forward<float>(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st);
-  if (s != LMOE_OK) return s;
-  if (bytes) LMOE_CUDA(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st), "D2H y");
+  const int64_t N = dims->n_tokens;
+  const size_t row = (size_t)dims->d * (dims->dtype == LMOE_BF16 ? 2 : 4);
+  char* xd = at<char>(ws, L.x);
+  char* yd = at<char>(ws, L.y);
+  if (N == 0) {
+    LMOE_TRY(dims->dtype == LMOE_BF16
+                 ? run_forward_tc(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st)
+                 : run_forward<float>(dims, weights, xd, yd, nullptr, nullptr, nullptr, ws, st));
+    LMOE_CUDA(cudaStreamSynchronize(st), "sync");
+    return LMOE_OK;
+  }
+  HostPipe* hp = nullptr;
+  LMOE_TRY(host_pipe(&hp));
+  const int C = host_chunks(dims);
+  const int64_t per = (N + C - 1) / C;
+  // copies wait for whatever the caller queued on its stream before this call
+  LMOE_CUDA(cudaEventRecord(hp->start, st), "event");
+  LMOE_CUDA(cudaStreamWaitEvent(hp->in, hp->start, 0), "wait");
+  LMOE_CUDA(cudaStreamWaitEvent(hp->out, hp->start, 0), "wait");
+  for (int c = 0; c < C; ++c) {  // every chunk's x in flight first (the copy engine streams them)
+    const int64_t t0 = c * per, n = std::min<int64_t>(per, N - t0);
+    if (n <= 0) break;
+    LMOE_CUDA(cudaMemcpyAsync(xd + t0 * row, static_cast<const char*>(x_host) + t0 * row, n * row,
+                              cudaMemcpyHostToDevice, hp->in),
+              "H2D x");
+    LMOE_CUDA(cudaEventRecord(hp->in_done[c], hp->in), "event");
+  }
+  for (int c = 0; c < C; ++c) {  // chunk c's forward on the caller's stream, its y copied back
+    const int64_t t0 = c * per, n = std::min<int64_t>(per, N - t0);
+    if (n <= 0) break;
+    lmoe_dims dc = *dims;
+    dc.n_tokens = n;
+    LMOE_CUDA(cudaStreamWaitEvent(st, hp->in_done[c], 0), "wait");
+    lmoe_status s = dims->dtype == LMOE_BF16
+                        ? run_forward_tc(&dc, weights, xd + t0 * row, yd + t0 * row, nullptr,
+                                         nullptr, nullptr, ws, st)
+                        : run_forward<float>(&dc, weights, xd + t0 * row, yd + t0 * row, nullptr,
+                                             nullptr, nullptr, ws, st);
+    if (s != LMOE_OK) return s;
+    LMOE_CUDA(cudaEventRecord(hp->fwd_done[c], st), "event");
+    LMOE_CUDA(cudaStreamWaitEvent(hp->out, hp->fwd_done[c], 0), "wait");
+    LMOE_CUDA(cudaMemcpyAsync(static_cast<char*>(y_host) + t0 * row, yd + t0 * row, n * row,
+                              cudaMemcpyDeviceToHost, hp->out),
+              "D2H y");
+  }
+  LMOE_CUDA(cudaEventRecord(hp->done, hp->out), "event");
+  LMOE_CUDA(cudaStreamWaitEvent(st, hp->done, 0), "wait");
   LMOE_CUDA(cudaStreamSynchronize(st), "sync");
   return LMOE_OK;
 }

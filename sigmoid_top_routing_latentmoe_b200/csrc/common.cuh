@@ -13,8 +13,12 @@ namespace lmoe {
 constexpr int kStatusDevice = LMOE_EDEVICE;
 constexpr int kStatusTimeout = LMOE_ETIMEOUT;
 
-// Routed GEMMs are scheduled in row tiles of this many sorted pairs.
+// Routed GEMMs are scheduled in row tiles of at most this many sorted pairs
+// of one expert: kTileM for single-CTA tiles (and the CUDA-core kernels), and
+// kRoutedPairTileM for the tensor-core GEMMs on CTA pairs.  Workspaces size
+// the tile list for kTileM, which bounds both.
 constexpr int kTileM = 128;
+constexpr int kRoutedPairTileM = 256;
 
 // Header at the start of every workspace.
 struct WsHeader {

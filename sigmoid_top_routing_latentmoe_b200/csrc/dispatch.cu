@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
     const int32_t* __restrict__ chunk_counts, int prefixed, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ n_mtiles, int4* __restrict__ tiles,
     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair, int subs,
-    const uint4* __restrict__ z, uint4* __restrict__ zp, int row_vecs) {
+    const uint4* __restrict__ z, uint4* __restrict__ zp, int row_vecs, int tile_m) {
   pdl_trigger();
   pdl_wait();
   // [kWarps][R] per-warp counts, then first slots; [R] this chunk's first slot
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
         }
       }
     }
-    const int32_t nt = (tot + kTileM - 1) / kTileM;
+    const int32_t nt = (tot + tile_m - 1) / tile_m;
     const int32_t ex_c = block_exclusive_scan(tot, warp_sums, &totals[0]) + carry[0];
     const int32_t ex_t = block_exclusive_scan(nt, warp_sums, &totals[1]) + carry[1];
     if (e < R) {
@@ -211,8 +211,8 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
       if (cb == 0 && sub == 0) {
         if (!prefixed) counts[e] = tot;
         offsets[e] = ex_c;
-        for (int t = 0; t * kTileM < tot; ++t)
-          tiles[ex_t + t] = make_int4(e, ex_c + t * kTileM, min(kTileM, tot - t * kTileM), 0);
+        for (int t = 0; t * tile_m < tot; ++t)
+          tiles[ex_t + t] = make_int4(e, ex_c + t * tile_m, min(tile_m, tot - t * tile_m), 0);
       }
     }
     __syncthreads();
@@ -378,7 +378,7 @@ __global__ void check_bitmap_kernel(const uint32_t* __restrict__ bitmap, int64_t
 
 // Tile list from offsets alone (for moe_expert_ffn called on its own).  One
 // warp: each lane scans a contiguous run of experts.
-__global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int R,
+__global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int R, int tile_m,
                                    int32_t* __restrict__ n_mtiles, int4* __restrict__ tiles) {
   pdl_trigger();
   pdl_wait();
@@ -386,7 +386,7 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int R,
   const int per = (R + 31) / 32;
   const int e0 = min(R, lane * per), e1 = min(R, e0 + per);
   int32_t mine = 0;
-  for (int e = e0; e < e1; ++e) mine += (offsets[e + 1] - offsets[e] + kTileM - 1) / kTileM;
+  for (int e = e0; e < e1; ++e) mine += (offsets[e + 1] - offsets[e] + tile_m - 1) / tile_m;
   int32_t inc = mine;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -396,8 +396,8 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int R,
   int32_t t = inc - mine;
   for (int e = e0; e < e1; ++e) {
     const int32_t off = offsets[e], c = offsets[e + 1] - off;
-    for (int j = 0; j * kTileM < c; ++j)
-      tiles[t++] = make_int4(e, off + j * kTileM, min(kTileM, c - j * kTileM), 0);
+    for (int j = 0; j * tile_m < c; ++j)
+      tiles[t++] = make_int4(e, off + j * tile_m, min(tile_m, c - j * tile_m), 0);
   }
   if (lane == 31) *n_mtiles = inc;
 }
@@ -418,7 +418,7 @@ int dispatch_blocks(int64_t n_pairs) {
 cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
                             const DispatchScratch& s, cudaStream_t st, const void* z, void* zp,
-                            int row_bytes) {
+                            int row_bytes, int tile_m) {
   const int64_t n_pairs = n * k;
   const int64_t chunk = chunk_pairs(n_pairs);
   const int nb = dispatch_blocks(n_pairs);
@@ -449,7 +449,7 @@ cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t
   e = launch_pdl(scatter_kernel, dim3((unsigned)(nb * subs)), dim3(kThreads), smem, st, 1, ids,
                  n_pairs, chunk, k, R, nb, (const int32_t*)s.block_counts, prefixed, counts,
                  offsets, s.n_mtiles, s.tiles, perm_token, inv_pair, subs,
-                 static_cast<const uint4*>(z), static_cast<uint4*>(zp), row_bytes / 16);
+                 static_cast<const uint4*>(z), static_cast<uint4*>(zp), row_bytes / 16, tile_m);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -477,9 +477,10 @@ cudaError_t launch_check_dispatch(const int32_t* ids, int64_t n, int k, int R,
 }
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
-                               cudaStream_t st) {
+                               cudaStream_t st, int tile_m) {
   count_launch();
-  return launch_pdl(build_tiles_kernel, dim3(1), dim3(32), 0, st, 1, offsets, R, n_mtiles, tiles);
+  return launch_pdl(build_tiles_kernel, dim3(1), dim3(32), 0, st, 1, offsets, R, tile_m, n_mtiles,
+                    tiles);
 }
 
 template <typename T>

@@ -38,13 +38,14 @@ struct DispatchScratch {
 };
 int dispatch_blocks(int64_t n_pairs);
 // With z != nullptr the scatter also copies each pair's z row (row_bytes, a
-// multiple of 16) to its sorted slot in zp.
+// multiple of 16) to its sorted slot in zp.  The routed tile list holds tiles
+// of at most tile_m rows of one expert (kTileM or kRoutedPairTileM).
 cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
                             const DispatchScratch& s, cudaStream_t st, const void* z = nullptr,
-                            void* zp = nullptr, int row_bytes = 0);
+                            void* zp = nullptr, int row_bytes = 0, int tile_m = 128);
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
-                               cudaStream_t st);
+                               cudaStream_t st, int tile_m = 128);
 // Consistency check of a permutation (bitmap: (N k + 31) / 32 words of scratch).
 cudaError_t launch_check_dispatch(const int32_t* ids, int64_t n, int k, int R,
                                   const int32_t* counts, const int32_t* offsets,

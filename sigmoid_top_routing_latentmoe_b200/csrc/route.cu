@@ -175,6 +175,147 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   select_topk<VPL, SOFTMAX>(s, key, R, k, ids + t * k, probs + t * k);
 }
 
+// Order-preserving map of a float to uint32 (larger float -> larger code).
+__device__ __forceinline__ uint32_t orderable(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Bitonic sort of 64 keys held two per lane (element i = lane + 32 r),
+// descending: afterwards element i is the i-th largest.
+__device__ __forceinline__ void warp_sort64_desc(uint64_t (&v)[2]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride == 32) {  // partner is the lane's other element
+        const bool desc = (lane & size) == 0;  // size == 64 here: always descending
+        const uint64_t hi = v[0] > v[1] ? v[0] : v[1], lo = v[0] > v[1] ? v[1] : v[0];
+        v[0] = desc ? hi : lo;
+        v[1] = desc ? lo : hi;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int i = lane + 32 * r;
+          const uint64_t pv = __shfl_xor_sync(0xffffffffu, v[r], stride);
+          const bool desc = (i & size) == 0;
+          const bool keep_max = ((lane & stride) == 0) == desc;  // lower index of the pair
+          v[r] = keep_max ? (v[r] > pv ? v[r] : pv) : (v[r] < pv ? v[r] : pv);
+        }
+      }
+    }
+  }
+}
+
+// Bitonic sort of 32 floats across the warp, descending (lane i gets the
+// i-th largest).
+__device__ __forceinline__ float warp_sort32_desc(float v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const float pv = __shfl_xor_sync(0xffffffffu, v, stride);
+      const bool desc = (lane & size) == 0 || size == 32;
+      const bool keep_max = ((lane & stride) == 0) == desc;
+      v = keep_max ? fmaxf(v, pv) : fminf(v, pv);
+    }
+  }
+  return v;
+}
+
+// Top-k for many experts (R > 96, k <= 32), one warp per token, same result
+// as select_topk (keys descending, ties to the lower expert index; p from the
+// exact scores in slot order):
+//   1. the k-th largest of the 32 lane maxima is a lower bound Lk on the k-th
+//      largest key (k distinct keys reach it), so every key of the top k is
+//      >= Lk;
+//   2. the keys >= Lk (typically a few dozen of R) are compacted by ballot
+//      into a per-warp list of (orderable key << 32 | ~expert) codes;
+//   3. up to 64 candidates are sorted by a warp bitonic sort; the first k are
+//      the slots.  More than 64 candidates (clustered keys) take the k-round
+//      selection over all R keys instead.
+// The selection keys use the fast exponential and division (|error| ~1e-7,
+// far below the routing margins); the selected scores are recomputed exactly.
+template <int VPL, bool SOFTMAX>
+__global__ void __launch_bounds__(256) route_topk_wide_kernel(const float* __restrict__ logits,
+                                                              int64_t ld,
+                                                              const float* __restrict__ bias,
+                                                              int64_t n, int R, int k,
+                                                              int32_t* __restrict__ ids,
+                                                              float* __restrict__ probs) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ uint64_t cand[8][64];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= n) return;
+  const float* lr = logits + t * ld;
+  float key[VPL];
+  float lmax = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int e = j * 32 + lane;
+    float kv = -INFINITY;
+    if (e < R) {
+      const float l = lr[e];
+      kv = SOFTMAX ? l
+                   : __fdividef(1.0f, 1.0f + __expf(-l)) + (bias != nullptr ? bias[e] : 0.0f);
+    }
+    key[j] = kv;
+    lmax = fmaxf(lmax, kv);
+  }
+  const float lk = __shfl_sync(0xffffffffu, warp_sort32_desc(lmax), k - 1);
+  int mine = 0;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) mine += key[j] >= lk ? 1 : 0;
+  int incl = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total > 64) {  // clustered keys: the k-round selection over everything
+    float sv[VPL], kv2[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = j * 32 + lane;
+      const float l = e < R ? lr[e] : 0.0f;
+      sv[j] = SOFTMAX ? l : sigmoid_f(l);
+      kv2[j] = SOFTMAX ? l : sv[j] + ((bias != nullptr && e < R) ? bias[e] : 0.0f);
+    }
+    select_topk<VPL, SOFTMAX>(sv, kv2, R, k, ids + t * k, probs + t * k);
+    return;
+  }
+  int at = incl - mine;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    if (key[j] >= lk) {
+      const uint32_t e = (uint32_t)(j * 32 + lane);
+      cand[warp][at++] = ((uint64_t)orderable(key[j]) << 32) | (uint64_t)(0xffffffffu - e);
+    }
+  }
+  __syncwarp();
+  uint64_t v[2];
+  v[0] = lane < total ? cand[warp][lane] : 0ull;
+  v[1] = lane + 32 < total ? cand[warp][lane + 32] : 0ull;
+  warp_sort64_desc(v);
+  // lane i < k holds slot i
+  const int e = (int)(0xffffffffu - (uint32_t)(v[0] & 0xffffffffu));
+  float sc = 0.0f;
+  if (lane < k) sc = SOFTMAX ? lr[e] : sigmoid_f(lr[e]);
+  float den = 0.0f, first = __shfl_sync(0xffffffffu, sc, 0);
+  if (SOFTMAX && lane < k) sc = expf(sc - first);
+  for (int slot = 0; slot < k; ++slot) den += __shfl_sync(0xffffffffu, sc, slot);
+  if (!SOFTMAX) den = fmaxf(den, 1e-9f);
+  if (lane < k) {
+    ids[t * k + lane] = e;
+    probs[t * k + lane] = sc / den;
+  }
+}
+
 }  // namespace
 
 template <typename T>
@@ -208,6 +349,25 @@ cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias
   const int warps = 8;
   unsigned blocks = (unsigned)((n + warps - 1) / warps);
   int vpl = (R + 31) / 32;
+  if (vpl >= 4 && k <= 32) {
+#define LMOE_TOPK_WIDE(V)                                                                    \
+    if (vpl <= V) {                                                                          \
+      count_launch();                                                                        \
+      return router ? launch_pdl(route_topk_wide_kernel<V, true>, dim3(blocks),              \
+                                 dim3(warps * 32), 0, st, 1, logits, ld, bias, n, R, k, ids, \
+                                 probs)                                                      \
+                    : launch_pdl(route_topk_wide_kernel<V, false>, dim3(blocks),             \
+                                 dim3(warps * 32), 0, st, 1, logits, ld, bias, n, R, k, ids, \
+                                 probs);                                                     \
+    }
+    LMOE_TOPK_WIDE(4)
+    LMOE_TOPK_WIDE(8)
+    LMOE_TOPK_WIDE(16)
+    LMOE_TOPK_WIDE(32)
+    LMOE_TOPK_WIDE(64)
+    LMOE_TOPK_WIDE(128)
+#undef LMOE_TOPK_WIDE
+  }
 #define LMOE_TOPK_CASE(V)                                                                  \
   if (vpl <= V) {                                                                          \
     count_launch();                                                                        \

@@ -266,36 +266,43 @@ __device__ __forceinline__ uint32_t tanh_h2(uint32_t v) {
   asm("tanh.approx.f16x2 %0, %1;" : "=r"(r) : "r"(v));
   return r;
 }
+__device__ __forceinline__ uint32_t ex2_h2(uint32_t v) {
+  uint32_t r;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ __half2 mufu_h2(uint32_t (*f)(uint32_t), __half2 x) {
+  uint32_t u = f(*reinterpret_cast<const uint32_t*>(&x));
+  return *reinterpret_cast<__half2*>(&u);
+}
 // Two SiTU-GLU hidden units at once, packed to bf16x2:
 //   h = beta1 tanh(a/beta1) sigmoid(a) * beta2 tanh(c/beta2),
-//   sigmoid(a) = 1/2 + tanh(a/2)/2,
-// on f16x2 pairs: a and c are rounded to f16 once and scaled there, the three
-// tanh are one MUFU op per pair, the bounded factors (each |.| <= 1) and the
-// scale beta1*beta2 (|h| <= beta1*beta2) are multiplied in f16x2.  An |a| or
-// |c| beyond the f16 range rounds to infinity, where every tanh saturates to
-// its limit +-1 as it should.
+// on f16x2 pairs: a and c are rounded to f16 once and scaled there; the
+// sigmoid is formed without cancellation for negative a,
+//   sigmoid(a) = 2^(min(a, 0) log2 e) * (1/2 + tanh(|a|/2)/2),
+// (e^a sigmoid(-a) = sigmoid(a)), so its error stays relative over the whole
+// range; the three tanh and the exponential are one MUFU op per pair each,
+// and the bounded factors (|tanh| <= 1, sigmoid <= 1) are multiplied in f16x2
+// after the scale beta1*beta2 (|h| <= beta1*beta2).  An |a| or |c| beyond the
+// f16 range rounds to infinity, where every factor reaches its limit.
 struct SituConsts {
-  __half2 inv_b1, inv_b2, b12, half;
+  __half2 inv_b1, inv_b2, b12, half, log2e, zero;
 };
 __device__ __forceinline__ SituConsts situ_consts(const Params& p) {
   return {__float2half2_rn(p.inv_beta1), __float2half2_rn(p.inv_beta2),
-          __float2half2_rn(p.beta12), __float2half2_rn(0.5f)};
+          __float2half2_rn(p.beta12), __float2half2_rn(0.5f),
+          __float2half2_rn(1.4426950408889634f), __float2half2_rn(0.0f)};
 }
 __device__ __forceinline__ uint32_t situ2_bf16(float a0, float a1, float c0, float c1,
                                                const SituConsts& k) {
   const __half2 a = __floats2half2_rn(a0, a1);
   const __half2 c = __floats2half2_rn(c0, c1);
-  const __half2 x1 = __hmul2(a, k.inv_b1);
-  const __half2 x2 = __hmul2(a, k.half);
-  const __half2 x3 = __hmul2(c, k.inv_b2);
-  uint32_t u1 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x1));
-  uint32_t u2 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x2));
-  uint32_t u3 = tanh_h2(*reinterpret_cast<const uint32_t*>(&x3));
-  const __half2 t1 = *reinterpret_cast<__half2*>(&u1);
-  const __half2 t2 = *reinterpret_cast<__half2*>(&u2);
-  const __half2 t3 = *reinterpret_cast<__half2*>(&u3);
-  const __half2 sg = __hfma2(t2, k.half, k.half);
-  const __half2 h = __hmul2(__hmul2(__hmul2(t1, sg), t3), k.b12);
+  const __half2 t1 = mufu_h2(tanh_h2, __hmul2(a, k.inv_b1));
+  const __half2 t2 = mufu_h2(tanh_h2, __hmul2(__habs2(a), k.half));
+  const __half2 em = mufu_h2(ex2_h2, __hmul2(__hmin2(a, k.zero), k.log2e));
+  const __half2 t3 = mufu_h2(tanh_h2, __hmul2(c, k.inv_b2));
+  const __half2 sg = __hmul2(__hfma2(t2, k.half, k.half), em);
+  const __half2 h = __hmul2(__hmul2(__hmul2(t1, k.b12), sg), t3);
   const float2 f = __half22float2(h);
   __nv_bfloat162 o = __floats2bfloat162_rn(f.x, f.y);
   return *reinterpret_cast<uint32_t*>(&o);
@@ -446,6 +453,8 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
     tl.rows = e.z;
     tl.bz[0] = tl.bz[1] = e.x;
     if (MODE == ROUTED1) {
+      // gate rows of W_g,e and the matching up rows of W_u,e (CG = 2: CTA 0
+      // loads the gate half, CTA 1 the up half)
       tl.n_sub = 2;
       tl.bmap[0] = 0;
       tl.bmap[1] = 1;
@@ -453,6 +462,17 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
       tl.epi = EPI_SITU;
       tl.ocol = n * SUB;
       tl.ncols = 2 * SUB;
+    } else if (CG == 2) {  // ROUTED2 on a pair: each CTA loads half of the bn W_o rows
+      const int n0 = n * p.bn;
+      tl.n_sub = 2;
+      tl.bmap[0] = tl.bmap[1] = 0;
+      tl.srows[0] = tl.srows[1] = p.bn / 2;
+      tl.scol[1] = p.bn / 2;
+      tl.brow[0] = n0;
+      tl.brow[1] = n0 + p.bn / 2;
+      tl.ncols = p.bn;
+      tl.epi = EPI_STORE;
+      tl.ocol = n0;
     } else {
       const int n0 = n * p.bn;
       tl.n_sub = (p.bn > SUB && n0 + SUB < p.L) ? 2 : 1;
@@ -513,6 +533,11 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
   for (int t = unit; t < total && ok; t += n_units) {
     const Tile tl = decode_tile<MODE, CG>(p, t);
     const int arow = tl.m0 + (CG == 2 ? BM * (int)rank : 0);
+    // A routed pair tile of <= 128 rows has none in CTA 1: it loads no A there
+    // (its accumulator rows are never stored) and the leader expects fewer bytes.
+    const bool routed = MODE == ROUTED1 || MODE == ROUTED2;
+    const int a_ctas = (CG == 2 && routed && tl.rows <= BM) ? 1 : CG;
+    const bool load_a = (int)rank < a_ctas;
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.status)) {
         ok = false;
@@ -523,7 +548,7 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
       const uint32_t own_bar = smem_u32(&full[stage]);
       const uint32_t bar = CG == 1 ? own_bar : map_to_rank(own_bar, 0);
       if (CG == 1 || rank == 0)
-        mbar_expect_tx(own_bar, CG * A_BYTES + tl.ncols * BK * 2);
+        mbar_expect_tx(own_bar, a_ctas * A_BYTES + tl.ncols * BK * 2);
       // sub-tiles this CTA loads: all of them (CG = 1) or the one of its rank
       const int s0 = CG == 1 ? 0 : (int)rank;
       const int s1 = CG == 1 ? tl.n_sub : (int)rank + 1;
@@ -547,7 +572,7 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
       } else {
         const int kk = kb * BK;
         if (CG == 1) tma_load_2d(a_dst, &p.tmA0, bar, kk, arow);
-        else tma2_load_2d(a_dst, &p.tmA0, bar, kk, arow);
+        else if (load_a) tma2_load_2d(a_dst, &p.tmA0, bar, kk, arow);
         for (int s = s0; s < s1; ++s) {
           int m = tl.bmap[s];
           const bool pad = (is_xpass<MODE>() && m == kPadMap);
@@ -1208,19 +1233,31 @@ cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   p.inv_beta2 = 1.0f / a.beta2;
   p.beta12 = a.beta1 * a.beta2;
   const int64_t bound = (int64_t)a.max_tiles * p.n_tiles;
-  const int units = a.max_units > 0 ? std::min(a.max_units, num_sms()) : num_sms();
-  return launch<ROUTED1, 1>(p, (int)std::min<int64_t>(bound, units), st);
+  const int cg = a.pairs ? 2 : 1;
+  const int cap = num_sms() / cg;
+  const int units = a.max_units > 0 ? std::min(a.max_units, cap) : cap;
+  const int grid = (int)std::min<int64_t>(bound, units);
+  return a.pairs ? launch<ROUTED1, 2>(p, grid, st) : launch<ROUTED1, 1>(p, grid, st);
 }
 
 cudaError_t umma_routed2(const RoutedArgs& a, int32_t* status, cudaStream_t st) {
   if (a.P == 0) return cudaSuccess;
   Params p = base_params(status);
-  const int cap = a.max_units > 0 ? std::min(a.max_units, num_sms()) : num_sms();
-  p.bn = pick_bn((int)((a.P + BM - 1) / BM) + a.R / 2, a.L, cap);
-  bool ok = make_map(&p.tmA0, a.a, a.F, a.P, 1, BM) && make_map3(&p.tmB0, a.w0, a.F, a.L, a.R, SUB) &&
-            (p.bn == SUB || make_map3(&p.tmB1, a.w0, a.F, a.L, a.R, p.bn - SUB));
+  const int cg = a.pairs ? 2 : 1;
+  const int cap0 = num_sms() / cg;
+  const int cap = a.max_units > 0 ? std::min(a.max_units, cap0) : cap0;
+  const int tile_m = BM * cg;
+  p.bn = pick_bn((int)((a.P + tile_m - 1) / tile_m) + a.R / 2, a.L, cap);
+  bool ok = make_map(&p.tmA0, a.a, a.F, a.P, 1, BM);
+  if (a.pairs) {  // each CTA of a pair loads bn / 2 rows of W_o,e
+    ok = ok && make_map3(&p.tmB0, a.w0, a.F, a.L, a.R, p.bn / 2);
+    p.map_mask = 1 | 4;
+  } else {
+    ok = ok && make_map3(&p.tmB0, a.w0, a.F, a.L, a.R, SUB) &&
+         (p.bn == SUB || make_map3(&p.tmB1, a.w0, a.F, a.L, a.R, p.bn - SUB));
+    p.map_mask = 1 | 4 | (p.bn == SUB ? 0 : 8);
+  }
   if (!ok) return cudaErrorInvalidValue;
-  p.map_mask = 1 | 4 | (p.bn == SUB ? 0 : 8);
   p.kb0 = (a.F + BK - 1) / BK;
   p.L = a.L;
   p.F = a.F;
@@ -1231,8 +1268,8 @@ cudaError_t umma_routed2(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   p.tiles = a.tiles;
   p.n_mtiles = a.n_mtiles;
   const int64_t bound = (int64_t)a.max_tiles * p.n_tiles;
-  const int units = a.max_units > 0 ? std::min(a.max_units, num_sms()) : num_sms();
-  return launch<ROUTED2, 1>(p, (int)std::min<int64_t>(bound, units), st);
+  const int grid = (int)std::min<int64_t>(bound, cap);
+  return a.pairs ? launch<ROUTED2, 2>(p, grid, st) : launch<ROUTED2, 1>(p, grid, st);
 }
 
 }  // namespace lmoe

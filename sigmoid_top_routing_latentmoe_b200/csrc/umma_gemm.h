@@ -71,7 +71,11 @@ struct RoutedArgs {
   const int32_t* n_mtiles;
   int max_tiles;
   float beta1, beta2;
-  int max_units;  // at most this many CTAs (0: one per SM)
+  int max_units;  // at most this many CTAs or CTA pairs (0: one per SM / pair of SMs)
+  // 1: CTA pairs (tcgen05 cta_group::2) over row tiles of <= 256 sorted pairs;
+  // 0: single CTAs over row tiles of <= 128.  The tile list must have been
+  // built with the matching height (kRoutedPairTileM or kTileM).
+  int pairs;
 };
 
 cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st);

@@ -57,6 +57,8 @@ SMALL_CASES = [
     ("halfb_skewed", 520),
     ("mid", 136),
     ("k3_width", 40),             # 640 pairs over 896 experts: most experts empty
+    ("halfb_skewed", 1200),       # routed GEMMs on CTA pairs: 0 to ~900 rows per expert
+    ("mid", 520),                 # CTA pairs, ~65 rows per expert (second CTA's rows empty)
 ]
 
 
@@ -99,10 +101,18 @@ def test_forward_parity_full_size(name, sample):
 
 # ---------------------------------------------------------- entry points
 
-@pytest.mark.parametrize("name,n", [("halfb_uniform", 333), ("mid", 200), ("k3_width", 64),
-                                    ("toy_fp32", 128)])
-def test_route_parity(name, n):
-    wl = W[name].with_tokens(n)
+ROUTE_CASES = [("halfb_uniform", 333, {}), ("mid", 200, {}), ("k3_width", 64, {}),
+               ("toy_fp32", 128, {}),
+               # many experts: threshold + candidate sort, k up to its limit of 32
+               ("mid", 150, dict(n_routed=100, top_k=32)),
+               ("mid", 150, dict(n_routed=300, top_k=5)),
+               ("mid", 150, dict(n_routed=2000, top_k=24)),
+               ("k3_width", 96, dict(router=1))]
+
+
+@pytest.mark.parametrize("name,n,over", ROUTE_CASES)
+def test_route_parity(name, n, over):
+    wl = W[name].with_tokens(n).replace(**over)
     inp = prepare(wl)
     dev = device_inputs(inp)
     dims = ldims(wl)
@@ -115,6 +125,24 @@ def test_route_parity(name, n):
                                         synth.to_f32(inp["w_router"]), inp["expert_bias"])
     np.testing.assert_array_equal(host(ids), r_ids)
     np.testing.assert_allclose(host(probs), r_probs, atol=P_ABS_TOL, rtol=0)
+
+
+@pytest.mark.parametrize("R,k", [(896, 16), (128, 32)])
+def test_route_all_keys_equal(R, k):
+    """A zero router gives every expert the same key: more candidates than the
+    candidate sort takes, so the k-round selection decides; ties go to the lower
+    expert index (ids 0..k-1) and p = 1/k."""
+    N = 40
+    dims = lm.make_dims(N, 256, 128, R, k, 0, 64, 64)
+    ws = lm.alloc_workspace(dims)
+    x = torch.randn(N, 256, device="cuda").to(torch.bfloat16)
+    w_r = torch.zeros(R, 256, device="cuda", dtype=torch.bfloat16)
+    ids = torch.empty(N, k, dtype=torch.int32, device="cuda")
+    probs = torch.empty(N, k, dtype=torch.float32, device="cuda")
+    lm.moe_route(dims, x, w_r, None, ids, probs, ws)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(ids), np.tile(np.arange(k, dtype=np.int32), (N, 1)))
+    np.testing.assert_allclose(host(probs), 1.0 / k, rtol=0, atol=P_ABS_TOL)
 
 
 def _random_ids(N, k, R, seed, skew=False):
@@ -151,7 +179,7 @@ def test_dispatch_parity_bit_exact(N, k, R, skew):
 
 def test_dispatch_flags_out_of_range_ids():
     ids_np = _random_ids(64, 2, 8, seed=3)
-    ids_np[5, 1] = 8                       # out of range: reported, never written
+    ids_np[5, 1] = 8                       # out of range: reported, its pair dropped
     dims = lm.make_dims(64, 64, 32, 8, 2, 0, 64, 64)
     ws = lm.alloc_workspace(dims)
     counts = torch.empty(8, dtype=torch.int32, device="cuda")
@@ -160,12 +188,15 @@ def test_dispatch_flags_out_of_range_ids():
     inv = torch.full((64, 2), -7, dtype=torch.int32, device="cuda")
     lm.moe_dispatch(dims, to_device(ids_np, ""), counts, offsets, perm, inv, ws)
     assert lm.get_device_status(ws) == lm.EDEVICE
-    assert host(counts).sum() == 127 and host(inv)[5, 1] == -7
+    assert host(counts).sum() == 127 and host(inv)[5, 1] == -1   # dropped: no sorted slot
     assert lm.get_device_status(ws) == lm.OK   # reading clears the word
 
 
 @pytest.mark.parametrize("name,n", [("halfb_uniform", 257), ("halfb_skewed", 300), ("mid", 96),
-                                    ("toy_fp32", 128)])
+                                    ("toy_fp32", 128),
+                                    # >= 64 pairs per expert: routed GEMMs on CTA pairs over
+                                    # 256-row tiles (tails of <= 128 rows, and experts over 256)
+                                    ("halfb_uniform", 700), ("halfb_skewed", 1500), ("mid", 600)])
 def test_expert_ffn_and_combine_parity(name, n):
     """moe_expert_ffn on the oracle's z and permutation vs the oracle's SiTU per
     pair; moe_combine on the oracle's expert outputs vs RMSNorm of the p-weighted sum."""
