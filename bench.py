@@ -431,6 +431,9 @@ def main():
                     help="time moe_route / moe_dispatch / moe_combine on their own instead")
     ap.add_argument("--backward", action="store_true",
                     help="time latent_moe_backward instead of the forward")
+    ap.add_argument("--sustained-seconds", type=float, default=1.0,
+                    help="length of the back-to-back replay pass whose clocks are reported as "
+                         "clocks_sustained (0: no such pass, e.g. under a profiler)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     if args.memory_kernels:
@@ -538,20 +541,15 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     region_s = region0.elapsed_time(region1) / 1e3
-    if graph is not None:
-        launches = launches_per_step * args.steps
-        lm.profile_read()
-    else:
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_per_step = max_over_ranks(float(sum(step_ms)), dev) / args.steps
+
+    if graph is None:                        # eager: the timed region's own launches and events
         launches = lm.launch_count()
         lm.profile_enable(None)
         k_ms, k_n = lm.profile_read(prof_tag)
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(float(sum(step_ms)), dev)
-    ms_per_step = total_ms / args.steps
-    value = world * wl.n_tokens / (ms_per_step / 1e3)
-    if lm.get_device_status(ws) != lm.OK:
-        raise SystemExit("device status not OK after the timed region")
-
+    # (both passes replay the graph, whose event-record nodes use the profiling
+    # events: they run before lm.profile_read() releases those events)
     # hot: the same K steps back to back, L2 not flushed (weights and x stay cached)
     h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -563,7 +561,7 @@ def main():
     torch.cuda.synchronize()
     hot_ms = max_over_ranks(h0.elapsed_time(h1) / args.steps, dev)
     # sustained clocks: >= 1 s of back-to-back replays, sampled like the timed region
-    n_sus = max(1, int(math.ceil(1.0 / max(ms_per_step / 1e3, 1e-6))))
+    n_sus = int(math.ceil(args.sustained_seconds / max(ms_per_step / 1e3, 1e-6)))
     sus = ClockSampler(local)
     if world > 1:
         dist.barrier()
@@ -577,7 +575,14 @@ def main():
     clk_sus = sus.stop()
     clk_sus["seconds"] = s0.elapsed_time(s1) / 1e3
     clk_sus["steps"] = n_sus
-    clk_sus["ms_per_step"] = s0.elapsed_time(s1) / n_sus
+    clk_sus["ms_per_step"] = s0.elapsed_time(s1) / n_sus if n_sus else None
+    if graph is not None:
+        launches = launches_per_step * args.steps
+        lm.profile_read()
+    value = world * wl.n_tokens / (ms_per_step / 1e3)
+    if lm.get_device_status(ws) != lm.OK:
+        raise SystemExit("device status not OK after the timed region")
+
 
     # per-kernel breakdown (a separate pass with every kernel bracketed by events)
     lm.profile_enable("*")

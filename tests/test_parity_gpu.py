@@ -124,7 +124,10 @@ def test_route_parity(name, n, over):
     r_ids, r_probs, _, _ = oracle.route(odims(wl), synth.to_f32(inp["x"]),
                                         synth.to_f32(inp["w_router"]), inp["expert_bias"])
     np.testing.assert_array_equal(host(ids), r_ids)
-    np.testing.assert_allclose(host(probs), r_probs, atol=P_ABS_TOL, rtol=0)
+    # the softmax over the selected logits passes the logits' rounding through
+    # undamped (the K3 rule's sigmoid damps it by s(1 - s) <= 1/4): 1e-5 there
+    np.testing.assert_allclose(host(probs), r_probs, atol=P_ABS_TOL if wl.router == 0 else 1e-5,
+                               rtol=0)
 
 
 @pytest.mark.parametrize("R,k", [(896, 16), (128, 32)])
