@@ -599,6 +599,16 @@ def main():
             breakdown[tag] = round(ms / min(args.steps, 20) * 1e3, 2)
     lm.profile_read()
 
+    # host time to enqueue one eager forward (the call returns once everything is queued)
+    enq = []
+    for _ in range(5):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        step()
+        enq.append(time.perf_counter() - t0)
+    torch.cuda.synchronize()
+    host_enqueue_us = statistics.median(enq) * 1e6
+
     # end to end through the host entry point: pinned x in, y out, copies timed
     ws_h = lm.alloc_workspace(dims, device=dev, host=True)
     x_h = x.cpu().pin_memory()
@@ -657,6 +667,7 @@ def main():
         "e2e": {"value": world * wl.n_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
         "gpu_launches": launches,
+        "host_enqueue_us": host_enqueue_us,
         "kernel_us": breakdown,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -231,12 +231,16 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
 }
 
 // The bf16 routed GEMMs run on CTA pairs over 256-row tiles when experts get
-// at least 64 sorted pairs on average (one tile then covers an expert's rows
-// with at most one pass over its weights per pair), and on single CTAs over
-// 128-row tiles for decode-like loads of a few rows per expert, where a
-// 256-row MMA would mostly multiply empty rows.
+// 64 to 256 sorted pairs on average: one pair tile then covers an expert's
+// rows, so its weights stream once per output tile, half through each SM (at
+// the K3 width, 146 rows per expert: W_o GEMM 1093 -> 889 us).  With more rows
+// per expert (512 at the 0.5b shape, 2048 at the mid one) single CTAs over
+// 128-row tiles were faster (0.5b: 18 + 11 us against 27 + 17 us), and for
+// decode-like loads of a few rows a 256-row MMA would mostly multiply empty
+// rows.
 static bool routed_pairs(const lmoe_dims* d) {
-  return d->dtype == LMOE_BF16 && d->n_tokens * (int64_t)d->top_k >= 64 * (int64_t)d->n_routed;
+  const int64_t pairs = d->n_tokens * (int64_t)d->top_k, R = d->n_routed;
+  return d->dtype == LMOE_BF16 && pairs >= 64 * R && pairs <= 256 * R;
 }
 static int routed_tile_m(const lmoe_dims* d) {
   return routed_pairs(d) ? kRoutedPairTileM : kTileM;
@@ -321,6 +325,13 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   return LMOE_OK;
 }
 
+// The x-pass uses 256 x 512 tiles (no accumulator double-buffering, 1.33x the
+// FLOPs per streamed byte) when K = d is long enough for the main loop to hide
+// the epilogue: d >= 2048 (mid shape -8 %, K3 width -17 %; +3 % at d = 768).
+static int xpass_wide(const lmoe_dims* d) {
+  return d->d >= 2048 ? 1 : 0;
+}
+
 // bf16 forward on the tensor cores, one stream: the x-pass (z, routing and the
 // shared experts' hidden units), dispatch, the routed experts, combine +
 // RMSNorm, and one GEMM for y = shared + W_up RMSNorm(u).
@@ -358,6 +369,7 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
     a.z = z; a.logits = logits; a.logits_ld = L.logits_ld;
     a.hsh = hsh; a.beta1 = d->beta1; a.beta2 = d->beta2;
     a.bias = w->expert_bias; a.ids = ids; a.probs = probs; a.top_k = k; a.router = d->router;
+    a.wide = xpass_wide(d);
     ProfScope ps("xpass", st);
     LMOE_CUDA(umma_xpass(a, status, st), "x-pass (tcgen05)");
   }

@@ -30,7 +30,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ eo,
   for (int v = 0; v < VPL; ++v)
 #pragma unroll
     for (int e = 0; e < E; ++e) u[v][e] = 0.0f;
-  for (int i = 0; i < k; ++i) {
+#pragma unroll 4
+  for (int i = 0; i < k; ++i) {  // unrolled: up to four slots' rows in flight
     const int64_t r = inv_pair[t * k + i];
     if (r < 0) continue;  // a pair the dispatch dropped (out-of-range id)
     const float p = probs[t * k + i];

@@ -225,6 +225,46 @@ __device__ __forceinline__ float warp_sort32_desc(float v) {
   return v;
 }
 
+// k rounds of a warp argmax over keys held VPL per lane (expert e = j*32 +
+// lane; ties to the lower expert), the selected experts' scores read back from
+// the logits row lr: the same slots and weights as select_topk, without a
+// second array of scores in registers.
+template <int VPL, bool SOFTMAX>
+__device__ __noinline__ void select_topk_keys(float (&key)[VPL], const float* __restrict__ lr, int R,
+                                              int k, int32_t* ids_row, float* probs_row) {
+  const int lane = threadIdx.x & 31;
+  float den = 0.0f, first = 0.0f;
+  for (int slot = 0; slot < k; ++slot) {
+    float bk = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = j * 32 + lane;
+      if (e < R && (key[j] > bk || (key[j] == bk && e < bi))) {
+        bk = key[j];
+        bi = e;
+      }
+    }
+    warp_argmax(bk, bi);
+#pragma unroll
+    for (int j = 0; j < VPL; ++j)
+      if (j * 32 + lane == bi) key[j] = -INFINITY;
+    float sc = SOFTMAX ? lr[bi] : sigmoid_f(lr[bi]);
+    if (SOFTMAX) {
+      if (slot == 0) first = sc;
+      sc = expf(sc - first);
+    }
+    den += sc;
+    if (lane == 0) {
+      ids_row[slot] = bi;
+      probs_row[slot] = sc;  // divided by the sum below
+    }
+  }
+  if (!SOFTMAX) den = fmaxf(den, 1e-9f);
+  __syncwarp();
+  for (int slot = lane; slot < k; slot += 32) probs_row[slot] = probs_row[slot] / den;
+}
+
 // Top-k for many experts (R > 96, k <= 32), one warp per token, same result
 // as select_topk (keys descending, ties to the lower expert index; p from the
 // exact scores in slot order):
@@ -239,7 +279,7 @@ __device__ __forceinline__ float warp_sort32_desc(float v) {
 // The selection keys use the fast exponential and division (|error| ~1e-7,
 // far below the routing margins); the selected scores are recomputed exactly.
 template <int VPL, bool SOFTMAX>
-__global__ void __launch_bounds__(256) route_topk_wide_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(256, VPL <= 32 ? 4 : 1) route_topk_wide_kernel(const float* __restrict__ logits,
                                                               int64_t ld,
                                                               const float* __restrict__ bias,
                                                               int64_t n, int R, int k,
@@ -278,15 +318,16 @@ __global__ void __launch_bounds__(256) route_topk_wide_kernel(const float* __res
   }
   const int total = __shfl_sync(0xffffffffu, incl, 31);
   if (total > 64) {  // clustered keys: the k-round selection over everything
-    float sv[VPL], kv2[VPL];
+    // exact keys (the fast ones above may differ in the last bits)
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
       const int e = j * 32 + lane;
-      const float l = e < R ? lr[e] : 0.0f;
-      sv[j] = SOFTMAX ? l : sigmoid_f(l);
-      kv2[j] = SOFTMAX ? l : sv[j] + ((bias != nullptr && e < R) ? bias[e] : 0.0f);
+      if (e < R) {
+        const float l = lr[e];
+        key[j] = SOFTMAX ? l : sigmoid_f(l) + (bias != nullptr ? bias[e] : 0.0f);
+      }
     }
-    select_topk<VPL, SOFTMAX>(sv, kv2, R, k, ids + t * k, probs + t * k);
+    select_topk_keys<VPL, SOFTMAX>(key, lr, R, k, ids + t * k, probs + t * k);
     return;
   }
   int at = incl - mine;

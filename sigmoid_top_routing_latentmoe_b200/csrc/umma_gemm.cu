@@ -30,6 +30,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -51,25 +52,37 @@ constexpr int EPI_WARPS = 8;    // two warps per TMEM lane quarter, splitting th
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint64_t WAIT_CAP_NS = 2000000000ull;
 
+// XPASS_F32: the x-pass with fp32 z and shared gate / up pre-activations (no SiTU)
+// XPASS_WIDE: the x-pass on 256 x 512 pair tiles (see Cfg)
+enum Mode { XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3, XPASS_F32 = 4, XPASS_WIDE = 5 };
+template <int MODE>
+constexpr bool is_xpass() { return MODE == XPASS || MODE == XPASS_F32 || MODE == XPASS_WIDE; }
+
 // CG = 1: one CTA computes a 128-row tile and loads every B sub-tile.
 // CG = 2: a CTA pair (cluster of 2) computes a 256-row tile with
 //         tcgen05.mma.cta_group::2; each CTA loads its own 128 rows of A and
 //         one of the two B sub-tiles (half of N), so each SM streams half of
 //         B per FLOP.
-template <int CG>
+// W = 2 (XPASS_WIDE, pairs only): each K step issues two N = 256 MMAs into
+//         the 512 TMEM columns, a 256 x 512 tile; each CTA loads 128 rows of A
+//         and two 128-row B sub-tiles per stage, so every byte an SM streams
+//         feeds 1.33x the FLOPs of a 256 x 256 tile.  The accumulator takes
+//         all of TMEM (one buffer): the next tile's MMAs wait for the
+//         epilogue, while the TMA ring keeps filling.
+template <int MODE, int CG>
 struct Cfg {
-  static constexpr int B_BYTES = (CG == 1 ? 2 : 1) * SUB * BK * 2;
+  static constexpr int W = MODE == XPASS_WIDE ? 2 : 1;
+  static constexpr int B_BYTES = (CG == 1 ? 2 : W) * SUB * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB or 32 KB
-  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr int STAGES = CG == 1 ? 4 : (W == 2 ? 4 : 6);
   static constexpr int EPI_STAGE = 32 * 128;             // per epilogue warp: 32 rows x 128 B
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * EPI_STAGE + 1024;
   static constexpr int MT = BM * CG;                     // tile rows
+  static constexpr int NACC = W == 2 ? 1 : 2;            // accumulator buffers in TMEM
+  static constexpr int ACC_STRIDE = TMEM_COLS / NACC;    // columns per buffer
 };
+static_assert(Cfg<XPASS_WIDE, 2>::SMEM_BYTES <= 232448, "wide x-pass exceeds shared memory");
 
-// XPASS_F32: the x-pass with fp32 z and shared gate / up pre-activations (no SiTU)
-enum Mode { XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3, XPASS_F32 = 4 };
-template <int MODE>
-constexpr bool is_xpass() { return MODE == XPASS || MODE == XPASS_F32; }
 enum Epi { EPI_Z = 1, EPI_SITU = 3, EPI_STORE = 4 };
 // B sub-tile sources of the x-pass: 0 W_down, 1 W_r, 2 W_g,sh, 3 W_u,sh,
 // 5 zero padding (a box outside W_r: loads zeros, stores nothing).
@@ -102,14 +115,17 @@ struct Params {
   float beta1, beta2, inv_beta1, inv_beta2, beta12;
 };
 
-struct Tile {
+template <int NS>  // at most NS B sub-tiles
+struct TileT {
   int m0, rows, n_sub;
-  int ncols;                    // MMA N: sum of the sub-tiles' rows
-  int bmap[2], brow[2], bz[2];  // B source map, first row, expert (3-D maps)
-  int srows[2];                 // rows of each sub-tile load
-  int scol[2];                  // accumulator / output column of each sub-tile
+  int ncols;                       // MMA N: sum of the sub-tiles' rows
+  int bmap[NS], brow[NS], bz[NS];  // B source map, first row, expert (3-D maps)
+  int srows[NS];                   // rows of each sub-tile load
+  int scol[NS];                    // accumulator / output column of each sub-tile
   int epi, ocol;
 };
+template <int MODE, int CG>
+using Tile = TileT<2 * Cfg<MODE, CG>::W>;
 
 // ------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -231,6 +247,28 @@ __device__ __forceinline__ void tc_ld32x2(uint32_t ta, float (&va)[32], uint32_t
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
+    va[i] = __uint_as_float(r[i]);
+    vb[i] = __uint_as_float(q[i]);
+  }
+}
+// Two 16-column TMEM loads in flight before one wait.
+__device__ __forceinline__ void tc_ld16x2(uint32_t ta, float (&va)[16], uint32_t tb,
+                                          float (&vb)[16]) {
+  uint32_t r[16], q[16];
+#define LMOE_TC_LD16(ADDR, R)                                                                   \
+  asm volatile(                                                                                 \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "                                                 \
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"                         \
+      : "=r"(R[0]), "=r"(R[1]), "=r"(R[2]), "=r"(R[3]), "=r"(R[4]), "=r"(R[5]), "=r"(R[6]),     \
+        "=r"(R[7]), "=r"(R[8]), "=r"(R[9]), "=r"(R[10]), "=r"(R[11]), "=r"(R[12]),             \
+        "=r"(R[13]), "=r"(R[14]), "=r"(R[15])                                                   \
+      : "r"(ADDR))
+  LMOE_TC_LD16(ta, r);
+  LMOE_TC_LD16(tb, q);
+#undef LMOE_TC_LD16
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
     va[i] = __uint_as_float(r[i]);
     vb[i] = __uint_as_float(q[i]);
   }
@@ -377,19 +415,21 @@ __device__ __forceinline__ uint32_t instr_desc_cg(int n) {
 // ---------------------------------------------------------- tile decoding
 template <int MODE, int CG>
 __device__ __forceinline__ int total_tiles(const Params& p) {
-  if (is_xpass<MODE>() || MODE == FINAL) return ((p.M + Cfg<CG>::MT - 1) / Cfg<CG>::MT) * p.n_tiles;
+  if (is_xpass<MODE>() || MODE == FINAL) return ((p.M + Cfg<MODE, CG>::MT - 1) / Cfg<MODE, CG>::MT) * p.n_tiles;
   return (*p.n_mtiles) * p.n_tiles;
 }
 
 template <int MODE, int CG>
-__device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
-  Tile tl;
-  tl.bz[0] = tl.bz[1] = 0;
-  tl.srows[0] = tl.srows[1] = SUB;
-  tl.scol[0] = 0;
-  tl.scol[1] = SUB;
+__device__ __forceinline__ Tile<MODE, CG> decode_tile(const Params& p, int t) {
+  Tile<MODE, CG> tl;
+#pragma unroll
+  for (int s = 0; s < 2 * Cfg<MODE, CG>::W; ++s) {
+    tl.bz[s] = 0;
+    tl.srows[s] = SUB;
+    tl.scol[s] = s * SUB;
+  }
   if (is_xpass<MODE>() || MODE == FINAL) {
-    constexpr int MT = Cfg<CG>::MT;
+    constexpr int MT = Cfg<MODE, CG>::MT;
     const int m_tiles = (p.M + MT - 1) / MT;
     const int mt = t % m_tiles, n = t / m_tiles;
     tl.m0 = mt * MT;
@@ -414,9 +454,11 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
       tl.epi = EPI_STORE;
       tl.ocol = n0;
     } else if (n < p.n_zr_tiles) {
+      // 2 W sub-tiles of z / router rows (sub-tile s: accumulator columns [128 s, 128 s + 128))
+      constexpr int NS = 2 * Cfg<MODE, CG>::W;
       tl.n_sub = 0;
-      for (int s = 0; s < 2; ++s) {
-        const int idx = 2 * n + s;
+      for (int s = 0; s < NS; ++s) {
+        const int idx = NS * n + s;
         if (idx < p.nz_sub) {
           tl.bmap[s] = 0;
           tl.brow[s] = idx * SUB;
@@ -430,21 +472,26 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
           tl.brow[s] = p.nr_sub * SUB;
         }
       }
-      if (CG == 2) tl.n_sub = 2;
+      if (CG == 2) tl.n_sub = NS;
       tl.epi = EPI_Z;  // per sub-tile: z, routing or padding, resolved in the epilogue
       tl.ocol = 0;
       tl.ncols = tl.n_sub * SUB;
     } else {
+      // W blocks of 128 hidden units of shared expert j: sub-tile 2b holds the gate
+      // rows of block b, sub-tile 2b + 1 the matching up rows
+      constexpr int W = Cfg<MODE, CG>::W;
       const int q = n - p.n_zr_tiles;
       const int j = q / p.g_blocks, fb = q % p.g_blocks;
-      tl.n_sub = 2;
-      tl.bmap[0] = 2;
-      tl.bmap[1] = 3;
-      tl.brow[0] = tl.brow[1] = fb * SUB;
-      tl.bz[0] = tl.bz[1] = j;
+      tl.n_sub = 2 * W;
+#pragma unroll
+      for (int sb = 0; sb < 2 * W; ++sb) {
+        tl.bmap[sb] = (sb & 1) ? 3 : 2;
+        tl.brow[sb] = fb * W * SUB + (sb >> 1) * SUB;
+        tl.bz[sb] = j;
+      }
       tl.epi = EPI_SITU;
-      tl.ocol = j * p.G + fb * SUB;
-      tl.ncols = 2 * SUB;
+      tl.ocol = j * p.G + fb * W * SUB;
+      tl.ncols = 2 * W * SUB;
     }
   } else {
     const int mt = t / p.n_tiles, n = t % p.n_tiles;
@@ -521,68 +568,78 @@ template <int MODE, int CG>
 __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t* full,
                                         uint64_t* empty, volatile int* abort_flag, uint32_t rank,
                                         int unit, int n_units) {
-  using C = Cfg<CG>;
+  using C = Cfg<MODE, CG>;
+  // This one thread refills every stage, so its per-stage path is kept short:
+  // everything that depends only on the tile is resolved before the K loop
+  // (no tile-array indexing inside it), and which stages hold loads in flight
+  // is tracked in two bit masks.
   int stage = 0;
   uint32_t phase = 0;
-  int issued_parity[C::STAGES];
-#pragma unroll
-  for (int s = 0; s < C::STAGES; ++s) issued_parity[s] = -1;
+  uint32_t issued = 0, issued_phase = 0;  // bit s: stage s was filled; its phase
   const int total = total_tiles<MODE, CG>(p);
   const int nkb = k_blocks<MODE>(p);
+  const uint32_t ring0 = smem_u32(ring);
+  const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
+  const uint32_t full0_leader = CG == 1 ? full0 : map_to_rank(full0, 0);
   bool ok = true;
   for (int t = unit; t < total && ok; t += n_units) {
-    const Tile tl = decode_tile<MODE, CG>(p, t);
+    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, t);
     const int arow = tl.m0 + (CG == 2 ? BM * (int)rank : 0);
     // A routed pair tile of <= 128 rows has none in CTA 1: it loads no A there
     // (its accumulator rows are never stored) and the leader expects fewer bytes.
-    const bool routed = MODE == ROUTED1 || MODE == ROUTED2;
-    const int a_ctas = (CG == 2 && routed && tl.rows <= BM) ? 1 : CG;
-    const bool load_a = (int)rank < a_ctas;
+    constexpr bool kRoutedPair = CG == 2 && (MODE == ROUTED1 || MODE == ROUTED2);
+    int a_ctas = CG;
+    if constexpr (kRoutedPair) a_ctas = tl.rows <= BM ? 1 : 2;
+    const bool load_a = CG == 1 || !kRoutedPair || (int)rank < a_ctas;
+    const uint32_t tx_bytes = (uint32_t)(a_ctas * A_BYTES + tl.ncols * BK * 2);
+    // the B sub-tiles this CTA loads: CG = 1 sub-tiles 0 (and 1); CG = 2 the
+    // sub-tile of its rank (and, for wide tiles, rank + 2 at B offset 1)
+    const int sa = CG == 1 ? 0 : (int)rank;
+    const bool two = (CG == 1 && tl.n_sub > 1) || C::W == 2;
+    const int sb = CG == 1 ? 1 : (int)rank + 2;
+    int ma = tl.bmap[sa], mb = two ? tl.bmap[sb] : 0;
+    const int row_a = tl.brow[sa], z_a = tl.bz[sa];
+    const int row_b = two ? tl.brow[sb] : 0, z_b = two ? tl.bz[sb] : 0;
+    if (is_xpass<MODE>() && ma == kPadMap) ma = 1;
+    if (is_xpass<MODE>() && mb == kPadMap) mb = 1;
+    const bool td_a = !(is_xpass<MODE>() && ma < 2), td_b = !(is_xpass<MODE>() && mb < 2);
+    const CUtensorMap* map_a = bmap_ptr(p, ma);
+    const CUtensorMap* map_b = bmap_ptr(p, mb);
+    const uint32_t off_b = SUB * BK * 2;  // the second sub-tile's B offset
     for (int kb = 0; kb < nkb; ++kb) {
-      if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, p.status)) {
+      if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) {
         ok = false;
         break;
       }
-      const uint32_t a_dst = smem_u32(ring + stage * C::STAGE_BYTES);
+      const uint32_t a_dst = ring0 + stage * C::STAGE_BYTES;
       const uint32_t b_dst = a_dst + A_BYTES;
-      const uint32_t own_bar = smem_u32(&full[stage]);
-      const uint32_t bar = CG == 1 ? own_bar : map_to_rank(own_bar, 0);
-      if (CG == 1 || rank == 0)
-        mbar_expect_tx(own_bar, a_ctas * A_BYTES + tl.ncols * BK * 2);
-      // sub-tiles this CTA loads: all of them (CG = 1) or the one of its rank
-      const int s0 = CG == 1 ? 0 : (int)rank;
-      const int s1 = CG == 1 ? tl.n_sub : (int)rank + 1;
+      const uint32_t own_bar = full0 + 8 * stage;
+      const uint32_t bar = full0_leader + 8 * stage;
+      if (CG == 1 || rank == 0) mbar_expect_tx(own_bar, tx_bytes);
       if (MODE == FINAL) {
         const int kb_sh = p.S * p.kb0;
         if (kb < kb_sh) {
           const int j = kb / p.kb0, kk = (kb % p.kb0) * BK;
           if (CG == 1) tma_load_2d(a_dst, &p.tmA0, bar, j * p.G + kk, arow);
           else tma2_load_2d(a_dst, &p.tmA0, bar, j * p.G + kk, arow);
-          for (int s = s0; s < s1; ++s)
-            load_b<CG>(b_dst + (CG == 1 ? s * SUB * BK * 2 : 0), s == 0 ? &p.tmB0 : &p.tmB2, true,
-                       bar, kk, tl.brow[s], j);
+          load_b<CG>(b_dst, sa == 0 ? &p.tmB0 : &p.tmB2, true, bar, kk, row_a, j);
+          if (CG == 1 && two) load_b<CG>(b_dst + off_b, &p.tmB2, true, bar, kk, row_b, j);
         } else {
           const int kk = (kb - kb_sh) * BK;
           if (CG == 1) tma_load_2d(a_dst, &p.tmA1, bar, kk, arow);
           else tma2_load_2d(a_dst, &p.tmA1, bar, kk, arow);
-          for (int s = s0; s < s1; ++s)
-            load_b<CG>(b_dst + (CG == 1 ? s * SUB * BK * 2 : 0), s == 0 ? &p.tmB1 : &p.tmB3, false,
-                       bar, kk, tl.brow[s], 0);
+          load_b<CG>(b_dst, sa == 0 ? &p.tmB1 : &p.tmB3, false, bar, kk, row_a, 0);
+          if (CG == 1 && two) load_b<CG>(b_dst + off_b, &p.tmB3, false, bar, kk, row_b, 0);
         }
       } else {
         const int kk = kb * BK;
         if (CG == 1) tma_load_2d(a_dst, &p.tmA0, bar, kk, arow);
         else if (load_a) tma2_load_2d(a_dst, &p.tmA0, bar, kk, arow);
-        for (int s = s0; s < s1; ++s) {
-          int m = tl.bmap[s];
-          const bool pad = (is_xpass<MODE>() && m == kPadMap);
-          if (pad) m = 1;
-          const bool three_d = !(is_xpass<MODE>() && m < 2);
-          load_b<CG>(b_dst + (CG == 1 ? s * SUB * BK * 2 : 0), bmap_ptr(p, m), three_d, bar, kk,
-                     tl.brow[s], tl.bz[s]);
-        }
+        load_b<CG>(b_dst, map_a, td_a, bar, kk, row_a, z_a);
+        if (two) load_b<CG>(b_dst + off_b, map_b, td_b, bar, kk, row_b, z_b);
       }
-      issued_parity[stage] = (int)phase;
+      issued |= 1u << stage;
+      issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
       if (++stage == C::STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -594,9 +651,9 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
   if (CG == 1 || rank == 0) {
 #pragma unroll
     for (int s = 0; s < C::STAGES; ++s)
-      if (issued_parity[s] >= 0) {
+      if (issued & (1u << s)) {
         volatile int no_abort = 0;
-        mbar_wait(smem_u32(&full[s]), (uint32_t)issued_parity[s], &no_abort, p.status);
+        mbar_wait(full0 + 8 * s, (issued_phase >> s) & 1u, &no_abort, p.status);
       }
   }
 }
@@ -607,7 +664,7 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
                                           uint64_t* empty, uint64_t* tfull, uint64_t* tempty,
                                           uint64_t* drain, uint32_t tmem, volatile int* abort_flag,
                                           int unit, int n_units) {
-  using C = Cfg<CG>;
+  using C = Cfg<MODE, CG>;
   int stage = 0;
   uint32_t phase = 0;
   int acc = 0;
@@ -616,11 +673,11 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
   const int nkb = k_blocks<MODE>(p);
   bool ok = true;
   for (int t = unit; t < total && ok; t += n_units) {
-    const Tile tl = decode_tile<MODE, CG>(p, t);
-    const uint32_t idesc = instr_desc_cg<CG>(tl.ncols);
+    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, t);
+    const uint32_t idesc = instr_desc_cg<CG>(tl.ncols / C::W);
     if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.status)) break;
     tc_fence_after();
-    const uint32_t d_tmem = tmem + acc * ACC_COLS;
+    const uint32_t d_tmem = tmem + acc * C::ACC_STRIDE;
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.status)) {
         ok = false;
@@ -632,10 +689,14 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
 #pragma unroll
       for (int k = 0; k < BK / 16; ++k) {
         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-        if (CG == 1)
-          tc_mma(d_tmem, smem_desc(a_addr + k * 32), smem_desc(b_addr + k * 32), idesc, accum);
-        else
-          tc2_mma(d_tmem, smem_desc(a_addr + k * 32), smem_desc(b_addr + k * 32), idesc, accum);
+#pragma unroll
+        for (int w = 0; w < C::W; ++w) {  // W = 2: columns [256 w, 256 w + 256) from B block w
+          const uint32_t bw = b_addr + w * SUB * BK * 2 + k * 32;
+          if (CG == 1)
+            tc_mma(d_tmem + w * 256, smem_desc(a_addr + k * 32), smem_desc(bw), idesc, accum);
+          else
+            tc2_mma(d_tmem + w * 256, smem_desc(a_addr + k * 32), smem_desc(bw), idesc, accum);
+        }
       }
       if (CG == 1)
         tc_commit(smem_u32(&empty[stage]));
@@ -651,7 +712,7 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
       tc_commit(smem_u32(&tfull[acc]));
     else
       tc2_commit_both(smem_u32(&tfull[acc]));
-    if (++acc == 2) {
+    if (++acc == C::NACC) {
       acc = 0;
       acc_phase ^= 1u;
     }
@@ -673,15 +734,29 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
 // Read back, each store instruction covers 4 rows x 128 contiguous bytes
 // instead of 32 rows x 16 bytes.  rows / bytes: how many of the block's rows
 // and leading bytes of each row (a multiple of 16) exist; ld in bytes.
+// 16-byte chunk q (0..7) of this lane's row in the warp's staging block.
+__device__ __forceinline__ void stage_chunk(uint32_t stage, int q, uint32_t w0, uint32_t w1,
+                                            uint32_t w2, uint32_t w3) {
+  const int lane = threadIdx.x & 31;
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                   stage + lane * 128 + ((q ^ (lane & 7)) << 4)),
+               "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+               : "memory");
+}
+// Stores the staged block (rows of 128 bytes; see warp_store_block).
+__device__ __forceinline__ void warp_flush_block(uint32_t stage, char* base, int64_t ld, int rows,
+                                                 int bytes);
+
 __device__ __forceinline__ void warp_store_block(uint32_t stage, const uint32_t (&w)[32],
                                                  char* base, int64_t ld, int rows, int bytes) {
-  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int q = 0; q < 8; ++q)
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                     stage + lane * 128 + ((q ^ (lane & 7)) << 4)),
-                 "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
-                 : "memory");
+  for (int q = 0; q < 8; ++q) stage_chunk(stage, q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  warp_flush_block(stage, base, ld, rows, bytes);
+}
+
+__device__ __forceinline__ void warp_flush_block(uint32_t stage, char* base, int64_t ld, int rows,
+                                                 int bytes) {
+  const int lane = threadIdx.x & 31;
   __syncwarp();
   const int q = lane & 7;
 #pragma unroll
@@ -696,6 +771,32 @@ __device__ __forceinline__ void warp_store_block(uint32_t stage, const uint32_t 
       *reinterpret_cast<uint4*>(base + (int64_t)row * ld + q * 16) = v;
   }
   __syncwarp();
+}
+
+// SiTU of the 64 hidden units at gate columns [c0, c0 + 64) and up columns
+// [c0 + 128, c0 + 192) of this warp's 32 TMEM lanes, packed to bf16 and
+// written to the warp's staging block (row = lane, 128 bytes); store it with
+// warp_flush_block.  Each quarter of 16 units is read from TMEM at once and its
+// eight-unit chunks go to shared memory as soon as they are formed, so that
+// few values are live besides 32 accumulator columns (the epilogue runs at the
+// 168-register cap of 320-thread CTAs).
+__device__ __forceinline__ void situ_stage64(uint32_t tbase, uint32_t c0, uint32_t stage,
+                                             const SituConsts& sk) {
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    float g[16], u[16];
+    tc_ld16x2(tbase + c0 + 16 * h, g, tbase + SUB + c0 + 16 * h, u);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = 8 * q + 2 * j;
+        w[j] = situ2_bf16(g[i], g[i + 1], u[i], u[i + 1], sk);
+      }
+      stage_chunk(stage, 2 * h + q, w[0], w[1], w[2], w[3]);
+    }
+  }
 }
 
 __device__ __forceinline__ void warp_store_bf16(uint32_t stage, const uint32_t (&w)[32],
@@ -783,10 +884,10 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
   uint32_t acc_phase = 0;
   const int total = total_tiles<MODE, CG>(p);
   for (int t = unit; t < total; t += n_units) {
-    const Tile tl = decode_tile<MODE, CG>(p, t);
+    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, t);
     if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.status)) break;
     tc_fence_after();
-    const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * ACC_COLS;
+    const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * Cfg<MODE, CG>::ACC_STRIDE;
     const int rows = min(32, tl.rows - wrow);  // rows of this warp inside the tile
     const int64_t grow0 = (int64_t)tl.m0 + wrow;
     if (rows <= 0) {
@@ -807,7 +908,19 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         ld = p.ld0;
       }
       const int cols = min(64, width - half * 64);
-      if (MODE == XPASS_F32) {
+      if (MODE == XPASS_WIDE) {
+        // blocks of 64 hidden units b = half, half + 2: gate columns
+        // 256 (b / 2) + 64 (b % 2), up columns 128 further
+#pragma unroll 1
+        for (int b = half; b < 4; b += 2) {
+          const int bcols = min(64, width - 64 * b);
+          if (bcols <= 0) break;
+          const uint32_t c0 = (uint32_t)((b >> 1) * 256 + (b & 1) * 64);
+          situ_stage64(tbase, c0, stage, sk);
+          warp_flush_block(stage, reinterpret_cast<char*>(out + grow0 * ld + tl.ocol + 64 * b),
+                           ld * 2, rows, bcols * 2);
+        }
+      } else if (MODE == XPASS_F32) {
         if (cols > 0) {  // the pre-activations themselves, fp32
           float g0[32], u0[32], g1[32], u1[32];
           const uint32_t c0 = half * 64;
@@ -824,19 +937,9 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
           }
         }
       } else if (cols > 0) {
-        uint32_t w[32];
-        {
-          float g0[32], u0[32], g1[32], u1[32];
-          const uint32_t c0 = half * 64;
-          tc_ld32x4(tbase + c0, g0, tbase + SUB + c0, u0, tbase + c0 + 32, g1,
-                    tbase + SUB + c0 + 32, u1);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            w[j] = situ2_bf16(g0[2 * j], g0[2 * j + 1], u0[2 * j], u0[2 * j + 1], sk);
-            w[16 + j] = situ2_bf16(g1[2 * j], g1[2 * j + 1], u1[2 * j], u1[2 * j + 1], sk);
-          }
-        }
-        warp_store_bf16(stage, w, out + grow0 * ld + tl.ocol + half * 64, ld, rows, cols);
+        situ_stage64(tbase, (uint32_t)(half * 64), stage, sk);
+        warp_flush_block(stage, reinterpret_cast<char*>(out + grow0 * ld + tl.ocol + half * 64),
+                         ld * 2, rows, cols * 2);
       }
     } else if (is_xpass<MODE>()) {
 #pragma unroll 1
@@ -917,7 +1020,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
       else  // the leader's MMA thread waits for both CTAs' epilogues
         mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[acc]), 0));
     }
-    if (++acc == 2) {
+    if (++acc == Cfg<MODE, CG>::NACC) {
       acc = 0;
       acc_phase ^= 1u;
     }
@@ -926,7 +1029,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
 
 template <int MODE, int CG>
 __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
-  using C = Cfg<CG>;
+  using C = Cfg<MODE, CG>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full[C::STAGES], empty[C::STAGES], tfull[2], tempty[2], drain;
   __shared__ uint32_t tmem_slot;
@@ -1032,34 +1135,62 @@ static EncodeTiledFn encode_fn() {
 }
 
 // bf16 tensor [dim2][dim1][dim0] (dim0 contiguous) with a box of 64 x rows
-// (x 1), 128-byte swizzle, zero fill outside the tensor.
-static bool make_map(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
-                     uint32_t box_rows) {
+// (x 1), 128-byte swizzle, zero fill outside the tensor; rank 2 or 3.
+// Encoded maps are cached per host thread: a map is a function of the base
+// address, the extents, the box and the rank only, so a cached entry with the
+// same key is the map the encoder would return (a forward encodes about a
+// dozen maps, every call, otherwise).
+struct MapKey {
+  const void* base;
+  uint64_t d0, d1, d2;
+  uint32_t box, rank;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && box == o.box &&
+           rank == o.rank;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+constexpr int kMapCache = 64;
+
+static bool encode_map(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1,
+                       uint64_t dim2, uint32_t box_rows, uint32_t rank) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr || dim0 == 0 || dim1 == 0 || dim2 == 0) return false;
+  static thread_local MapEntry cache[kMapCache];
+  const MapKey key{base, dim0, dim1, dim2, box_rows, rank};
+  uint64_t h = reinterpret_cast<uintptr_t>(base) ^ (dim0 * 0x9E3779B97F4A7C15ull) ^
+               (dim1 * 0xC2B2AE3D27D4EB4Full) ^ (dim2 << 17) ^ ((uint64_t)box_rows << 7) ^ rank;
+  h ^= h >> 29;
+  MapEntry& e = cache[h % kMapCache];
+  if (e.valid && e.key == key) {
+    *m = e.map;
+    return true;
+  }
   cuuint64_t dims[3] = {dim0, dim1, dim2};
   cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
   cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  const cuuint32_t rank = dim2 > 1 ? 3 : 2;
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  e.key = key;
+  e.map = *m;
+  e.valid = true;
+  return true;
+}
+static bool make_map(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                     uint32_t box_rows) {
+  return encode_map(m, base, dim0, dim1, dim2, box_rows, dim2 > 1 ? 3 : 2);
 }
 // Always 3D maps for expert-stacked weights (so the kernel can pass 3 coordinates).
 static bool make_map3(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
                       uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr || dim0 == 0 || dim1 == 0 || dim2 == 0) return false;
-  cuuint64_t dims[3] = {dim0, dim1, dim2};
-  cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
-  cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_map(m, base, dim0, dim1, dim2, box_rows, 3);
 }
 
 // Per-device launch state: the SM count, and whether each kernel instance has
@@ -1096,7 +1227,7 @@ static cudaError_t launch(const Params& p, int grid, cudaStream_t st) {
     if (!attr[dev]) {
       cudaError_t e = cudaFuncSetAttribute(umma_gemm_kernel<MODE, CG>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           Cfg<CG>::SMEM_BYTES);
+                                           Cfg<MODE, CG>::SMEM_BYTES);
       if (e != cudaSuccess) return e;
       attr[dev] = true;
     }
@@ -1104,7 +1235,7 @@ static cudaError_t launch(const Params& p, int grid, cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
   count_launch();
   return launch_pdl(umma_gemm_kernel<MODE, CG>, dim3(CG * grid), dim3(THREADS),
-                    (size_t)Cfg<CG>::SMEM_BYTES, st, CG, p);
+                    (size_t)Cfg<MODE, CG>::SMEM_BYTES, st, CG, p);
 }
 
 // Tile width for the plain-store GEMMs: the one of 256, 192, 128 columns that
@@ -1152,12 +1283,14 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   p.S = a.S;
   p.G = a.G;
   p.d = a.d;
+  const bool f32 = a.z32 != nullptr;
+  const bool wide = a.wide && !f32;
+  const int ns = wide ? 4 : 2;  // B sub-tiles of 128 rows per tile
   p.nz_sub = (a.L + SUB - 1) / SUB;
   p.nr_sub = (a.R + SUB - 1) / SUB;
-  p.n_zr_tiles = (p.nz_sub + p.nr_sub + 1) / 2;
-  p.g_blocks = a.S > 0 ? (a.G + SUB - 1) / SUB : 0;
+  p.n_zr_tiles = (p.nz_sub + p.nr_sub + ns - 1) / ns;
+  p.g_blocks = a.S > 0 ? (a.G + SUB * (ns / 2) - 1) / (SUB * (ns / 2)) : 0;
   p.n_tiles = p.n_zr_tiles + a.S * p.g_blocks;
-  const bool f32 = a.z32 != nullptr;
   p.out0 = f32 ? (void*)a.z32 : (void*)a.z;
   p.ld0 = a.L;
   p.out1 = a.logits;
@@ -1178,8 +1311,9 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   p.probs = a.probs;
   const int total = (int)((a.N + 2 * BM - 1) / (2 * BM)) * p.n_tiles;
   const int units = a.max_units > 0 ? std::min(a.max_units, num_sms() / 2) : num_sms() / 2;
-  return f32 ? launch<XPASS_F32, 2>(p, std::min(total, units), st)
-             : launch<XPASS, 2>(p, std::min(total, units), st);
+  if (f32) return launch<XPASS_F32, 2>(p, std::min(total, units), st);
+  return wide ? launch<XPASS_WIDE, 2>(p, std::min(total, units), st)
+              : launch<XPASS, 2>(p, std::min(total, units), st);
 }
 
 cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {

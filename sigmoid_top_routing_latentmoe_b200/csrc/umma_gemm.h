@@ -42,6 +42,9 @@ struct XpassArgs {
   float* probs;
   int top_k;
   int max_units;  // at most this many CTA pairs (0: one per pair of SMs)
+  // 1: 256 x 512 tiles (two N = 256 MMAs per K step, one TMEM accumulator);
+  // 0: 256 x 256 tiles (double-buffered accumulator).  Ignored for z32.
+  int wide;
 };
 
 // final: y [N, d] = sum_j hsh[:, jG:(j+1)G] W_o,sh_j^T + uhat W_up^T
