@@ -88,14 +88,14 @@ def kernel_work(wl: synth.Workload, tag: str):
 
 class ClockSampler:
     """Samples the SM clock and the clock-event (throttle) reasons with NVML
-    while a region runs, as fast as NVML answers (a sample every ~0.2 ms)."""
+    while a region runs, as fast as NVML answers (a sample every ~0.1 ms)."""
 
     REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
                "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
                "display_clock_setting": 0x100}
 
-    def __init__(self, index: int, period_s: float = 2e-4):
+    def __init__(self, index: int, period_s: float = 5e-5):
         self.index = index
         self.period_s = period_s
         self.samples = []
@@ -626,6 +626,25 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, dev)
     io_bytes = wl.n_tokens * wl.d * (2 if wl.dtype == "bf16" else 4)
+    # the copies alone: x in and y out through the same pinned buffers, on two
+    # streams at once (what the host link allows per step, with no compute)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x_d, y_d = torch.empty_like(x), torch.empty_like(x)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for it in range(e2e_steps + 3):
+        if it == 3:
+            c0.record(stream)
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        with torch.cuda.stream(s_in):
+            x_d.copy_(x_h, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            y_h.copy_(y_d, non_blocking=True)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    copy_ms = c0.elapsed_time(c1) / e2e_steps
 
     peaks = _peaks()
     if k_n > 0:
@@ -665,7 +684,10 @@ def main():
         "hot": {"value": world * wl.n_tokens / (hot_ms / 1e3), "unit": "tokens/s",
                 "ms_per_step": hot_ms, "l2": "not flushed (back-to-back steps)"},
         "e2e": {"value": world * wl.n_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
+                "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
+                "ms_per_step": e2e_ms,
+                "copies_alone_ms_per_step": copy_ms,
+                "copy_bound": world * wl.n_tokens / (copy_ms / 1e3)},
         "gpu_launches": launches,
         "host_enqueue_us": host_enqueue_us,
         "kernel_us": breakdown,

@@ -286,8 +286,11 @@ LMOE_API lmoe_status moe_dispatch_noalloc(const lmoe_dims* dims, const int32_t* 
                                           int32_t* counts, int32_t* offsets, int32_t* perm_token,
                                           int32_t* inv_pair, lmoe_stream stream);
 
-/* Zeroes the workspace header (status word and scheduling counters).  Call
- * once on a new workspace before its first use. */
+/* Zeroes the workspace header (status word and scheduling counters) and the
+ * synchronisation area that follows it (the final GEMM's per-tile row counts
+ * for its fused combine, which every launch leaves zeroed).  Call once on a
+ * new workspace before its first use, and again after a call reported
+ * LMOE_ETIMEOUT (an aborted launch can leave counts behind). */
 LMOE_API lmoe_status lmoe_workspace_init(void* ws, size_t ws_bytes, lmoe_stream stream);
 
 /* Waits for `stream`, then reads and clears the workspace status word.

@@ -134,8 +134,8 @@ static lmoe_status check_dims(const lmoe_dims* d) {
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t header, z, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, zp, h, eo,
-      hsh, uhat, loss, x, y, total;
+  size_t header, sync, z, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, zp, h,
+      eo, hsh, uhat, loss, x, y, total;
   int64_t logits_ld;
   int max_tiles;
 };
@@ -150,6 +150,7 @@ static Layout layout(const lmoe_dims* d, bool host_copies) {
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t at = off; off += align256(bytes); return at; };
   L.header = take(sizeof(WsHeader));
+  L.sync = take((size_t)kSyncWords * 4);  // right after the header: cleared with it
   L.z = take((size_t)N * d->latent * es);
   L.logits = take((size_t)N * L.logits_ld * 4);
   L.ids = take((size_t)P * 4);
@@ -385,7 +386,11 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
   const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * sizeof(T) <= (16u << 20);
   LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
   LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
-  {
+  // For l <= 1024 the combine runs inside the final GEMM (its epilogue warps
+  // write RMSNorm(u) while the K loop goes through the shared experts' blocks);
+  // wider rows get the combine kernel first.
+  const bool fuse_combine = Lt <= 1024 && (N + 255) / 256 <= kSyncWords - 1;
+  if (!fuse_combine) {
     ProfScope ps("combine", st);
     LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, k, Lt, d->rms_eps, uhat, st),
               "combine");
@@ -395,6 +400,10 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
     FinalArgs a{};
     a.hsh = hsh; a.N = N; a.S = S; a.G = G; a.ws_o = (const T*)w->ws_o; a.d = D;
     a.uhat = uhat; a.L = Lt; a.w_up = (const T*)w->w_up; a.y = (T*)y;
+    if (fuse_combine) {
+      a.eo = eo; a.inv = inv; a.probs = probs; a.rms_w = w->rms_weight; a.top_k = k;
+      a.rms_eps = d->rms_eps; a.sync = at<int32_t>(ws, L.sync);
+    }
     ProfScope ps("final", st);
     LMOE_CUDA(umma_final(a, status, st), "final (tcgen05)");
   }
@@ -527,32 +536,35 @@ static lmoe_status host_pipe(HostPipe** out) {
   return LMOE_OK;
 }
 
-// Number of token chunks for the host entry point, from a rough cost model:
-// per chunk of n tokens, the copies take n*d*es / 50 GB/s each way and the
-// forward max(FLOPs / 1 PFLOP/s, bytes / 6 TB/s) + 15 us of launch latency,
-// where every chunk streams the weights of the experts it selects again.  The
-// pipeline costs copy_in(first) + sum over chunks of the slowest stage +
-// copy_out(last); the count with the least estimate wins (1 when streaming the
-// weights dominates, as at widths where they are gigabytes).
+// Number of token chunks for the host entry point, from a cost model of the
+// pipeline copy_in(first) + sum over chunks of the slowest stage +
+// copy_out(last): per chunk of n tokens the copies take n d es / 50 GB/s each
+// way, and the forward its dense GEMMs' FLOPs at 0.8 PFLOP/s plus the routed
+// experts' max(FLOPs at 0.8 PFLOP/s, weights of the experts the chunk selects
+// at 6 TB/s) plus 60 us of launch latency and tile tails (a 1024-token chunk of
+// the 0.5b layer takes ~90 us against 122 us for 4096 tokens: small chunks
+// leave most SMs idle).  A chunked plan must beat one chunk by 15 %.
 static int host_chunks(const lmoe_dims* d) {
   const double N = (double)d->n_tokens, es = d->dtype == LMOE_BF16 ? 2.0 : 4.0;
   const double D = d->d, L = d->latent, R = d->n_routed, k = d->top_k, F = d->ff_routed;
   const double SG = (double)d->n_shared * (d->n_shared > 0 ? d->ff_shared : 0);
-  const double flops_tok = 2 * D * L + 2 * D * R + 6 * k * L * F + 6 * SG * D + 2 * L * D;
-  const double w_dense = (2 * D * L + D * R + 3 * SG * D) * es, w_expert = 3 * F * L * es;
-  const double copy_bw = 50e9, flop_rate = d->dtype == LMOE_BF16 ? 1.0e15 : 2.0e13,
-               hbm = 6.0e12, launch = 15e-6;
-  double best = 0.0;
+  const double dense_tok = 2 * D * L + 2 * D * R + 6 * SG * D + 2 * L * D;
+  const double routed_tok = 6 * k * L * F;
+  const double w_expert = 3 * F * L * es;
+  const double copy_bw = 50e9, flop_rate = d->dtype == LMOE_BF16 ? 0.8e15 : 2.0e13,
+               hbm = 6.0e12, fixed = 60e-6;
+  double t1 = 0.0, best = 0.0;
   int best_c = 1;
   for (int c = 1; c <= kMaxHostChunks; ++c) {
     const double n = std::ceil(N / c);
     if (c > 1 && n < 256) break;
     const double used = R * (1.0 - std::pow(1.0 - k / R, n));  // experts a chunk selects
     const double t_copy = n * D * es / copy_bw;
-    const double t_fwd = std::max(n * flops_tok / flop_rate,
-                                  (w_dense + used * w_expert + 6 * n * D * es) / hbm) + launch;
+    const double t_fwd = n * dense_tok / flop_rate +
+                         std::max(n * routed_tok / flop_rate, used * w_expert / hbm) + fixed;
     const double t = 2 * t_copy + c * std::max(t_copy, t_fwd);
-    if (c == 1 || t < best) {
+    if (c == 1) t1 = t;
+    if (c == 1 || (t < best && t < 0.85 * t1)) {
       best = t;
       best_c = c;
     }
@@ -895,7 +907,9 @@ lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offsets, int32_
 lmoe_status lmoe_workspace_init(void* ws, size_t ws_bytes, lmoe_stream stream) {
   LMOE_PTR(ws, "ws");
   if (ws_bytes < sizeof(WsHeader)) return fail(LMOE_EWORKSPACE, "workspace smaller than its header");
-  LMOE_CUDA(cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream), "memset header");
+  // the header and the synchronisation area after it
+  const size_t n = std::min(ws_bytes, align256(sizeof(WsHeader)) + (size_t)kSyncWords * 4);
+  LMOE_CUDA(cudaMemsetAsync(ws, 0, n, (cudaStream_t)stream), "memset header");
   return LMOE_OK;
 }
 

@@ -5,6 +5,7 @@
 //   u_normed_t = u_t * (1 / sqrt(mean(u_t^2) + eps)) * w
 // Each token is reduced by one warp in a fixed order: no float atomics, so
 // the result is deterministic.  Rows are read with 16-byte vectors.
+#include "combine_row.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "launch.h"
@@ -20,52 +21,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ eo,
                                                       int k, int L, float eps, T* __restrict__ out) {
   pdl_trigger();
   pdl_wait();
-  constexpr int E = 16 / sizeof(T);  // elements per vector
-  const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= n) return;
-  const int nvec = L / E;
-  float u[VPL][E];
-#pragma unroll
-  for (int v = 0; v < VPL; ++v)
-#pragma unroll
-    for (int e = 0; e < E; ++e) u[v][e] = 0.0f;
-#pragma unroll 4
-  for (int i = 0; i < k; ++i) {  // unrolled: up to four slots' rows in flight
-    const int64_t r = inv_pair[t * k + i];
-    if (r < 0) continue;  // a pair the dispatch dropped (out-of-range id)
-    const float p = probs[t * k + i];
-    const uint4* row = reinterpret_cast<const uint4*>(eo + r * L);
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      int vi = v * 32 + lane;
-      if (vi < nvec) {
-        uint4 raw = row[vi];
-        const T* el = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-        for (int e = 0; e < E; ++e) u[v][e] = fmaf(p, to_f(el[e]), u[v][e]);
-      }
-    }
-  }
-  float ss = 0.0f;
-#pragma unroll
-  for (int v = 0; v < VPL; ++v)
-#pragma unroll
-    for (int e = 0; e < E; ++e) ss = fmaf(u[v][e], u[v][e], ss);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  const float inv = rsqrtf(ss / (float)L + eps);
-#pragma unroll
-  for (int v = 0; v < VPL; ++v) {
-    int vi = v * 32 + lane;
-    if (vi < nvec) {
-      uint4 raw;
-      T* el = reinterpret_cast<T*>(&raw);
-#pragma unroll
-      for (int e = 0; e < E; ++e) el[e] = from_f<T>(u[v][e] * inv * rms_w[vi * E + e]);
-      reinterpret_cast<uint4*>(out + t * L)[vi] = raw;
-    }
-  }
+  combine_row<T, VPL>(eo, inv_pair, probs, rms_w, t, k, L, eps, out);
 }
 
 // Wide rows (l > 1024): one 128-thread block per token, VPT 16-byte vectors

@@ -20,6 +20,12 @@ constexpr int kStatusTimeout = LMOE_ETIMEOUT;
 constexpr int kTileM = 128;
 constexpr int kRoutedPairTileM = 256;
 
+// Words of the synchronisation area that follows the workspace header: the
+// final GEMM with the fused combine counts the RMSNorm(u) rows ready per
+// 256-row tile there (up to kSyncWords - 1 tiles) and keeps a finished-CTA
+// counter in the last word; every such launch leaves it zeroed again.
+constexpr int kSyncWords = 1024;
+
 // Header at the start of every workspace.
 struct WsHeader {
   int32_t status;        // 0, or the first failure code recorded on the device

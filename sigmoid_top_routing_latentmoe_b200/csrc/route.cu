@@ -225,10 +225,17 @@ __device__ __forceinline__ float warp_sort32_desc(float v) {
   return v;
 }
 
-// k rounds of a warp argmax over keys held VPL per lane (expert e = j*32 +
-// lane; ties to the lower expert), the selected experts' scores read back from
-// the logits row lr: the same slots and weights as select_topk, without a
-// second array of scores in registers.
+// Expert held as value j of a lane in the wide top-k: the row is read as
+// float4 groups, group g of 128 experts giving lane l experts 128 g + 4 l ...
+// 128 g + 4 l + 3.
+__device__ __forceinline__ int wide_expert(int j, int lane) {
+  return (j >> 2) * 128 + lane * 4 + (j & 3);
+}
+
+// k rounds of a warp argmax over keys held VPL per lane (expert
+// wide_expert(j, lane); ties to the lower expert), the selected experts'
+// scores read back from the logits row lr: the same slots and weights as
+// select_topk, without a second array of scores in registers.
 template <int VPL, bool SOFTMAX>
 __device__ __noinline__ void select_topk_keys(float (&key)[VPL], const float* __restrict__ lr, int R,
                                               int k, int32_t* ids_row, float* probs_row) {
@@ -239,7 +246,7 @@ __device__ __noinline__ void select_topk_keys(float (&key)[VPL], const float* __
     int bi = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
-      const int e = j * 32 + lane;
+      const int e = wide_expert(j, lane);
       if (e < R && (key[j] > bk || (key[j] == bk && e < bi))) {
         bk = key[j];
         bi = e;
@@ -248,7 +255,7 @@ __device__ __noinline__ void select_topk_keys(float (&key)[VPL], const float* __
     warp_argmax(bk, bi);
 #pragma unroll
     for (int j = 0; j < VPL; ++j)
-      if (j * 32 + lane == bi) key[j] = -INFINITY;
+      if (wide_expert(j, lane) == bi) key[j] = -INFINITY;
     float sc = SOFTMAX ? lr[bi] : sigmoid_f(lr[bi]);
     if (SOFTMAX) {
       if (slot == 0) first = sc;
@@ -279,32 +286,47 @@ __device__ __noinline__ void select_topk_keys(float (&key)[VPL], const float* __
 // The selection keys use the fast exponential and division (|error| ~1e-7,
 // far below the routing margins); the selected scores are recomputed exactly.
 template <int VPL, bool SOFTMAX>
-__global__ void __launch_bounds__(256, VPL <= 32 ? 4 : 1) route_topk_wide_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(256, VPL <= 32 ? (SOFTMAX ? 3 : 4) : 1) route_topk_wide_kernel(const float* __restrict__ logits,
                                                               int64_t ld,
                                                               const float* __restrict__ bias,
                                                               int64_t n, int R, int k,
                                                               int32_t* __restrict__ ids,
                                                               float* __restrict__ probs) {
   pdl_trigger();
-  pdl_wait();
   __shared__ uint64_t cand[8][64];
+  extern __shared__ float sbias[];  // [R]: the bias, read once per block
+  if (!SOFTMAX) {
+    for (int e = threadIdx.x; e < R; e += blockDim.x) sbias[e] = bias != nullptr ? bias[e] : 0.0f;
+    __syncthreads();
+  }
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= n) return;
-  const float* lr = logits + t * ld;
+  const float* lr = logits + t * ld;  // ld: a multiple of 16 floats, >= R
   float key[VPL];
   float lmax = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    const int e = j * 32 + lane;
-    float kv = -INFINITY;
-    if (e < R) {
-      const float l = lr[e];
-      kv = SOFTMAX ? l
-                   : __fdividef(1.0f, 1.0f + __expf(-l)) + (bias != nullptr ? bias[e] : 0.0f);
+  for (int g = 0; g < VPL / 4; ++g) {
+    const int e0 = g * 128 + lane * 4;
+    float4 l4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (VPL <= 64) {  // one 16-byte load per group (e0 + 3 < ld)
+      if (e0 < R) l4 = *reinterpret_cast<const float4*>(lr + e0);
+    } else {  // the widest rows: scalar loads keep fewer values live
+      if (e0 < R) l4.x = lr[e0];
+      if (e0 + 1 < R) l4.y = lr[e0 + 1];
+      if (e0 + 2 < R) l4.z = lr[e0 + 2];
+      if (e0 + 3 < R) l4.w = lr[e0 + 3];
     }
-    key[j] = kv;
-    lmax = fmaxf(lmax, kv);
+    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float kv = -INFINITY;
+      if (e0 + c < R)
+        kv = SOFTMAX ? lv[c] : __fdividef(1.0f, 1.0f + __expf(-lv[c])) + sbias[e0 + c];
+      key[4 * g + c] = kv;
+      lmax = fmaxf(lmax, kv);
+    }
   }
   const float lk = __shfl_sync(0xffffffffu, warp_sort32_desc(lmax), k - 1);
   int mine = 0;
@@ -321,10 +343,10 @@ __global__ void __launch_bounds__(256, VPL <= 32 ? 4 : 1) route_topk_wide_kernel
     // exact keys (the fast ones above may differ in the last bits)
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
-      const int e = j * 32 + lane;
+      const int e = wide_expert(j, lane);
       if (e < R) {
         const float l = lr[e];
-        key[j] = SOFTMAX ? l : sigmoid_f(l) + (bias != nullptr ? bias[e] : 0.0f);
+        key[j] = SOFTMAX ? l : sigmoid_f(l) + sbias[e];
       }
     }
     select_topk_keys<VPL, SOFTMAX>(key, lr, R, k, ids + t * k, probs + t * k);
@@ -334,7 +356,7 @@ __global__ void __launch_bounds__(256, VPL <= 32 ? 4 : 1) route_topk_wide_kernel
 #pragma unroll
   for (int j = 0; j < VPL; ++j) {
     if (key[j] >= lk) {
-      const uint32_t e = (uint32_t)(j * 32 + lane);
+      const uint32_t e = (uint32_t)wide_expert(j, lane);
       cand[warp][at++] = ((uint64_t)orderable(key[j]) << 32) | (uint64_t)(0xffffffffu - e);
     }
   }
@@ -398,8 +420,8 @@ cudaError_t launch_route_topk(const float* logits, int64_t ld, const float* bias
                                  dim3(warps * 32), 0, st, 1, logits, ld, bias, n, R, k, ids, \
                                  probs)                                                      \
                     : launch_pdl(route_topk_wide_kernel<V, false>, dim3(blocks),             \
-                                 dim3(warps * 32), 0, st, 1, logits, ld, bias, n, R, k, ids, \
-                                 probs);                                                     \
+                                 dim3(warps * 32), (size_t)R * sizeof(float), st, 1, logits, \
+                                 ld, bias, n, R, k, ids, probs);                             \
     }
     LMOE_TOPK_WIDE(4)
     LMOE_TOPK_WIDE(8)

@@ -34,6 +34,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "combine_row.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "umma_gemm.h"
@@ -48,7 +49,14 @@ constexpr int SUB = 128;         // rows of a full B sub-tile
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
-constexpr int EPI_WARPS = 8;    // two warps per TMEM lane quarter, splitting the columns
+#ifndef LMOE_EPI_WARPS
+#define LMOE_EPI_WARPS 8
+#endif
+// Epilogue warps: 8 = two per TMEM lane quarter, splitting the column blocks;
+// 4 = one per quarter, each taking every column block.
+constexpr int EPI_WARPS = LMOE_EPI_WARPS;
+static_assert(EPI_WARPS == 4 || EPI_WARPS == 8, "4 or 8 epilogue warps");
+constexpr int HS = EPI_WARPS / 4;  // column-block stride of one epilogue warp
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint64_t WAIT_CAP_NS = 2000000000ull;
 
@@ -113,6 +121,15 @@ struct Params {
   const int32_t* n_mtiles;
   int32_t* status;
   float beta1, beta2, inv_beta1, inv_beta2, beta12;
+  // FINAL with the fused combine (see FinalArgs)
+  const __nv_bfloat16* c_eo;
+  const int32_t* c_inv;
+  const float* c_probs;
+  const float* c_rms;
+  __nv_bfloat16* c_uhat;
+  int32_t* c_sync;
+  int c_k, c_vpl, fuse_combine;
+  float c_eps;
 };
 
 template <int NS>  // at most NS B sub-tiles
@@ -175,6 +192,31 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
   return true;
 }
+// Capped wait until the counter at c reaches target (acquire), then a proxy
+// fence so that TMA loads issued afterwards see the global writes it counted.
+__device__ __forceinline__ bool wait_count(const int32_t* c, int target, volatile int* abort_flag,
+                                           int32_t* status) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 1;; ++it) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+    if (v >= target) break;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      const uint64_t now = global_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > WAIT_CAP_NS) {
+        *abort_flag = 1;
+        record_status(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1) {
   asm volatile(
@@ -607,6 +649,13 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
     const CUtensorMap* map_b = bmap_ptr(p, mb);
     const uint32_t off_b = SUB * BK * 2;  // the second sub-tile's B offset
     for (int kb = 0; kb < nkb; ++kb) {
+      if (MODE == FINAL && p.fuse_combine && kb == p.S * p.kb0) {
+        // the uhat rows of this tile are written by the kernel's own epilogue warps
+        if (!wait_count(p.c_sync + tl.m0 / Cfg<MODE, CG>::MT, tl.rows, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+      }
       if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) {
         ok = false;
         break;
@@ -876,10 +925,33 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
                                          uint32_t tmem, uint32_t stage, volatile int* abort_flag,
                                          uint32_t rank, int unit, int n_units) {
   const int ew = (threadIdx.x >> 5) & 3;  // TMEM lane quarter this warp may access
-  const int half = ((threadIdx.x >> 5) - 2) >> 2;  // which half of the column blocks
+  // first column block of this warp (then every HS-th)
+  const int h0 = EPI_WARPS == 8 ? ((threadIdx.x >> 5) - 2) >> 2 : 0;
   const int lane = threadIdx.x & 31;
   const int wrow = ew * 32 + (CG == 2 ? BM * (int)rank : 0);  // first tile row of this warp
   const SituConsts sk = situ_consts(p);
+  if (MODE == FINAL && p.fuse_combine) {
+    // The fused combine: uhat rows of an even share per CTA, one warp per row,
+    // each row counted in its 256-row tile's word once written.  Runs while the
+    // first tile's K loop goes through the shared experts' blocks.
+    const int ewarp = (threadIdx.x >> 5) - 2;
+    const int64_t per = (p.M + gridDim.x - 1) / gridDim.x;
+    const int64_t r0 = (int64_t)blockIdx.x * per, r1 = min((int64_t)p.M, r0 + per);
+    for (int64_t t = r0 + ewarp; t < r1; t += EPI_WARPS) {
+      if (p.c_vpl == 1)
+        combine_row<__nv_bfloat16, 1>(p.c_eo, p.c_inv, p.c_probs, p.c_rms, t, p.c_k, p.L, p.c_eps,
+                                      p.c_uhat);
+      else if (p.c_vpl == 2)
+        combine_row<__nv_bfloat16, 2>(p.c_eo, p.c_inv, p.c_probs, p.c_rms, t, p.c_k, p.L, p.c_eps,
+                                      p.c_uhat);
+      else
+        combine_row<__nv_bfloat16, 4>(p.c_eo, p.c_inv, p.c_probs, p.c_rms, t, p.c_k, p.L, p.c_eps,
+                                      p.c_uhat);
+      __threadfence();  // every lane's stores of the row, then one count
+      __syncwarp();
+      if (lane == 0) atomicAdd(p.c_sync + t / Cfg<MODE, CG>::MT, 1);
+    }
+  }
   int acc = 0;
   uint32_t acc_phase = 0;
   const int total = total_tiles<MODE, CG>(p);
@@ -894,7 +966,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
       // nothing of this warp's rows exists in the tile
     } else if (tl.epi == EPI_SITU) {
       // columns [0,128) hold gate pre-activations, [128,256) the matching up ones;
-      // this warp writes hidden units [64 half, 64 half + 64)
+      // this warp writes the blocks of 64 hidden units h0, h0 + HS, ...
       int width;
       __nv_bfloat16* out;
       int64_t ld;
@@ -907,12 +979,11 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         out = static_cast<__nv_bfloat16*>(p.out0);
         ld = p.ld0;
       }
-      const int cols = min(64, width - half * 64);
       if (MODE == XPASS_WIDE) {
-        // blocks of 64 hidden units b = half, half + 2: gate columns
-        // 256 (b / 2) + 64 (b % 2), up columns 128 further
+        // blocks of 64 hidden units b (of 4): gate columns 256 (b / 2) + 64 (b % 2),
+        // up columns 128 further
 #pragma unroll 1
-        for (int b = half; b < 4; b += 2) {
+        for (int b = h0; b < 4; b += HS) {
           const int bcols = min(64, width - 64 * b);
           if (bcols <= 0) break;
           const uint32_t c0 = (uint32_t)((b >> 1) * 256 + (b & 1) * 64);
@@ -921,12 +992,15 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
                            ld * 2, rows, bcols * 2);
         }
       } else if (MODE == XPASS_F32) {
-        if (cols > 0) {  // the pre-activations themselves, fp32
+#pragma unroll 1
+        for (int b = h0; b < 2; b += HS) {  // the pre-activations themselves, fp32
+          const int cols = min(64, width - b * 64);
+          if (cols <= 0) break;
           float g0[32], u0[32], g1[32], u1[32];
-          const uint32_t c0 = half * 64;
+          const uint32_t c0 = b * 64;
           tc_ld32x4(tbase + c0, g0, tbase + SUB + c0, u0, tbase + c0 + 32, g1,
                     tbase + SUB + c0 + 32, u1);
-          const int64_t at = grow0 * p.ld2 + tl.ocol + half * 64;
+          const int64_t at = grow0 * p.ld2 + tl.ocol + b * 64;
           float* ga = static_cast<float*>(p.out2) + at;
           float* ua = static_cast<float*>(p.out3) + at;
           warp_store_f32(stage, g0, ga, p.ld2, rows, min(32, cols));
@@ -936,10 +1010,15 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
             warp_store_f32(stage, u1, ua + 32, p.ld2, rows, cols - 32);
           }
         }
-      } else if (cols > 0) {
-        situ_stage64(tbase, (uint32_t)(half * 64), stage, sk);
-        warp_flush_block(stage, reinterpret_cast<char*>(out + grow0 * ld + tl.ocol + half * 64),
-                         ld * 2, rows, cols * 2);
+      } else {
+#pragma unroll 1
+        for (int b = h0; b < 2; b += HS) {
+          const int cols = min(64, width - b * 64);
+          if (cols <= 0) break;
+          situ_stage64(tbase, (uint32_t)(b * 64), stage, sk);
+          warp_flush_block(stage, reinterpret_cast<char*>(out + grow0 * ld + tl.ocol + b * 64),
+                           ld * 2, rows, cols * 2);
+        }
       }
     } else if (is_xpass<MODE>()) {
 #pragma unroll 1
@@ -948,7 +1027,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         if (tl.bmap[s] == 1) {  // router logits
           if (p.fuse_topk) {
             // all R <= 32 router logits of a row sit in one 32-column chunk
-            if (half == 0) {
+            if (h0 == 0) {
               float lg[32];
               tc_ld32(tbase + tl.scol[s], lg);
               if (lane < rows) {
@@ -964,7 +1043,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
             continue;
           }
 #pragma unroll 1
-          for (int c = half; c < tl.srows[s] / 32; c += 2) {
+          for (int c = h0; c < tl.srows[s] / 32; c += HS) {
             float v[32];
             tc_ld32(tbase + tl.scol[s] + c * 32, v);
             if (lane >= rows) continue;
@@ -978,30 +1057,33 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
           }
           continue;
         }
-        // z columns [brow + 64 half, +64)
-        const int col = tl.brow[s] + half * 64;
-        const int cols = min(64, p.L - col);
-        if (cols <= 0) continue;
-        float a[32], b[32];
-        tc_ld32x2(tbase + tl.scol[s] + half * 64, a, tbase + tl.scol[s] + half * 64 + 32, b);
-        if (MODE == XPASS_F32) {
-          float* zf = static_cast<float*>(p.out0) + grow0 * p.ld0 + col;
-          warp_store_f32(stage, a, zf, p.ld0, rows, min(32, cols));
-          if (cols > 32) warp_store_f32(stage, b, zf + 32, p.ld0, rows, cols - 32);
-          continue;
+        // z columns [brow + 64 hb, +64) for the blocks hb of this warp
+#pragma unroll 1
+        for (int hb = h0; hb < 2; hb += HS) {
+          const int col = tl.brow[s] + hb * 64;
+          const int cols = min(64, p.L - col);
+          if (cols <= 0) break;
+          float a[32], b[32];
+          tc_ld32x2(tbase + tl.scol[s] + hb * 64, a, tbase + tl.scol[s] + hb * 64 + 32, b);
+          if (MODE == XPASS_F32) {
+            float* zf = static_cast<float*>(p.out0) + grow0 * p.ld0 + col;
+            warp_store_f32(stage, a, zf, p.ld0, rows, min(32, cols));
+            if (cols > 32) warp_store_f32(stage, b, zf + 32, p.ld0, rows, cols - 32);
+            continue;
+          }
+          uint32_t w[32];
+          pack_block(a, b, w);
+          warp_store_bf16(stage, w, static_cast<__nv_bfloat16*>(p.out0) + grow0 * p.ld0 + col,
+                          p.ld0, rows, cols);
         }
-        uint32_t w[32];
-        pack_block(a, b, w);
-        warp_store_bf16(stage, w, static_cast<__nv_bfloat16*>(p.out0) + grow0 * p.ld0 + col,
-                        p.ld0, rows, cols);
       }
     } else {
       // FINAL / ROUTED2: accumulator columns [0, ncols) are output columns
-      // [ocol, ocol + ncols); this warp writes the 64-column blocks half, half + 2
+      // [ocol, ocol + ncols); this warp writes the 64-column blocks h0, h0 + HS, ...
       const int width = (MODE == FINAL ? p.d : p.L) - tl.ocol;
       const int ncols = min(tl.ncols, width);
 #pragma unroll 1
-      for (int cb = half; cb * 64 < ncols; cb += 2) {
+      for (int cb = h0; cb * 64 < ncols; cb += HS) {
         const int cols = min(64, ncols - cb * 64);
         const int64_t col = tl.ocol + cb * 64;
         float a[32], b[32];
@@ -1103,6 +1185,16 @@ __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_cons
   __syncthreads();
   if (CG == 2) cluster_sync();  // neither CTA frees TMEM or exits while its pair still works
   tc_fence_after();
+  if (MODE == FINAL && p.fuse_combine && threadIdx.x == 0) {
+    // the last CTA to finish (every CTA is past its waits) zeroes the counts
+    // for the next launch
+    __threadfence();
+    if (atomicAdd(p.c_sync + (kSyncWords - 1), 1) == (int)gridDim.x - 1) {
+      const int n_mt = (p.M + C::MT - 1) / C::MT;
+      for (int i = 0; i < n_mt; ++i) atomicExch(p.c_sync + i, 0);
+      atomicExch(p.c_sync + (kSyncWords - 1), 0);
+    }
+  }
   if (warp == 1) {
     if (CG == 1)
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -1341,6 +1433,20 @@ cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
   p.n_tiles = (a.d + p.bn - 1) / p.bn;
   p.out0 = a.y;
   p.ld0 = a.d;
+  if (a.eo != nullptr) {
+    const int nvec = a.L / 8;
+    p.fuse_combine = 1;
+    p.c_eo = a.eo;
+    p.c_inv = a.inv;
+    p.c_probs = a.probs;
+    p.c_rms = a.rms_w;
+    p.c_uhat = const_cast<__nv_bfloat16*>(a.uhat);
+    p.c_sync = a.sync;
+    p.c_k = a.top_k;
+    p.c_eps = a.rms_eps;
+    p.c_vpl = nvec <= 32 ? 1 : nvec <= 64 ? 2 : 4;
+    if (nvec > 128 || m_tiles > kSyncWords - 1) return cudaErrorInvalidValue;
+  }
   const int total = m_tiles * p.n_tiles;
   return launch<FINAL, 2>(p, std::min(total, units), st);
 }

@@ -59,6 +59,18 @@ struct FinalArgs {
   const __nv_bfloat16* w_up;  // [d, L]
   __nv_bfloat16* y;
   int max_units;  // at most this many CTA pairs (0: one per pair of SMs)
+  // Fused combine (eo != nullptr, L <= 1024): the kernel's epilogue warps first
+  // write uhat = RMSNorm(sum_i probs[t, i] eo[inv[t, i]]) * rms_w for an even
+  // share of the rows (the combine kernel's arithmetic), counting finished rows
+  // per 256-row tile in sync[]; each CTA's producer waits for its tile's count
+  // before loading the uhat K blocks, which come after the shared experts' ones.
+  const __nv_bfloat16* eo;  // [N k, L] expert outputs, sorted-pair order
+  const int32_t* inv;       // [N, k]
+  const float* probs;       // [N, k]
+  const float* rms_w;       // [L]
+  int top_k;
+  float rms_eps;
+  int32_t* sync;            // kSyncWords zeroed words (left zeroed)
 };
 
 // routed GEMM1: h [P, F] = SiTU(zp W_g,e^T, zp W_u,e^T) per row tile of expert e

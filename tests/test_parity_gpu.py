@@ -410,3 +410,25 @@ def test_check_dispatch_flags_corruptions():
     inv3 = inv.clone()
     inv3[1] = inv[0]
     assert flagged(inv=inv3)
+
+
+@pytest.mark.parametrize("name,n", [("halfb_uniform", 700), ("mid", 300)])
+def test_fused_combine_matches_combine_entry_point(name, n):
+    """For l <= 1024 the forward's final GEMM computes RMSNorm(u) itself (the
+    combine fused into its epilogue warps).  Its rows must equal moe_combine on
+    the same expert outputs bit for bit, and every launch must leave the
+    synchronisation area after the workspace header zeroed for the next one."""
+    wl = W[name].with_tokens(n)
+    inp = prepare(wl)
+    dev = device_inputs(inp)
+    y, ids, probs, counts, ws = _run_forward(wl, dev)
+    dims = ldims(wl)
+    v = lm.workspace_views(dims, ws)
+    u2 = torch.empty_like(v["uhat"])
+    lm.moe_combine(dims, v["eo"], v["inv"], probs, dev["rms_weight"], u2)
+    torch.cuda.synchronize()
+    assert torch.equal(u2, v["uhat"])
+    sync = ws[256:256 + 4096].view(torch.int32)
+    assert int(sync.abs().sum().item()) == 0
+    y2, _, _, _, _ = _run_forward(wl, dev, ws)
+    assert torch.equal(y, y2)
