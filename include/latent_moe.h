@@ -246,7 +246,8 @@ LMOE_API lmoe_status latent_moe_backward(const lmoe_dims* dims, const lmoe_weigh
  * x has landed, and its y is copied out on a second library-owned stream while
  * the next chunk computes.  The chunk count comes from a cost model of copy
  * time against forward time (one chunk when streaming the expert weights
- * dominates).  The copy streams and their events are created on the first
+ * dominates; the environment variable LMOE_HOST_CHUNKS=1..8 overrides it).
+ * The copy streams and their events are created on the first
  * call on each device and kept until the process exits; the copies wait for
  * work queued on `stream` before the call, and the call returns after all of
  * it has finished.  Pinned host buffers are needed for the copies to overlap. */

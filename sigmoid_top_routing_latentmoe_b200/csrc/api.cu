@@ -3,6 +3,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -298,6 +299,8 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   ra.P = P; ra.L = Lt; ra.F = F; ra.R = d->n_routed; ra.tiles = tiles; ra.n_mtiles = n_tiles;
   ra.max_tiles = L.max_tiles; ra.beta1 = d->beta1; ra.beta2 = d->beta2;
   ra.pairs = routed_pairs(d) ? 1 : 0;
+  // pairs with a long K (l >= 2048): GEMM1 on 256 x 512 tiles, 256 hidden units each
+  ra.wide = ra.pairs && Lt >= 2048 ? 1 : 0;
   {
     ProfScope ps("expert_gemm1", st);
     if (tc) {
@@ -386,10 +389,13 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
   const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * sizeof(T) <= (16u << 20);
   LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
   LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
-  // For l <= 1024 the combine runs inside the final GEMM (its epilogue warps
-  // write RMSNorm(u) while the K loop goes through the shared experts' blocks);
-  // wider rows get the combine kernel first.
-  const bool fuse_combine = Lt <= 1024 && (N + 255) / 256 <= kSyncWords - 1;
+  // For l <= 1024 and up to 64 MB of expert outputs the combine runs inside
+  // the final GEMM (its epilogue warps write RMSNorm(u) while the K loop goes
+  // through the shared experts' blocks; 0.5b shape: combine + final 34 -> 31 us).
+  // Larger volumes get the combine kernel first: their reads compete with the
+  // final GEMM's own (mid shape, 268 MB: +23 us per step fused).
+  const bool fuse_combine = Lt <= 1024 && (N + 255) / 256 <= kSyncWords - 1 &&
+                            (double)N * k * Lt * sizeof(T) <= 64.0 * (1 << 20);
   if (!fuse_combine) {
     ProfScope ps("combine", st);
     LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, k, Lt, d->rms_eps, uhat, st),
@@ -400,6 +406,8 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
     FinalArgs a{};
     a.hsh = hsh; a.N = N; a.S = S; a.G = G; a.ws_o = (const T*)w->ws_o; a.d = D;
     a.uhat = uhat; a.L = Lt; a.w_up = (const T*)w->w_up; a.y = (T*)y;
+    // wide output rows (d >= 4096) with a long K: 256 x 512 tiles
+    a.wide = D >= 4096 && S * G + Lt >= 4096 ? 1 : 0;
     if (fuse_combine) {
       a.eo = eo; a.inv = inv; a.probs = probs; a.rms_w = w->rms_weight; a.top_k = k;
       a.rms_eps = d->rms_eps; a.sync = at<int32_t>(ws, L.sync);
@@ -545,6 +553,11 @@ static lmoe_status host_pipe(HostPipe** out) {
 // the 0.5b layer takes ~90 us against 122 us for 4096 tokens: small chunks
 // leave most SMs idle).  A chunked plan must beat one chunk by 15 %.
 static int host_chunks(const lmoe_dims* d) {
+  // LMOE_HOST_CHUNKS=c (1..8) overrides the model
+  if (const char* v = getenv("LMOE_HOST_CHUNKS")) {
+    const int c = atoi(v);
+    if (c >= 1 && c <= kMaxHostChunks) return c;
+  }
   const double N = (double)d->n_tokens, es = d->dtype == LMOE_BF16 ? 2.0 : 4.0;
   const double D = d->d, L = d->latent, R = d->n_routed, k = d->top_k, F = d->ff_routed;
   const double SG = (double)d->n_shared * (d->n_shared > 0 ? d->ff_shared : 0);

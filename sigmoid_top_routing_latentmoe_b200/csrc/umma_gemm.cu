@@ -61,8 +61,18 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint64_t WAIT_CAP_NS = 2000000000ull;
 
 // XPASS_F32: the x-pass with fp32 z and shared gate / up pre-activations (no SiTU)
-// XPASS_WIDE: the x-pass on 256 x 512 pair tiles (see Cfg)
-enum Mode { XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3, XPASS_F32 = 4, XPASS_WIDE = 5 };
+// XPASS_WIDE, FINAL_WIDE, ROUTED1_WIDE: those GEMMs on 256 x 512 pair tiles (see Cfg)
+enum Mode {
+  XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3, XPASS_F32 = 4,
+  XPASS_WIDE = 5, FINAL_WIDE = 6, ROUTED1_WIDE = 7
+};
+template <int MODE>
+constexpr bool is_wide() { return MODE == XPASS_WIDE || MODE == FINAL_WIDE || MODE == ROUTED1_WIDE; }
+// the GEMM a mode computes (a wide mode computes its base mode's GEMM)
+template <int MODE>
+constexpr int base_of() {
+  return MODE == XPASS_WIDE ? XPASS : MODE == FINAL_WIDE ? FINAL : MODE == ROUTED1_WIDE ? ROUTED1 : MODE;
+}
 template <int MODE>
 constexpr bool is_xpass() { return MODE == XPASS || MODE == XPASS_F32 || MODE == XPASS_WIDE; }
 
@@ -79,7 +89,7 @@ constexpr bool is_xpass() { return MODE == XPASS || MODE == XPASS_F32 || MODE ==
 //         epilogue, while the TMA ring keeps filling.
 template <int MODE, int CG>
 struct Cfg {
-  static constexpr int W = MODE == XPASS_WIDE ? 2 : 1;
+  static constexpr int W = is_wide<MODE>() ? 2 : 1;
   static constexpr int B_BYTES = (CG == 1 ? 2 : W) * SUB * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB or 32 KB
   static constexpr int STAGES = CG == 1 ? 4 : (W == 2 ? 4 : 6);
@@ -89,7 +99,7 @@ struct Cfg {
   static constexpr int NACC = W == 2 ? 1 : 2;            // accumulator buffers in TMEM
   static constexpr int ACC_STRIDE = TMEM_COLS / NACC;    // columns per buffer
 };
-static_assert(Cfg<XPASS_WIDE, 2>::SMEM_BYTES <= 232448, "wide x-pass exceeds shared memory");
+static_assert(Cfg<XPASS_WIDE, 2>::SMEM_BYTES <= 232448, "wide tiles exceed shared memory");
 
 enum Epi { EPI_Z = 1, EPI_SITU = 3, EPI_STORE = 4 };
 // B sub-tile sources of the x-pass: 0 W_down, 1 W_r, 2 W_g,sh, 3 W_u,sh,
@@ -457,7 +467,7 @@ __device__ __forceinline__ uint32_t instr_desc_cg(int n) {
 // ---------------------------------------------------------- tile decoding
 template <int MODE, int CG>
 __device__ __forceinline__ int total_tiles(const Params& p) {
-  if (is_xpass<MODE>() || MODE == FINAL) return ((p.M + Cfg<MODE, CG>::MT - 1) / Cfg<MODE, CG>::MT) * p.n_tiles;
+  if (is_xpass<MODE>() || base_of<MODE>() == FINAL) return ((p.M + Cfg<MODE, CG>::MT - 1) / Cfg<MODE, CG>::MT) * p.n_tiles;
   return (*p.n_mtiles) * p.n_tiles;
 }
 
@@ -470,15 +480,23 @@ __device__ __forceinline__ Tile<MODE, CG> decode_tile(const Params& p, int t) {
     tl.srows[s] = SUB;
     tl.scol[s] = s * SUB;
   }
-  if (is_xpass<MODE>() || MODE == FINAL) {
+  if (is_xpass<MODE>() || base_of<MODE>() == FINAL) {
     constexpr int MT = Cfg<MODE, CG>::MT;
     const int m_tiles = (p.M + MT - 1) / MT;
     const int mt = t % m_tiles, n = t / m_tiles;
     tl.m0 = mt * MT;
     tl.rows = min(MT, p.M - tl.m0);
-    if (MODE == FINAL) {
+    if (base_of<MODE>() == FINAL) {
       const int n0 = n * p.bn;
-      if (CG == 2) {  // each CTA loads half of the tile's columns
+      if (Cfg<MODE, CG>::W == 2) {  // four 128-row sub-tiles: CTA r loads r and r + 2
+        tl.n_sub = 4;
+#pragma unroll
+        for (int sb = 0; sb < 2 * Cfg<MODE, CG>::W; ++sb) {
+          tl.brow[sb] = n0 + sb * SUB;
+          tl.bmap[sb] = 0;
+        }
+        tl.ncols = 4 * SUB;
+      } else if (CG == 2) {  // each CTA loads half of the tile's columns
         tl.n_sub = 2;
         tl.srows[0] = tl.srows[1] = p.bn / 2;
         tl.scol[1] = p.bn / 2;
@@ -540,8 +558,21 @@ __device__ __forceinline__ Tile<MODE, CG> decode_tile(const Params& p, int t) {
     const int4 e = p.tiles[mt];
     tl.m0 = e.y;
     tl.rows = e.z;
-    tl.bz[0] = tl.bz[1] = e.x;
-    if (MODE == ROUTED1) {
+#pragma unroll
+    for (int sb = 0; sb < 2 * Cfg<MODE, CG>::W; ++sb) tl.bz[sb] = e.x;
+    if (Cfg<MODE, CG>::W == 2) {  // ROUTED1_WIDE: 256 hidden units of expert e
+      // sub-tile 2b: gate rows of block b of W_g,e; 2b + 1: the up rows of W_u,e
+      // (CTA 0 loads the gate sub-tiles, CTA 1 the up ones)
+      tl.n_sub = 4;
+#pragma unroll
+      for (int sb = 0; sb < 2 * Cfg<MODE, CG>::W; ++sb) {
+        tl.bmap[sb] = sb & 1;
+        tl.brow[sb] = n * 2 * SUB + (sb >> 1) * SUB;
+      }
+      tl.epi = EPI_SITU;
+      tl.ocol = n * 2 * SUB;
+      tl.ncols = 4 * SUB;
+    } else if (base_of<MODE>() == ROUTED1) {
       // gate rows of W_g,e and the matching up rows of W_u,e (CG = 2: CTA 0
       // loads the gate half, CTA 1 the up half)
       tl.n_sub = 2;
@@ -580,7 +611,7 @@ __device__ __forceinline__ Tile<MODE, CG> decode_tile(const Params& p, int t) {
 
 template <int MODE>
 __device__ __forceinline__ int k_blocks(const Params& p) {
-  return MODE == FINAL ? p.S * p.kb0 + p.kb1 : p.kb0;
+  return base_of<MODE>() == FINAL ? p.S * p.kb0 + p.kb1 : p.kb0;
 }
 
 __device__ __forceinline__ const CUtensorMap* bmap_ptr(const Params& p, int i) {
@@ -629,7 +660,7 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
     const int arow = tl.m0 + (CG == 2 ? BM * (int)rank : 0);
     // A routed pair tile of <= 128 rows has none in CTA 1: it loads no A there
     // (its accumulator rows are never stored) and the leader expects fewer bytes.
-    constexpr bool kRoutedPair = CG == 2 && (MODE == ROUTED1 || MODE == ROUTED2);
+    constexpr bool kRoutedPair = CG == 2 && (base_of<MODE>() == ROUTED1 || MODE == ROUTED2);
     int a_ctas = CG;
     if constexpr (kRoutedPair) a_ctas = tl.rows <= BM ? 1 : 2;
     const bool load_a = CG == 1 || !kRoutedPair || (int)rank < a_ctas;
@@ -649,7 +680,7 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
     const CUtensorMap* map_b = bmap_ptr(p, mb);
     const uint32_t off_b = SUB * BK * 2;  // the second sub-tile's B offset
     for (int kb = 0; kb < nkb; ++kb) {
-      if (MODE == FINAL && p.fuse_combine && kb == p.S * p.kb0) {
+      if (base_of<MODE>() == FINAL && p.fuse_combine && kb == p.S * p.kb0) {
         // the uhat rows of this tile are written by the kernel's own epilogue warps
         if (!wait_count(p.c_sync + tl.m0 / Cfg<MODE, CG>::MT, tl.rows, abort_flag, p.status)) {
           ok = false;
@@ -665,20 +696,20 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
       const uint32_t own_bar = full0 + 8 * stage;
       const uint32_t bar = full0_leader + 8 * stage;
       if (CG == 1 || rank == 0) mbar_expect_tx(own_bar, tx_bytes);
-      if (MODE == FINAL) {
+      if (base_of<MODE>() == FINAL) {
         const int kb_sh = p.S * p.kb0;
         if (kb < kb_sh) {
           const int j = kb / p.kb0, kk = (kb % p.kb0) * BK;
           if (CG == 1) tma_load_2d(a_dst, &p.tmA0, bar, j * p.G + kk, arow);
           else tma2_load_2d(a_dst, &p.tmA0, bar, j * p.G + kk, arow);
           load_b<CG>(b_dst, sa == 0 ? &p.tmB0 : &p.tmB2, true, bar, kk, row_a, j);
-          if (CG == 1 && two) load_b<CG>(b_dst + off_b, &p.tmB2, true, bar, kk, row_b, j);
+          if (two) load_b<CG>(b_dst + off_b, &p.tmB2, true, bar, kk, row_b, j);
         } else {
           const int kk = (kb - kb_sh) * BK;
           if (CG == 1) tma_load_2d(a_dst, &p.tmA1, bar, kk, arow);
           else tma2_load_2d(a_dst, &p.tmA1, bar, kk, arow);
           load_b<CG>(b_dst, sa == 0 ? &p.tmB1 : &p.tmB3, false, bar, kk, row_a, 0);
-          if (CG == 1 && two) load_b<CG>(b_dst + off_b, &p.tmB3, false, bar, kk, row_b, 0);
+          if (two) load_b<CG>(b_dst + off_b, &p.tmB3, false, bar, kk, row_b, 0);
         }
       } else {
         const int kk = kb * BK;
@@ -930,7 +961,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
   const int lane = threadIdx.x & 31;
   const int wrow = ew * 32 + (CG == 2 ? BM * (int)rank : 0);  // first tile row of this warp
   const SituConsts sk = situ_consts(p);
-  if (MODE == FINAL && p.fuse_combine) {
+  if (base_of<MODE>() == FINAL && p.fuse_combine) {
     // The fused combine: uhat rows of an even share per CTA, one warp per row,
     // each row counted in its 256-row tile's word once written.  Runs while the
     // first tile's K loop goes through the shared experts' blocks.
@@ -979,7 +1010,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
         out = static_cast<__nv_bfloat16*>(p.out0);
         ld = p.ld0;
       }
-      if (MODE == XPASS_WIDE) {
+      if (Cfg<MODE, CG>::W == 2) {
         // blocks of 64 hidden units b (of 4): gate columns 256 (b / 2) + 64 (b % 2),
         // up columns 128 further
 #pragma unroll 1
@@ -1080,7 +1111,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
     } else {
       // FINAL / ROUTED2: accumulator columns [0, ncols) are output columns
       // [ocol, ocol + ncols); this warp writes the 64-column blocks h0, h0 + HS, ...
-      const int width = (MODE == FINAL ? p.d : p.L) - tl.ocol;
+      const int width = (base_of<MODE>() == FINAL ? p.d : p.L) - tl.ocol;
       const int ncols = min(tl.ncols, width);
 #pragma unroll 1
       for (int cb = h0; cb * 64 < ncols; cb += HS) {
@@ -1185,7 +1216,7 @@ __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_cons
   __syncthreads();
   if (CG == 2) cluster_sync();  // neither CTA frees TMEM or exits while its pair still works
   tc_fence_after();
-  if (MODE == FINAL && p.fuse_combine && threadIdx.x == 0) {
+  if (base_of<MODE>() == FINAL && p.fuse_combine && threadIdx.x == 0) {
     // the last CTA to finish (every CTA is past its waits) zeroes the counts
     // for the next launch
     __threadfence();
@@ -1413,8 +1444,9 @@ cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
   Params p = base_params(status);
   const int m_tiles = (int)((a.N + 2 * BM - 1) / (2 * BM));
   const int units = a.max_units > 0 ? std::min(a.max_units, num_sms() / 2) : num_sms() / 2;
-  p.bn = pick_bn(m_tiles, a.d, units);
-  const uint32_t hb = p.bn / 2;  // rows of B each CTA of the pair loads
+  // wide: 256 x 512 tiles, each CTA loading two 128-row B sub-tiles
+  p.bn = a.wide ? 4 * SUB : pick_bn(m_tiles, a.d, units);
+  const uint32_t hb = a.wide ? SUB : p.bn / 2;  // rows of each B box a CTA loads
   bool ok = make_map(&p.tmA1, a.uhat, a.L, a.N, 1, BM) && make_map(&p.tmB1, a.w_up, a.L, a.d, 1, hb) &&
             make_map(&p.tmB3, a.w_up, a.L, a.d, 1, hb);
   if (a.S > 0)
@@ -1448,7 +1480,8 @@ cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
     if (nvec > 128 || m_tiles > kSyncWords - 1) return cudaErrorInvalidValue;
   }
   const int total = m_tiles * p.n_tiles;
-  return launch<FINAL, 2>(p, std::min(total, units), st);
+  return a.wide ? launch<FINAL_WIDE, 2>(p, std::min(total, units), st)
+                : launch<FINAL, 2>(p, std::min(total, units), st);
 }
 
 cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) {
@@ -1462,7 +1495,8 @@ cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   p.L = a.L;
   p.F = a.F;
   p.R = a.R;
-  p.n_tiles = (a.F + SUB - 1) / SUB;
+  const bool wide = a.wide && a.pairs;  // 256 hidden units per tile (pairs only)
+  p.n_tiles = wide ? (a.F + 2 * SUB - 1) / (2 * SUB) : (a.F + SUB - 1) / SUB;
   p.out0 = a.out;
   p.ld0 = a.F;
   p.tiles = a.tiles;
@@ -1477,6 +1511,7 @@ cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) 
   const int cap = num_sms() / cg;
   const int units = a.max_units > 0 ? std::min(a.max_units, cap) : cap;
   const int grid = (int)std::min<int64_t>(bound, units);
+  if (wide) return launch<ROUTED1_WIDE, 2>(p, grid, st);
   return a.pairs ? launch<ROUTED1, 2>(p, grid, st) : launch<ROUTED1, 1>(p, grid, st);
 }
 

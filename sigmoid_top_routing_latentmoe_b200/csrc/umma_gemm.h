@@ -59,6 +59,7 @@ struct FinalArgs {
   const __nv_bfloat16* w_up;  // [d, L]
   __nv_bfloat16* y;
   int max_units;  // at most this many CTA pairs (0: one per pair of SMs)
+  int wide;       // 1: 256 x 512 tiles (two N = 256 MMAs per K step, one accumulator)
   // Fused combine (eo != nullptr, L <= 1024): the kernel's epilogue warps first
   // write uhat = RMSNorm(sum_i probs[t, i] eo[inv[t, i]]) * rms_w for an even
   // share of the rows (the combine kernel's arithmetic), counting finished rows
@@ -91,6 +92,8 @@ struct RoutedArgs {
   // 0: single CTAs over row tiles of <= 128.  The tile list must have been
   // built with the matching height (kRoutedPairTileM or kTileM).
   int pairs;
+  // GEMM1 with pairs: 1 = tiles of 256 hidden units (256 x 512 accumulator).
+  int wide;
 };
 
 cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st);

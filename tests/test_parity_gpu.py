@@ -432,3 +432,31 @@ def test_fused_combine_matches_combine_entry_point(name, n):
     assert int(sync.abs().sum().item()) == 0
     y2, _, _, _, _ = _run_forward(wl, dev, ws)
     assert torch.equal(y, y2)
+
+
+def test_wide_routed_gemm_parity():
+    """Routed experts at the K3 latent width (l = 3584) with 64..256 rows per
+    expert: CTA pairs and 256 x 512 tiles of 256 hidden units for GEMM1.
+    moe_expert_ffn on the oracle's z and permutation, every 8th sorted row
+    against the oracle's SiTU expert (bf16 tolerance of the forward)."""
+    wl = W["k3_width"].with_tokens(512).replace(n_routed=16, top_k=4)
+    inp = prepare(wl)
+    ow = oracle_weights(inp)
+    ref = oracle.forward(odims(wl), ow, synth.to_f32(inp["x"]), want=("z",))
+    counts, offsets, perm, inv = oracle.permute(ref["ids"], wl.n_routed)
+    assert (counts >= 64).all() and (counts <= 256).all()
+    z = round_act(ref["z"], wl)
+    P = wl.n_tokens * wl.top_k
+    dims = ldims(wl)
+    ws = lm.alloc_workspace(dims)
+    dev = device_inputs({k: inp[k] for k in ("w_g", "w_u", "w_o")})
+    eo = torch.empty(P, wl.latent, dtype=torch.bfloat16, device="cuda")
+    lm.moe_expert_ffn(dims, torch.from_numpy(z).to("cuda", torch.bfloat16), to_device(perm, ""),
+                      to_device(offsets, ""), dev["w_g"], dev["w_u"], dev["w_o"], eo, ws)
+    torch.cuda.synchronize()
+    assert lm.get_device_status(ws) == lm.OK
+    rows = np.arange(0, P, 8)
+    expert = np.searchsorted(offsets, rows, side="right") - 1
+    exp_eo = np.stack([oracle.situ(ow["w_g"][e], ow["w_u"][e], ow["w_o"][e], z[perm[r]],
+                                   wl.beta1, wl.beta2)[0] for r, e in zip(rows, expert)])
+    assert rel_err(host(eo)[rows], exp_eo) <= 2e-2
