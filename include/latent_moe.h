@@ -199,7 +199,12 @@ LMOE_API lmoe_status moe_router_losses(const lmoe_dims* dims, const float* logit
 /* The whole layer: y [N, d] = s_sh + W_up RMSNorm(u).  Optional outputs (NULL
  * to skip): ids_out [N, k], probs_out [N, k], counts_out [R].  All work is on
  * `stream`; no host synchronisation.  The router logits stay in the
- * workspace for moe_router_losses. */
+ * workspace for moe_router_losses.  Results are bitwise repeatable for given
+ * dims on a given GPU.  When whole output tiles would fill the SMs' last wave
+ * below 90%, the final GEMM (bf16) splits the K loop of some tiles between
+ * CTA pairs (stream-K) and adds the fp32 partials in a fixed order; the
+ * environment variable LMOE_STREAM_K=0 turns that off, =1 uses it whenever
+ * its scratch fits. */
 LMOE_API lmoe_status latent_moe_forward(const lmoe_dims* dims, const lmoe_weights* weights, const void* x,
                                void* y, int32_t* ids_out, float* probs_out, int32_t* counts_out,
                                void* ws, size_t ws_bytes, lmoe_stream stream);
@@ -240,8 +245,10 @@ LMOE_API lmoe_status latent_moe_backward(const lmoe_dims* dims, const lmoe_weigh
  * waits for the stream.  Weights and workspace are device memory.  The
  * workspace must be lmoe_workspace_size_host(dims) bytes (it also holds the
  * device copies of x and y).
- * The tokens may be processed in up to 8 chunks (tokens are independent, so y
- * is bit-identical to one latent_moe_forward over all N): x chunks are copied
+ * The tokens may be processed in up to 8 chunks (tokens are independent; y
+ * equals one latent_moe_forward over all N to within the final GEMM's fp32
+ * summation order, which may split K differently per chunk size, and is
+ * bit-identical when one chunk is used): x chunks are copied
  * in on a library-owned stream, each chunk's forward runs on `stream` once its
  * x has landed, and its y is copied out on a second library-owned stream while
  * the next chunk computes.  The chunk count comes from a cost model of copy
@@ -259,8 +266,10 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
 /* Byte offsets of the forward's intermediates inside the workspace, for
  * inspection after latent_moe_forward: offsets[0..6] = z [N,l], router logits
  * [N, ld] fp32, shared hidden units [N, S*G], RMSNorm(u) [N,l], routed expert
- * outputs [N*k, l], routed hidden units [N*k, F], sorted z rows [N*k, l];
- * offsets[7] = ld, the row stride (elements) of the logits.  With n >= 11
+ * outputs [N*k, l], routed hidden units [N*k, F], sorted z rows [N*k, l]
+ * (these two hold the final GEMM's stream-K scratch instead when it splits
+ * K, see latent_moe_forward); offsets[7] = ld, the row stride (elements) of
+ * the logits.  With n >= 11
  * also offsets[8..10] = the permutation the forward built: expert offsets
  * [R+1], perm_token [N*k] and inv_pair [N,k], all int32.  n < 8 is EINVAL. */
 LMOE_API lmoe_status lmoe_workspace_layout(const lmoe_dims* dims, size_t* offsets, int32_t n);

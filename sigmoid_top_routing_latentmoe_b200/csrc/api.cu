@@ -133,10 +133,11 @@ static lmoe_status check_dims(const lmoe_dims* d) {
 
 // ------------------------------------------------------------ workspace
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+constexpr int kSkMaxPairs = 80;  // CTA pairs the stream-K scratch is sized for
 
 struct Layout {
   size_t header, sync, z, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, zp, h,
-      eo, hsh, uhat, loss, x, y, total;
+      skx, eo, hsh, uhat, loss, x, y, total;
   int64_t logits_ld;
   int max_tiles;
 };
@@ -164,6 +165,15 @@ static Layout layout(const lmoe_dims* d, bool host_copies) {
   L.tiles = take((size_t)L.max_tiles * sizeof(int4));
   L.zp = take((size_t)P * d->latent * es);
   L.h = take((size_t)P * d->ff_routed * es);
+  // The final GEMM's stream-K partials reuse [zp, eo), dead by then; this
+  // tops it up to one 256-row tile of fp32 per CTA pair (up to kSkMaxPairs).
+  if (d->dtype == LMOE_BF16) {
+    const size_t bn_max = d->d >= 4096 ? 512 : 256;
+    const size_t need = (size_t)kSkMaxPairs * 2 * 128 * bn_max * 4, have = off - L.zp;
+    L.skx = take(need > have ? need - have : 0);
+  } else {
+    L.skx = take(0);
+  }
   L.eo = take((size_t)P * d->latent * es);
   L.hsh = take((size_t)N * d->n_shared * (size_t)d->ff_shared * es);
   L.uhat = take((size_t)N * d->latent * es);
@@ -329,6 +339,16 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   return LMOE_OK;
 }
 
+// Stream-K for the final GEMM: chosen by the wave fill unless LMOE_STREAM_K
+// is 0 (never) or 1 (whenever its scratch fits).
+static int stream_k_mode() {
+  if (const char* v = getenv("LMOE_STREAM_K")) {
+    if (v[0] == '0') return 0;
+    if (v[0] == '1') return 1;
+  }
+  return -1;
+}
+
 // The x-pass uses 256 x 512 tiles (no accumulator double-buffering, 1.33x the
 // FLOPs per streamed byte) when K = d is long enough for the main loop to hide
 // the epilogue: d >= 2048 (mid shape -8 %, K3 width -17 %; +3 % at d = 768).
@@ -410,8 +430,14 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
     a.wide = D >= 4096 && S * G + Lt >= 4096 ? 1 : 0;
     if (fuse_combine) {
       a.eo = eo; a.inv = inv; a.probs = probs; a.rms_w = w->rms_weight; a.top_k = k;
-      a.rms_eps = d->rms_eps; a.sync = at<int32_t>(ws, L.sync);
+      a.rms_eps = d->rms_eps;
     }
+    a.sync = at<int32_t>(ws, L.sync);
+    // stream-K partials go to the sorted z copy and the routed hidden units,
+    // both dead once the routed GEMMs are done
+    a.sk_part = at<float>(ws, L.zp);
+    a.sk_bytes = L.eo - L.zp;
+    a.stream_k = stream_k_mode();
     ProfScope ps("final", st);
     LMOE_CUDA(umma_final(a, status, st), "final (tcgen05)");
   }
@@ -551,7 +577,10 @@ static lmoe_status host_pipe(HostPipe** out) {
 // experts' max(FLOPs at 0.8 PFLOP/s, weights of the experts the chunk selects
 // at 6 TB/s) plus 60 us of launch latency and tile tails (a 1024-token chunk of
 // the 0.5b layer takes ~90 us against 122 us for 4096 tokens: small chunks
-// leave most SMs idle).  A chunked plan must beat one chunk by 15 %.
+// leave most SMs idle).  A chunked plan must beat one chunk by 15 %, and of
+// the counts within 3 % of the best estimate the smallest is taken (measured:
+// 0.5b shape 2 chunks 12.0 M tokens/s against 10.8 M for one and 9.7 M for
+// four; mid shape 4 chunks 6.5 M, 7 chunks 6.2 M, one 4.0 M).
 static int host_chunks(const lmoe_dims* d) {
   // LMOE_HOST_CHUNKS=c (1..8) overrides the model
   if (const char* v = getenv("LMOE_HOST_CHUNKS")) {
@@ -566,8 +595,9 @@ static int host_chunks(const lmoe_dims* d) {
   const double w_expert = 3 * F * L * es;
   const double copy_bw = 50e9, flop_rate = d->dtype == LMOE_BF16 ? 0.8e15 : 2.0e13,
                hbm = 6.0e12, fixed = 60e-6;
-  double t1 = 0.0, best = 0.0;
-  int best_c = 1;
+  double est[kMaxHostChunks + 1] = {0.0};
+  int n_c = 0;
+  double best = 0.0;
   for (int c = 1; c <= kMaxHostChunks; ++c) {
     const double n = std::ceil(N / c);
     if (c > 1 && n < 256) break;
@@ -575,14 +605,13 @@ static int host_chunks(const lmoe_dims* d) {
     const double t_copy = n * D * es / copy_bw;
     const double t_fwd = n * dense_tok / flop_rate +
                          std::max(n * routed_tok / flop_rate, used * w_expert / hbm) + fixed;
-    const double t = 2 * t_copy + c * std::max(t_copy, t_fwd);
-    if (c == 1) t1 = t;
-    if (c == 1 || (t < best && t < 0.85 * t1)) {
-      best = t;
-      best_c = c;
-    }
+    est[c] = 2 * t_copy + c * std::max(t_copy, t_fwd);
+    n_c = c;
+    if (c == 1 || (est[c] < best && est[c] < 0.85 * est[1])) best = est[c];
   }
-  return best_c;
+  for (int c = 1; c <= n_c; ++c)
+    if (est[c] <= 1.03 * best && (c == 1 || est[c] < 0.85 * est[1])) return c;
+  return 1;
 }
 
 }  // namespace lmoe

@@ -140,6 +140,11 @@ struct Params {
   int32_t* c_sync;
   int c_k, c_vpl, fuse_combine;
   float c_eps;
+  // FINAL with stream-K scheduling: each unit (CTA pair) takes an equal share
+  // of the tiles' K-block iterations; see next_work and the epilogue
+  int stream_k;
+  float* sk_part;     // [units][2 ranks][4 lane quarters][bn / 64][16][32] float4 partials
+  int32_t* sk_flags;  // [units] warps that stored the unit's partial
 };
 
 template <int NS>  // at most NS B sub-tiles
@@ -614,6 +619,60 @@ __device__ __forceinline__ int k_blocks(const Params& p) {
   return base_of<MODE>() == FINAL ? p.S * p.kb0 + p.kb1 : p.kb0;
 }
 
+// The work of one unit (a CTA or CTA pair): K blocks [kb0, kb1) of tile t.
+// Plain scheduling gives a unit whole tiles unit, unit + n_units, ...; stream-K
+// (FINAL, p.stream_k) gives it the iterations [u Q / U, (u + 1) Q / U) of the
+// Q = tiles x K-blocks iterations, in order, so a tile can be split between
+// consecutive units.  All three roles walk the same sequence.
+struct Work {
+  int t, kb0, kb1;
+};
+struct WorkIter {
+  int64_t cur, end;
+  int nkb, step;
+  bool sk;
+};
+template <int MODE, int CG>
+__device__ __forceinline__ WorkIter work_begin(const Params& p, int unit, int n_units) {
+  WorkIter it;
+  it.nkb = k_blocks<MODE>(p);
+  it.sk = base_of<MODE>() == FINAL && p.stream_k;
+  const int64_t total = total_tiles<MODE, CG>(p);
+  if (it.sk) {
+    const int64_t q = total * it.nkb;
+    it.cur = q * unit / n_units;
+    it.end = q * (unit + 1) / n_units;
+    it.step = 0;
+  } else {
+    it.cur = unit;
+    it.end = total;
+    it.step = n_units;
+  }
+  return it;
+}
+__device__ __forceinline__ bool work_next(WorkIter& it, Work& w) {
+  if (it.cur >= it.end) return false;
+  if (!it.sk) {
+    w.t = (int)it.cur;
+    w.kb0 = 0;
+    w.kb1 = it.nkb;
+    it.cur += it.step;
+    return true;
+  }
+  w.t = (int)(it.cur / it.nkb);
+  w.kb0 = (int)(it.cur - (int64_t)w.t * it.nkb);
+  w.kb1 = (int)min((int64_t)it.nkb, w.kb0 + (it.end - it.cur));
+  it.cur += w.kb1 - w.kb0;
+  return true;
+}
+// Stream-K: the unit whose share holds iteration i.
+__device__ __forceinline__ int sk_unit_of(int64_t i, int64_t q, int n_units) {
+  int u = (int)((i * n_units) / q);
+  while (u + 1 < n_units && q * (u + 1) / n_units <= i) ++u;
+  while (u > 0 && q * u / n_units > i) --u;
+  return u;
+}
+
 __device__ __forceinline__ const CUtensorMap* bmap_ptr(const Params& p, int i) {
   return i == 0 ? &p.tmB0 : i == 1 ? &p.tmB1 : i == 2 ? &p.tmB2 : &p.tmB3;
 }
@@ -649,14 +708,14 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
   int stage = 0;
   uint32_t phase = 0;
   uint32_t issued = 0, issued_phase = 0;  // bit s: stage s was filled; its phase
-  const int total = total_tiles<MODE, CG>(p);
-  const int nkb = k_blocks<MODE>(p);
   const uint32_t ring0 = smem_u32(ring);
   const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
   const uint32_t full0_leader = CG == 1 ? full0 : map_to_rank(full0, 0);
   bool ok = true;
-  for (int t = unit; t < total && ok; t += n_units) {
-    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, t);
+  WorkIter wi = work_begin<MODE, CG>(p, unit, n_units);
+  Work wk;
+  while (ok && work_next(wi, wk)) {
+    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, wk.t);
     const int arow = tl.m0 + (CG == 2 ? BM * (int)rank : 0);
     // A routed pair tile of <= 128 rows has none in CTA 1: it loads no A there
     // (its accumulator rows are never stored) and the leader expects fewer bytes.
@@ -679,9 +738,10 @@ __device__ __forceinline__ void produce(const Params& p, uint8_t* ring, uint64_t
     const CUtensorMap* map_a = bmap_ptr(p, ma);
     const CUtensorMap* map_b = bmap_ptr(p, mb);
     const uint32_t off_b = SUB * BK * 2;  // the second sub-tile's B offset
-    for (int kb = 0; kb < nkb; ++kb) {
-      if (base_of<MODE>() == FINAL && p.fuse_combine && kb == p.S * p.kb0) {
-        // the uhat rows of this tile are written by the kernel's own epilogue warps
+    for (int kb = wk.kb0; kb < wk.kb1; ++kb) {
+      if (base_of<MODE>() == FINAL && p.fuse_combine && kb == max(p.S * p.kb0, wk.kb0)) {
+        // the uhat rows of this tile are written by the kernel's own epilogue
+        // warps (checked before this unit's first uhat K block of the tile)
         if (!wait_count(p.c_sync + tl.m0 / Cfg<MODE, CG>::MT, tl.rows, abort_flag, p.status)) {
           ok = false;
           break;
@@ -749,16 +809,16 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
   uint32_t phase = 0;
   int acc = 0;
   uint32_t acc_phase = 0;
-  const int total = total_tiles<MODE, CG>(p);
-  const int nkb = k_blocks<MODE>(p);
   bool ok = true;
-  for (int t = unit; t < total && ok; t += n_units) {
-    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, t);
+  WorkIter wi = work_begin<MODE, CG>(p, unit, n_units);
+  Work wk;
+  while (ok && work_next(wi, wk)) {
+    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, wk.t);
     const uint32_t idesc = instr_desc_cg<CG>(tl.ncols / C::W);
     if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, p.status)) break;
     tc_fence_after();
     const uint32_t d_tmem = tmem + acc * C::ACC_STRIDE;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = wk.kb0; kb < wk.kb1; ++kb) {
       if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.status)) {
         ok = false;
         break;
@@ -768,7 +828,7 @@ __device__ __forceinline__ void mma_issue(const Params& p, uint8_t* ring, uint64
       const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
       for (int k = 0; k < BK / 16; ++k) {
-        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+        const uint32_t accum = (kb > wk.kb0 || k > 0) ? 1u : 0u;
 #pragma unroll
         for (int w = 0; w < C::W; ++w) {  // W = 2: columns [256 w, 256 w + 256) from B block w
           const uint32_t bw = b_addr + w * SUB * BK * 2 + k * 32;
@@ -985,9 +1045,26 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
   }
   int acc = 0;
   uint32_t acc_phase = 0;
-  const int total = total_tiles<MODE, CG>(p);
-  for (int t = unit; t < total; t += n_units) {
-    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, t);
+  const int nkb = k_blocks<MODE>(p);
+  const int64_t q_sk = (int64_t)total_tiles<MODE, CG>(p) * nkb;  // stream-K iterations
+  WorkIter wi = work_begin<MODE, CG>(p, unit, n_units);
+  Work wk;
+  while (work_next(wi, wk)) {
+    const Tile<MODE, CG> tl = decode_tile<MODE, CG>(p, wk.t);
+    // Stream-K (FINAL): a unit that holds K blocks after the first of a tile
+    // stores its fp32 partial (role 1) and counts its warps in sk_flags; the
+    // unit that holds the tile's first K blocks (role 2) works on them last,
+    // waits for the partials of the units after it that hold the rest, and
+    // adds them in unit order before the epilogue: a fixed summation order.
+    int sk_role = 0, sk_last = unit;
+    if (base_of<MODE>() == FINAL && p.stream_k) {
+      if (wk.kb0 > 0) {
+        sk_role = 1;
+      } else if (wk.kb1 < nkb) {
+        sk_role = 2;
+        sk_last = sk_unit_of((int64_t)wk.t * nkb + nkb - 1, q_sk, n_units);
+      }
+    }
     if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.status)) break;
     tc_fence_after();
     const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * Cfg<MODE, CG>::ACC_STRIDE;
@@ -1113,17 +1190,54 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
       // [ocol, ocol + ncols); this warp writes the 64-column blocks h0, h0 + HS, ...
       const int width = (base_of<MODE>() == FINAL ? p.d : p.L) - tl.ocol;
       const int ncols = min(tl.ncols, width);
+      bool waited = true;
+      if (sk_role == 2 && lane == 0)  // the partials of units unit + 1 .. sk_last
+        for (int u2 = unit + 1; u2 <= sk_last && waited; ++u2)
+          waited = wait_count(p.sk_flags + u2, CG * EPI_WARPS, abort_flag, p.status);
+      waited = __shfl_sync(0xffffffffu, (int)waited, 0) != 0;
+      __syncwarp();  // lane 0's acquire orders the other lanes' partial reads
+      const int nblk = p.bn / 64;
 #pragma unroll 1
-      for (int cb = h0; cb * 64 < ncols; cb += HS) {
+      for (int cb = h0; waited && cb * 64 < ncols; cb += HS) {
         const int cols = min(64, ncols - cb * 64);
         const int64_t col = tl.ocol + cb * 64;
         float a[32], b[32];
         tc_ld32x2(tbase + cb * 64, a, tbase + cb * 64 + 32, b);
+        if (sk_role != 0) {
+          // partial blocks: [unit][rank][lane quarter][64-column block][16 float4][32 lanes]
+          auto part = [&](int u) {
+            return reinterpret_cast<float4*>(p.sk_part) +
+                   ((((size_t)u * 2 + rank) * 4 + ew) * nblk + cb) * 16 * 32 + lane;
+          };
+          if (sk_role == 1) {
+            float4* dst = part(unit);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              dst[j * 32] = make_float4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
+              dst[(8 + j) * 32] = make_float4(b[4 * j], b[4 * j + 1], b[4 * j + 2], b[4 * j + 3]);
+            }
+            continue;
+          }
+          for (int u2 = unit + 1; u2 <= sk_last; ++u2) {
+            const float4* src = part(u2);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 pa = __ldcg(src + j * 32), pb = __ldcg(src + (8 + j) * 32);
+              a[4 * j] += pa.x; a[4 * j + 1] += pa.y; a[4 * j + 2] += pa.z; a[4 * j + 3] += pa.w;
+              b[4 * j] += pb.x; b[4 * j + 1] += pb.y; b[4 * j + 2] += pb.z; b[4 * j + 3] += pb.w;
+            }
+          }
+        }
         uint32_t w[32];
         pack_block(a, b, w);
         warp_store_bf16(stage, w, static_cast<__nv_bfloat16*>(p.out0) + grow0 * p.ld0 + col,
                         p.ld0, rows, cols);
       }
+    }
+    if (sk_role == 1) {  // every warp counts, whether or not it had rows to store
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicAdd(p.sk_flags + unit, 1);
     }
     tc_fence_before();
     __syncwarp();
@@ -1216,13 +1330,17 @@ __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_cons
   __syncthreads();
   if (CG == 2) cluster_sync();  // neither CTA frees TMEM or exits while its pair still works
   tc_fence_after();
-  if (base_of<MODE>() == FINAL && p.fuse_combine && threadIdx.x == 0) {
+  if (base_of<MODE>() == FINAL && (p.fuse_combine || p.stream_k) && threadIdx.x == 0) {
     // the last CTA to finish (every CTA is past its waits) zeroes the counts
-    // for the next launch
+    // and flags for the next launch
     __threadfence();
     if (atomicAdd(p.c_sync + (kSyncWords - 1), 1) == (int)gridDim.x - 1) {
-      const int n_mt = (p.M + C::MT - 1) / C::MT;
-      for (int i = 0; i < n_mt; ++i) atomicExch(p.c_sync + i, 0);
+      if (p.fuse_combine) {
+        const int n_mt = (p.M + C::MT - 1) / C::MT;
+        for (int i = 0; i < n_mt; ++i) atomicExch(p.c_sync + i, 0);
+      }
+      if (p.stream_k)
+        for (int i = 0; i < n_units; ++i) atomicExch(p.sk_flags + i, 0);
       atomicExch(p.c_sync + (kSyncWords - 1), 0);
     }
   }
@@ -1480,8 +1598,27 @@ cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
     if (nvec > 128 || m_tiles > kSyncWords - 1) return cudaErrorInvalidValue;
   }
   const int total = m_tiles * p.n_tiles;
-  return a.wide ? launch<FINAL_WIDE, 2>(p, std::min(total, units), st)
-                : launch<FINAL, 2>(p, std::min(total, units), st);
+  int grid = std::min(total, units);
+  // Stream-K where whole tiles fill the last wave below 90% (and every pair
+  // still gets >= 8 K blocks): the pairs' flags sit after the combine's counts.
+  // Not with the fused combine: a pair's first share is the tail of a tile,
+  // whose uhat K blocks then wait for the combine rows at once instead of
+  // after the shared experts' blocks (0.5b shape: final 35 -> 51 us).
+  const int64_t iters = (int64_t)total * (p.S * p.kb0 + p.kb1);
+  const int waves = (total + units - 1) / units;
+  const bool sk_fits = a.sk_part != nullptr && a.sync != nullptr &&
+                       (size_t)units * 2 * BM * p.bn * 4 <= a.sk_bytes &&
+                       (p.fuse_combine ? m_tiles : 0) + units <= kSyncWords - 1;
+  const bool sk_pays =
+      !p.fuse_combine && (double)total < 0.9 * waves * units && iters >= 8LL * units;
+  if (sk_fits && (a.stream_k == 1 || (a.stream_k < 0 && sk_pays))) {
+    p.stream_k = 1;
+    p.sk_part = a.sk_part;
+    p.sk_flags = a.sync + (kSyncWords - 1 - units);
+    p.c_sync = a.sync;  // its last word counts finished CTAs for the flags' reset
+    grid = (int)std::min<int64_t>(units, iters);  // every pair holds >= 1 iteration
+  }
+  return a.wide ? launch<FINAL_WIDE, 2>(p, grid, st) : launch<FINAL, 2>(p, grid, st);
 }
 
 cudaError_t umma_routed1(const RoutedArgs& a, int32_t* status, cudaStream_t st) {

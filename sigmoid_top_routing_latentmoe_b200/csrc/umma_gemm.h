@@ -72,6 +72,14 @@ struct FinalArgs {
   int top_k;
   float rms_eps;
   int32_t* sync;            // kSyncWords zeroed words (left zeroed)
+  // Stream-K: when whole tiles would leave a late wave part-empty, each CTA
+  // pair takes an equal share of the tiles x K-blocks iterations; a tile split
+  // between pairs is summed in fp32 through sk_part (sk_bytes long, scratch)
+  // by the pair holding its first K blocks.  Flags live in sync[].
+  // stream_k: -1 chooses by the wave fill, 0 never, 1 whenever sk_part fits.
+  float* sk_part;
+  size_t sk_bytes;
+  int stream_k;
 };
 
 // routed GEMM1: h [P, F] = SiTU(zp W_g,e^T, zp W_u,e^T) per row tile of expert e

@@ -434,6 +434,33 @@ def test_fused_combine_matches_combine_entry_point(name, n):
     assert torch.equal(y, y2)
 
 
+@pytest.mark.parametrize("name,n,mode", [("k3_width", 320, None), ("halfb_uniform", 300, "1"),
+                                         ("mid", 136, "1"), ("halfb_uniform", 4096, "1")])
+def test_stream_k_final_gemm(name, n, mode, monkeypatch):
+    """Stream-K final GEMM: the CTA pairs share the tiles x K-blocks iterations
+    and a tile split between pairs is summed in fp32 in a fixed order.  At the
+    K3 width with 320 tokens (14 tiles of 256 x 512) it is the default;
+    LMOE_STREAM_K=1 forces it, here also together with the fused combine.
+    y against the oracle on sampled rows, bitwise repeatable, within bf16
+    rounding of the whole-tile schedule (LMOE_STREAM_K=0) and not equal to it
+    everywhere (the split path ran), with the flags left zeroed."""
+    wl = W[name].with_tokens(n)
+    inp = prepare(wl)
+    dev = device_inputs(inp)
+    if mode is not None:
+        monkeypatch.setenv("LMOE_STREAM_K", mode)
+    y, ids, probs, _, ws = _run_forward(wl, dev)
+    _compare_forward(wl, inp, y, ids, probs, rows=np.arange(0, n, max(1, n // 128)))
+    sync = ws[256:256 + 4096].view(torch.int32)
+    assert int(sync.abs().sum().item()) == 0
+    y2, _, _, _, _ = _run_forward(wl, dev, ws)
+    assert torch.equal(y, y2)
+    monkeypatch.setenv("LMOE_STREAM_K", "0")
+    y0, _, _, _, _ = _run_forward(wl, dev, ws)
+    assert rel_err(host(y), host(y0)) <= 1e-2
+    assert not torch.equal(y, y0)
+
+
 def test_wide_routed_gemm_parity():
     """Routed experts at the K3 latent width (l = 3584) with 64..256 rows per
     expert: CTA pairs and 256 x 512 tiles of 256 hidden units for GEMM1.
