@@ -320,9 +320,13 @@ LMOE_API const char* lmoe_status_string(lmoe_status status);
 LMOE_API const char* lmoe_last_error(void);
 
 /* Brackets every launch of the kernels named in `tags` (a comma-separated
- * list, "*" for all, NULL or "" to turn it off) with CUDA events on their
- * stream.  Tags: "xpass", "route", "dispatch", "gather", "expert_gemm1",
- * "expert_gemm2", "combine", "final". */
+ * list, "*" for all, NULL or "" to turn it off) with CUDA events, per thread.
+ * Each event is recorded on a library-owned side stream forked from the
+ * launching stream right before / after the launch (so it never sits between
+ * two kernels and cuts their programmatic overlap); the public call joins
+ * the side stream back into its own stream before it returns, so a stream
+ * capture of the call stays closed.  Tags: "xpass", "route", "dispatch",
+ * "gather", "expert_gemm1", "expert_gemm2", "combine", "final". */
 LMOE_API lmoe_status lmoe_profile_enable(const char* tags);
 /* Waits for the recorded events of kernel `tag` (NULL: every tag); returns the
  * summed device time (ms) and the number of bracketed launches since the last

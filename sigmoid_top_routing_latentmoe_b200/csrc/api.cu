@@ -24,8 +24,13 @@ void count_launch(int n) { g_launches += (uint64_t)n; }
 void set_last_error(const char* msg) { g_last_error = msg; }
 
 // --------------------------------------------------------------- profiling
-// Optional CUDA-event brackets around the launches of named kernels, on the
-// stream they are launched on.  Off unless lmoe_profile_enable names tags.
+// Optional CUDA-event brackets around the launches of named kernels.  Off
+// unless lmoe_profile_enable names tags.  Each event is recorded on a side
+// branch forked from the launching stream at that point (a library-owned
+// stream per thread and device), so no event sits between two kernels of the
+// launching stream: it would cut their programmatic (PDL) overlap, about
+// 3 us per bracket in a graph replay.  The branch is joined back into the
+// launching stream when the public call returns (ProfJoin).
 struct ProfRec {
   std::string tag;
   cudaEvent_t a, b;
@@ -38,6 +43,46 @@ static bool prof_wanted(const char* tag) {
   if (g_prof_tags == "*") return true;
   return g_prof_tags.find("," + std::string(tag) + ",") != std::string::npos;
 }
+
+static thread_local cudaStream_t g_prof_side[64];
+static thread_local cudaStream_t g_prof_forked = nullptr;  // side stream forked in this call
+
+static bool prof_record(cudaEvent_t ev, cudaStream_t st, unsigned flags) {
+  int dev = 0;
+  cudaStream_t side = nullptr;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+    if (g_prof_side[dev] == nullptr &&
+        cudaStreamCreateWithFlags(&g_prof_side[dev], cudaStreamNonBlocking) != cudaSuccess)
+      g_prof_side[dev] = nullptr;
+    side = g_prof_side[dev];
+  }
+  if (side == nullptr) return cudaEventRecordWithFlags(ev, st, flags) == cudaSuccess;
+  cudaEvent_t fork;
+  if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess) return false;
+  const bool ok = cudaEventRecord(fork, st) == cudaSuccess &&
+                  cudaStreamWaitEvent(side, fork, 0) == cudaSuccess &&
+                  cudaEventRecordWithFlags(ev, side, flags) == cudaSuccess;
+  cudaEventDestroy(fork);
+  g_prof_forked = side;
+  return ok;
+}
+
+// Joins the profiling side branch back into the call's stream (a stream
+// capture must end with every forked stream joined).
+struct ProfJoin {
+  cudaStream_t st;
+  explicit ProfJoin(cudaStream_t s) : st(s) {}
+  ~ProfJoin() {
+    if (g_prof_forked == nullptr) return;
+    cudaEvent_t j;
+    if (cudaEventCreateWithFlags(&j, cudaEventDisableTiming) == cudaSuccess) {
+      cudaEventRecord(j, g_prof_forked);
+      cudaStreamWaitEvent(st, j, 0);
+      cudaEventDestroy(j);
+    }
+    g_prof_forked = nullptr;
+  }
+};
 
 struct ProfScope {
   bool on = false;
@@ -52,11 +97,11 @@ struct ProfScope {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
       flags = cudaEventRecordExternal;
-    on = cudaEventRecordWithFlags(r.a, st, flags) == cudaSuccess;
+    on = prof_record(r.a, st, flags);
   }
   ~ProfScope() {
     if (!on) return;
-    cudaEventRecordWithFlags(r.b, st, flags);
+    prof_record(r.b, st, flags);
     g_prof.push_back(r);
   }
 };
@@ -644,6 +689,7 @@ lmoe_status moe_route(const lmoe_dims* dims, const void* x, const void* w_router
     return fail(LMOE_EINVAL, "expert_bias is not 16-byte aligned");
   LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
   LMOE_TRY(check_device());
+  ProfJoin pj((cudaStream_t)stream);  // joins the profiling branch on return
   cudaStream_t st = (cudaStream_t)stream;
   if (dims->dtype == LMOE_BF16)
     return run_route<__nv_bfloat16>(dims, x, w_router, expert_bias, ids, probs, ws, st);
@@ -663,6 +709,7 @@ lmoe_status moe_dispatch(const lmoe_dims* dims, const int32_t* ids, int32_t* cou
   LMOE_PTR(offsets, "offsets");
   LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
   LMOE_TRY(check_device());
+  ProfJoin pj((cudaStream_t)stream);  // joins the profiling branch on return
   return run_dispatch(dims, ids, counts, offsets, perm_token, inv_pair, ws, (cudaStream_t)stream);
 }
 
@@ -682,6 +729,7 @@ lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const int32_t* 
   LMOE_PTR(w_o, "w_o");
   LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
   LMOE_TRY(check_device());
+  ProfJoin pj((cudaStream_t)stream);  // joins the profiling branch on return
   cudaStream_t st = (cudaStream_t)stream;
   const Layout L = layout(dims, false);
   LMOE_CUDA(launch_build_tiles(offsets, dims->n_routed, &at<WsHeader>(ws, L.header)->n_mtiles,
@@ -769,6 +817,7 @@ lmoe_status latent_moe_backward(const lmoe_dims* dims, const lmoe_weights* w, co
   if (ws_bytes < need)
     return fail(LMOE_EWORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
   LMOE_TRY(check_device());
+  ProfJoin pj((cudaStream_t)stream);  // joins the profiling branch on return
   cudaStream_t st = (cudaStream_t)stream;
   LMOE_CUDA(cudaMemsetAsync(ws, 0, 256, st), "clear the header");
   if (dims->n_tokens == 0) {  // no tokens: every gradient is 0
@@ -815,6 +864,7 @@ lmoe_status moe_router_losses(const lmoe_dims* dims, const float* logits, int64_
     return fail(LMOE_EINVAL, "logits: ld < n_routed or misaligned");
   }
   LMOE_TRY(check_device());
+  ProfJoin pj((cudaStream_t)stream);  // joins the profiling branch on return
   const int64_t nb = loss_blocks(dims->n_tokens);
   float* part_s = at<float>(ws, L.loss);
   int32_t* part_c = reinterpret_cast<int32_t*>(part_s + nb * dims->n_routed);
@@ -868,6 +918,7 @@ lmoe_status latent_moe_forward(const lmoe_dims* dims, const lmoe_weights* weight
   if (counts_out && !aligned16(counts_out)) return fail(LMOE_EINVAL, "counts_out is not 16-byte aligned");
   LMOE_TRY(check_ws(dims, ws, ws_bytes, false));
   LMOE_TRY(check_device());
+  ProfJoin pj((cudaStream_t)stream);  // joins the profiling branch on return
   cudaStream_t st = (cudaStream_t)stream;
   if (dims->dtype == LMOE_BF16)
     return run_forward_tc(dims, weights, x, y, ids_out, probs_out, counts_out, ws, st);
@@ -883,6 +934,7 @@ lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_weights* w
     return fail(LMOE_EINVAL, "x_host / y_host is NULL");
   LMOE_TRY(check_ws(dims, ws, ws_bytes, true));
   LMOE_TRY(check_device());
+  ProfJoin pj((cudaStream_t)stream);  // joins the profiling branch on return
   cudaStream_t st = (cudaStream_t)stream;
   const Layout L = layout(dims, true);
   const int64_t N = dims->n_tokens;

@@ -1601,16 +1601,18 @@ cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {
   int grid = std::min(total, units);
   // Stream-K where whole tiles fill the last wave below 90% (and every pair
   // still gets >= 8 K blocks): the pairs' flags sit after the combine's counts.
-  // Not with the fused combine: a pair's first share is the tail of a tile,
-  // whose uhat K blocks then wait for the combine rows at once instead of
-  // after the shared experts' blocks (0.5b shape: final 35 -> 51 us).
+  // With the fused combine only while the tiles fill at most half the pairs:
+  // a pair's first share is the tail of a tile, whose uhat K blocks then wait
+  // for the combine rows at once instead of after the shared experts' blocks
+  // (0.5b shape, 64 tiles: final 35 -> 51 us; 12 and 24 tiles at 512 and
+  // 1024 tokens: forward 75 -> 71 and 80 -> 75 us).
   const int64_t iters = (int64_t)total * (p.S * p.kb0 + p.kb1);
   const int waves = (total + units - 1) / units;
   const bool sk_fits = a.sk_part != nullptr && a.sync != nullptr &&
                        (size_t)units * 2 * BM * p.bn * 4 <= a.sk_bytes &&
                        (p.fuse_combine ? m_tiles : 0) + units <= kSyncWords - 1;
-  const bool sk_pays =
-      !p.fuse_combine && (double)total < 0.9 * waves * units && iters >= 8LL * units;
+  const bool sk_pays = (!p.fuse_combine || 2 * total <= units) &&
+                       (double)total < 0.9 * waves * units && iters >= 8LL * units;
   if (sk_fits && (a.stream_k == 1 || (a.stream_k < 0 && sk_pays))) {
     p.stream_k = 1;
     p.sk_part = a.sk_part;
