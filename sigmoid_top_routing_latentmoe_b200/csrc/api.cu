@@ -181,8 +181,8 @@ static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 constexpr int kSkMaxPairs = 80;  // CTA pairs the stream-K scratch is sized for
 
 struct Layout {
-  size_t header, sync, z, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, zp, h,
-      skx, eo, hsh, uhat, loss, x, y, total;
+  size_t header, sync, z, logits, ids, probs, counts, offsets, perm, inv, block_counts, tiles, tiles2,
+      zp, h, skx, eo, hsh, uhat, loss, x, y, total;
   int64_t logits_ld;
   int max_tiles;
 };
@@ -208,6 +208,7 @@ static Layout layout(const lmoe_dims* d, bool host_copies) {
   L.inv = take((size_t)P * 4);
   L.block_counts = take((size_t)dispatch_blocks(P) * R * 4);
   L.tiles = take((size_t)L.max_tiles * sizeof(int4));
+  L.tiles2 = take((size_t)L.max_tiles * sizeof(int4));
   L.zp = take((size_t)P * d->latent * es);
   L.h = take((size_t)P * d->ff_routed * es);
   // The final GEMM's stream-K partials reuse [zp, eo), dead by then; this
@@ -295,12 +296,20 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
 // 128-row tiles were faster (0.5b: 18 + 11 us against 27 + 17 us), and for
 // decode-like loads of a few rows a 256-row MMA would mostly multiply empty
 // rows.
-static bool routed_pairs(const lmoe_dims* d) {
+// Routed GEMMs on CTA pairs over <= 256-row tiles, or single CTAs over <= 128.
+// Pairs when experts average 64 to 256 pairs (one tile per expert: its weights
+// stream once per output tile); with more, GEMM1 stays on pairs only for a
+// long K (l >= 1024; mid shape, 2048 rows per expert: GEMM1 528 -> 469 us on
+// pairs, GEMM2 280 -> 418 us, so GEMM2 stays single; 0.5b shape, l = 384:
+// both slower on pairs, 14.7 -> 19.8 and 8.1 -> 10.8 us).
+static bool routed_pairs(const lmoe_dims* d, int gemm) {
   const int64_t pairs = d->n_tokens * (int64_t)d->top_k, R = d->n_routed;
-  return d->dtype == LMOE_BF16 && pairs >= 64 * R && pairs <= 256 * R;
+  if (d->dtype != LMOE_BF16 || pairs < 64 * R) return false;
+  return pairs <= 256 * R || (gemm == 1 && d->latent >= 1024);
 }
-static int routed_tile_m(const lmoe_dims* d) {
-  return routed_pairs(d) ? kRoutedPairTileM : kTileM;
+// height of the tile list the dispatch writes (GEMM1's)
+static int routed_tile_m(const lmoe_dims* d, int gemm = 1) {
+  return routed_pairs(d, gemm) ? kRoutedPairTileM : kTileM;
 }
 
 // z != nullptr: the scatter also writes the sorted rows of z to the workspace
@@ -329,8 +338,9 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
 // (rows_sorted).
 template <typename T>
 static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32_t* perm,
-                                  const void* w_g, const void* w_u, const void* w_o, void* eo,
-                                  void* ws, cudaStream_t st, bool rows_sorted = false) {
+                                  const int32_t* offsets, const void* w_g, const void* w_u,
+                                  const void* w_o, void* eo, void* ws, cudaStream_t st,
+                                  bool rows_sorted = false) {
   const Layout L = layout(d, false);
   const int64_t P = d->n_tokens * d->top_k;
   if (P == 0) return LMOE_OK;
@@ -340,6 +350,16 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   const int4* tiles = at<int4>(ws, L.tiles);
   const int32_t* n_tiles = &at<WsHeader>(ws, L.header)->n_mtiles;
   const bool tc = std::is_same<T, __nv_bfloat16>::value;
+  // GEMM2's tile list: GEMM1's, or its own at the other height
+  const int4* tiles2 = tiles;
+  const int32_t* n_tiles2 = n_tiles;
+  if (routed_tile_m(d, 2) != routed_tile_m(d, 1)) {
+    tiles2 = at<int4>(ws, L.tiles2);
+    n_tiles2 = &at<WsHeader>(ws, L.header)->n_mtiles2;
+    LMOE_CUDA(launch_build_tiles(offsets, d->n_routed, const_cast<int32_t*>(n_tiles2),
+                                 const_cast<int4*>(tiles2), st, routed_tile_m(d, 2)),
+              "build_tiles");
+  }
   if (!rows_sorted) {
     ProfScope ps("gather", st);
     LMOE_CUDA(launch_gather_rows<T>((const T*)z, perm, P, Lt, zp, st), "gather");
@@ -353,7 +373,7 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   RoutedArgs ra{};
   ra.P = P; ra.L = Lt; ra.F = F; ra.R = d->n_routed; ra.tiles = tiles; ra.n_mtiles = n_tiles;
   ra.max_tiles = L.max_tiles; ra.beta1 = d->beta1; ra.beta2 = d->beta2;
-  ra.pairs = routed_pairs(d) ? 1 : 0;
+  ra.pairs = routed_pairs(d, 1) ? 1 : 0;
   // pairs with a long K (l >= 2048): GEMM1 on 256 x 512 tiles, 256 hidden units each
   ra.wide = ra.pairs && Lt >= 2048 ? 1 : 0;
   {
@@ -369,13 +389,15 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   SimtGemm g2{};
   g2.A[0] = h; g2.lda[0] = F; g2.B[0] = w_o; g2.ldb[0] = F; g2.K[0] = F; g2.nseg = 1;
   g2.b_expert_stride = (int64_t)Lt * F;
-  g2.C = eo; g2.ldc = Lt; g2.N = Lt; g2.tiles = tiles; g2.n_tiles = n_tiles;
+  g2.C = eo; g2.ldc = Lt; g2.N = Lt; g2.tiles = tiles2; g2.n_tiles = n_tiles2;
   g2.max_tiles = L.max_tiles; g2.mode = kStore;
   {
     ProfScope ps("expert_gemm2", st);
     if (tc) {
       ra.a = (const __nv_bfloat16*)h; ra.w0 = (const __nv_bfloat16*)w_o; ra.w1 = nullptr;
       ra.out = (__nv_bfloat16*)eo;
+      ra.pairs = routed_pairs(d, 2) ? 1 : 0;
+      ra.tiles = tiles2; ra.n_mtiles = n_tiles2;
       LMOE_CUDA(umma_routed2(ra, status, st), "routed gemm2 (tcgen05)");
     } else {
       LMOE_CUDA(launch_simt_gemm<T>(g2, st), "routed gemm2");
@@ -453,7 +475,7 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
   // launch; larger ones by the gather kernel, which has more memory parallelism.
   const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * sizeof(T) <= (16u << 20);
   LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
-  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
+  LMOE_TRY(run_expert_ffn<T>(d, z, perm, offsets, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
   // For l <= 1024 and up to 64 MB of expert outputs the combine runs inside
   // the final GEMM (its epilogue warps write RMSNorm(u) while the K loop goes
   // through the shared experts' blocks; 0.5b shape: combine + final 34 -> 31 us).
@@ -535,7 +557,7 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
   // launch; larger ones by the gather kernel, which has more memory parallelism.
   const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * sizeof(T) <= (16u << 20);
   LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
-  LMOE_TRY(run_expert_ffn<T>(d, z, perm, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
+  LMOE_TRY(run_expert_ffn<T>(d, z, perm, offsets, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
   {
     ProfScope ps("combine", st);
     LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, d->top_k, Lt, d->rms_eps, uhat,
@@ -736,8 +758,9 @@ lmoe_status moe_expert_ffn(const lmoe_dims* dims, const void* z, const int32_t* 
                                at<int4>(ws, L.tiles), st, routed_tile_m(dims)),
             "build_tiles");
   if (dims->dtype == LMOE_BF16)
-    return run_expert_ffn<__nv_bfloat16>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
-  return run_expert_ffn<float>(dims, z, perm_token, w_g, w_u, w_o, expert_out, ws, st);
+    return run_expert_ffn<__nv_bfloat16>(dims, z, perm_token, offsets, w_g, w_u, w_o, expert_out,
+                                         ws, st);
+  return run_expert_ffn<float>(dims, z, perm_token, offsets, w_g, w_u, w_o, expert_out, ws, st);
 }
 
 lmoe_status lmoe_check_dispatch(const lmoe_dims* dims, const int32_t* ids, const int32_t* counts,

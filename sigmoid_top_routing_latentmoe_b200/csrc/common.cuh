@@ -30,7 +30,8 @@ constexpr int kSyncWords = 1024;
 struct WsHeader {
   int32_t status;        // 0, or the first failure code recorded on the device
   int32_t n_mtiles;      // number of routed row tiles (written by dispatch)
-  int32_t pad[62];
+  int32_t n_mtiles2;     // routed GEMM2's own list, when its tile height differs
+  int32_t pad[61];
 };
 
 __device__ __forceinline__ float to_f(float v) { return v; }

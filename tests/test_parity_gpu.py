@@ -461,6 +461,36 @@ def test_stream_k_final_gemm(name, n, mode, monkeypatch):
     assert not torch.equal(y, y0)
 
 
+def test_routed_gemms_on_different_tile_heights():
+    """Experts over 256 pairs with l >= 1024: routed GEMM1 on CTA pairs over
+    256-row tiles, GEMM2 on single CTAs over its own 128-row tile list.
+    moe_expert_ffn on the oracle's z and permutation, sampled sorted rows
+    against the oracle's SiTU expert (bf16 tolerance of the forward)."""
+    wl = W["mid"].with_tokens(2200)          # 17600 pairs over 64 experts: ~275 each
+    inp = prepare(wl)
+    ow = oracle_weights(inp)
+    ref = oracle.forward(odims(wl), ow, synth.to_f32(inp["x"]), want=("z",))
+    counts, offsets, perm, inv = oracle.permute(ref["ids"], wl.n_routed)
+    assert counts.mean() > 256
+    z = round_act(ref["z"], wl)
+    P = wl.n_tokens * wl.top_k
+    dims = ldims(wl)
+    ws = lm.alloc_workspace(dims)
+    dev = device_inputs({k: inp[k] for k in ("w_g", "w_u", "w_o")})
+    eo = torch.empty(P, wl.latent, dtype=torch.bfloat16, device="cuda")
+    lm.moe_expert_ffn(dims, torch.from_numpy(z).to("cuda", torch.bfloat16), to_device(perm, ""),
+                      to_device(offsets, ""), dev["w_g"], dev["w_u"], dev["w_o"], eo, ws)
+    torch.cuda.synchronize()
+    assert lm.get_device_status(ws) == lm.OK
+    # every expert's first and last rows (tile edges of both heights) and a stride
+    rows = np.unique(np.concatenate([offsets[:-1], offsets[1:] - 1, np.arange(0, P, 41)]))
+    rows = rows[(rows >= 0) & (rows < P)]
+    expert = np.searchsorted(offsets, rows, side="right") - 1
+    exp_eo = np.stack([oracle.situ(ow["w_g"][e], ow["w_u"][e], ow["w_o"][e], z[perm[r]],
+                                   wl.beta1, wl.beta2)[0] for r, e in zip(rows, expert)])
+    assert rel_err(host(eo)[rows], exp_eo) <= 2e-2
+
+
 def test_wide_routed_gemm_parity():
     """Routed experts at the K3 latent width (l = 3584) with 64..256 rows per
     expert: CTA pairs and 256 x 512 tiles of 256 hidden units for GEMM1.
