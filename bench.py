@@ -489,6 +489,7 @@ def main():
         raise SystemExit("device status not OK after warm-up")
 
     prof_tag = args.profile_kernel or "xpass"
+    plan = lm.forward_plan(dims)
     bound, work = kernel_work(wl, prof_tag)
     lm.profile_read()                       # drop anything recorded so far
     clocks = ClockSampler(local)
@@ -691,6 +692,7 @@ def main():
         "gpu_launches": launches,
         "host_enqueue_us": host_enqueue_us,
         "kernel_us": breakdown,
+        "plan": [name for name, on in plan.items() if on],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.seed)

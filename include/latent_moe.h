@@ -263,6 +263,26 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
                                     const void* x_host, void* y_host, void* ws, size_t ws_bytes,
                                     lmoe_stream stream);
 
+/* The launch plan latent_moe_forward takes for these dims (host only,
+ * nothing is launched), as LMOE_PLAN_* bits in *flags:
+ *   COMBINE_FUSED     the combine + RMSNorm runs in the final GEMM's epilogue;
+ *   XPASS_WIDE        x-pass on 256 x 512 tiles;
+ *   GEMM1_PAIRS / GEMM2_PAIRS  routed GEMM1 / GEMM2 on CTA pairs (256-row tiles);
+ *   GEMM1_WIDE        routed GEMM1 on 256 x 512 tiles;
+ *   ROWS_IN_SCATTER   the dispatch's scatter writes the sorted copy of z
+ *                     (else a gather kernel does).
+ * The final GEMM's stream-K choice is made at launch and not reported here.
+ * EINVAL on bad dims or flags == NULL. */
+enum {
+  LMOE_PLAN_COMBINE_FUSED = 1,
+  LMOE_PLAN_XPASS_WIDE = 2,
+  LMOE_PLAN_GEMM1_PAIRS = 4,
+  LMOE_PLAN_GEMM2_PAIRS = 8,
+  LMOE_PLAN_GEMM1_WIDE = 16,
+  LMOE_PLAN_ROWS_IN_SCATTER = 32
+};
+LMOE_API lmoe_status lmoe_forward_plan(const lmoe_dims* dims, int32_t* flags);
+
 /* Byte offsets of the forward's intermediates inside the workspace, for
  * inspection after latent_moe_forward: offsets[0..6] = z [N,l], router logits
  * [N, ld] fp32, shared hidden units [N, S*G], RMSNorm(u) [N,l], routed expert
@@ -326,7 +346,8 @@ LMOE_API const char* lmoe_last_error(void);
  * two kernels and cuts their programmatic overlap); the public call joins
  * the side stream back into its own stream before it returns, so a stream
  * capture of the call stays closed.  Tags: "xpass", "route", "dispatch",
- * "gather", "expert_gemm1", "expert_gemm2", "combine", "final". */
+ * "gather", "expert_gemm1", "expert_gemm2", "combine", "final",
+ * "router_losses". */
 LMOE_API lmoe_status lmoe_profile_enable(const char* tags);
 /* Waits for the recorded events of kernel `tag` (NULL: every tag); returns the
  * summed device time (ms) and the number of bracketed launches since the last

@@ -90,6 +90,7 @@ _sigs = {
     "lmoe_launch_count": (ctypes.c_uint64, [ctypes.c_int32]),
     "lmoe_profile_enable": (_S, [ctypes.c_char_p]),
     "lmoe_workspace_layout": (_S, [_DP, ctypes.POINTER(ctypes.c_size_t), ctypes.c_int32]),
+    "lmoe_forward_plan": (_S, [_DP, ctypes.POINTER(ctypes.c_int32)]),
     "lmoe_profile_read": (_S, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     "lmoe_profile_read_tag": (_S, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
                                    ctypes.POINTER(ctypes.c_int64)]),
@@ -169,6 +170,17 @@ def workspace_views(dims: Dims, ws: torch.Tensor) -> dict:
             "offsets": view(off[8], 1, dims.n_routed + 1, torch.int32, 4)[0],
             "perm": view(off[9], 1, N * k, torch.int32, 4)[0],
             "inv": view(off[10], N, k, torch.int32, 4)}
+
+
+PLAN_BITS = {"combine_fused": 1, "xpass_wide": 2, "gemm1_pairs": 4, "gemm2_pairs": 8,
+             "gemm1_wide": 16, "rows_in_scatter": 32}
+
+
+def forward_plan(dims: Dims) -> dict:
+    """The launch plan of latent_moe_forward for ``dims`` (lmoe_forward_plan)."""
+    f = ctypes.c_int32(0)
+    _check(_lib.lmoe_forward_plan(ctypes.byref(dims), ctypes.byref(f)), "lmoe_forward_plan")
+    return {name: bool(f.value & bit) for name, bit in PLAN_BITS.items()}
 
 
 def workspace_init(ws: torch.Tensor, stream=None):

@@ -423,6 +423,13 @@ static int xpass_wide(const lmoe_dims* d) {
   return d->d >= 2048 ? 1 : 0;
 }
 
+// The combine inside the final GEMM (bf16, l <= 1024, <= 64 MB of expert outputs).
+static bool combine_fused(const lmoe_dims* d) {
+  return d->dtype == LMOE_BF16 && d->latent <= 1024 &&
+         (d->n_tokens + 255) / 256 <= kSyncWords - 1 &&
+         (double)d->n_tokens * d->top_k * d->latent * 2.0 <= 64.0 * (1 << 20);
+}
+
 // bf16 forward on the tensor cores, one stream: the x-pass (z, routing and the
 // shared experts' hidden units), dispatch, the routed experts, combine +
 // RMSNorm, and one GEMM for y = shared + W_up RMSNorm(u).
@@ -481,8 +488,7 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
   // through the shared experts' blocks; 0.5b shape: combine + final 34 -> 31 us).
   // Larger volumes get the combine kernel first: their reads compete with the
   // final GEMM's own (mid shape, 268 MB: +23 us per step fused).
-  const bool fuse_combine = Lt <= 1024 && (N + 255) / 256 <= kSyncWords - 1 &&
-                            (double)N * k * Lt * sizeof(T) <= 64.0 * (1 << 20);
+  const bool fuse_combine = combine_fused(d);
   if (!fuse_combine) {
     ProfScope ps("combine", st);
     LMOE_CUDA(launch_combine<T>(eo, inv, probs, w->rms_weight, N, k, Lt, d->rms_eps, uhat, st),
@@ -1008,6 +1014,24 @@ lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_weights* w
   LMOE_CUDA(cudaEventRecord(hp->done, hp->out), "event");
   LMOE_CUDA(cudaStreamWaitEvent(st, hp->done, 0), "wait");
   LMOE_CUDA(cudaStreamSynchronize(st), "sync");
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_forward_plan(const lmoe_dims* dims, int32_t* flags) {
+  LMOE_TRY(check_dims(dims));
+  if (flags == nullptr) return fail(LMOE_EINVAL, "flags is NULL");
+  const lmoe_dims* d = dims;
+  const bool bf16 = d->dtype == LMOE_BF16;
+  const size_t es = bf16 ? 2 : 4;
+  const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * es <= (16u << 20);
+  int32_t f = 0;
+  if (bf16 && combine_fused(d)) f |= LMOE_PLAN_COMBINE_FUSED;
+  if (bf16 && xpass_wide(d)) f |= LMOE_PLAN_XPASS_WIDE;
+  if (routed_pairs(d, 1)) f |= LMOE_PLAN_GEMM1_PAIRS;
+  if (routed_pairs(d, 2)) f |= LMOE_PLAN_GEMM2_PAIRS;
+  if (routed_pairs(d, 1) && d->latent >= 2048) f |= LMOE_PLAN_GEMM1_WIDE;
+  if (fuse_rows) f |= LMOE_PLAN_ROWS_IN_SCATTER;
+  *flags = f;
   return LMOE_OK;
 }
 

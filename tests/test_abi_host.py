@@ -75,3 +75,21 @@ def test_misaligned_and_short_workspace_rejected(lm):
     st = lm._lib.latent_moe_forward(ctypes.byref(d), ctypes.byref(w), fake + 4, fake, None, None,
                                     None, fake, 10 ** 9, None)
     assert st == lm.EINVAL                           # x misaligned
+
+
+def test_forward_plan(lm):
+    """lmoe_forward_plan: the launch plan the forward takes, decided on the host."""
+    import torch
+    on = lambda dims: {k for k, v in lm.forward_plan(dims).items() if v}
+    halfb = lm.make_dims(4096, 768, 384, 16, 2, 2, 768, 1536)
+    mid = lm.make_dims(16384, 2048, 1024, 64, 8, 1, 1024, 4096)
+    k3 = lm.make_dims(8192, 7168, 3584, 896, 16, 1, 512, 2048)
+    assert on(halfb) == {"combine_fused", "rows_in_scatter"}
+    assert on(mid) == {"xpass_wide", "gemm1_pairs"}     # GEMM2 on single CTAs
+    assert on(k3) == {"xpass_wide", "gemm1_pairs", "gemm2_pairs", "gemm1_wide"}
+    assert on(lm.make_dims(128, 256, 128, 16, 2, 2, 256, 512, dtype=torch.float32)) \
+        == {"rows_in_scatter"}
+    flags = ctypes.c_int32(0)
+    assert lm._lib.lmoe_forward_plan(ctypes.byref(halfb), None) == lm.EINVAL
+    bad = lm.make_dims(4096, 770, 384, 16, 2, 2, 768, 1536)
+    assert lm._lib.lmoe_forward_plan(ctypes.byref(bad), ctypes.byref(flags)) == lm.EINVAL

@@ -419,6 +419,7 @@ def test_fused_combine_matches_combine_entry_point(name, n):
     the same expert outputs bit for bit, and every launch must leave the
     synchronisation area after the workspace header zeroed for the next one."""
     wl = W[name].with_tokens(n)
+    assert lm.forward_plan(ldims(wl))["combine_fused"]
     inp = prepare(wl)
     dev = device_inputs(inp)
     y, ids, probs, counts, ws = _run_forward(wl, dev)
@@ -467,6 +468,8 @@ def test_routed_gemms_on_different_tile_heights():
     moe_expert_ffn on the oracle's z and permutation, sampled sorted rows
     against the oracle's SiTU expert (bf16 tolerance of the forward)."""
     wl = W["mid"].with_tokens(2200)          # 17600 pairs over 64 experts: ~275 each
+    plan = lm.forward_plan(ldims(wl))
+    assert plan["gemm1_pairs"] and not plan["gemm2_pairs"]
     inp = prepare(wl)
     ow = oracle_weights(inp)
     ref = oracle.forward(odims(wl), ow, synth.to_f32(inp["x"]), want=("z",))
