@@ -308,15 +308,26 @@ __global__ void gather_rows_kernel(const T* __restrict__ z, const int32_t* __res
                                    int64_t n_rows, int width, T* __restrict__ zp) {
   pdl_trigger();
   pdl_wait();
-  // one warp per row, 16-byte vectors
+  // one warp per row, 16-byte vectors: up to 8 loads per lane in flight
+  // before their stores; the sorted copy is written once and read once by
+  // routed GEMM1, so its stores stream past L2 (st.global.cs)
+  constexpr int U = 8;
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= n_rows) return;
   const int64_t src = perm_token[r];
-  const int vec = 16 / sizeof(T);
+  const int nv = width / (int)(16 / sizeof(T));
   const uint4* s = reinterpret_cast<const uint4*>(z + src * width);
   uint4* d = reinterpret_cast<uint4*>(zp + r * width);
-  for (int i = lane; i < width / vec; i += 32) d[i] = s[i];
+  for (int i0 = lane; i0 < nv; i0 += 32 * U) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (i0 + 32 * u < nv) v[u] = __ldg(s + i0 + 32 * u);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (i0 + 32 * u < nv) __stcs(d + i0 + 32 * u, v[u]);
+  }
 }
 
 // Consistency check of a permutation: ids in range, counts summing to N k,
