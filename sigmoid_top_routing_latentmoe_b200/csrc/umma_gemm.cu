@@ -141,7 +141,7 @@ struct Params {
   int c_k, c_vpl, fuse_combine;
   float c_eps;
   // FINAL with stream-K scheduling: each unit (CTA pair) takes an equal share
-  // of the tiles' K-block iterations; see next_work and the epilogue
+  // of the tiles' K-block iterations; see work_begin / work_next and the epilogue
   int stream_k;
   float* sk_part;     // [units][2 ranks][4 lane quarters][bn / 64][16][32] float4 partials
   int32_t* sk_flags;  // [units] warps that stored the unit's partial
