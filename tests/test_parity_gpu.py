@@ -436,7 +436,9 @@ def test_fused_combine_matches_combine_entry_point(name, n):
 
 
 @pytest.mark.parametrize("name,n,mode", [("k3_width", 320, None), ("halfb_uniform", 300, "1"),
-                                         ("mid", 136, "1"), ("halfb_uniform", 4096, "1")])
+                                         ("mid", 136, "1"), ("halfb_uniform", 4096, "1"),
+                                         # one row tile split many ways: 1 K block per pair
+                                         ("halfb_uniform", 1, "1"), ("k3_width", 3, "1")])
 def test_stream_k_final_gemm(name, n, mode, monkeypatch):
     """Stream-K final GEMM: the CTA pairs share the tiles x K-blocks iterations
     and a tile split between pairs is summed in fp32 in a fixed order.  At the
@@ -459,7 +461,8 @@ def test_stream_k_final_gemm(name, n, mode, monkeypatch):
     monkeypatch.setenv("LMOE_STREAM_K", "0")
     y0, _, _, _, _ = _run_forward(wl, dev, ws)
     assert rel_err(host(y), host(y0)) <= 1e-2
-    assert not torch.equal(y, y0)
+    if n >= 100:   # enough outputs that some bf16 rounding must differ
+        assert not torch.equal(y, y0)
 
 
 def test_routed_gemms_on_different_tile_heights():
