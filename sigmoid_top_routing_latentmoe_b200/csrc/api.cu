@@ -468,6 +468,11 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
     a.hsh = hsh; a.beta1 = d->beta1; a.beta2 = d->beta2;
     a.bias = w->expert_bias; a.ids = ids; a.probs = probs; a.top_k = k; a.router = d->router;
     a.wide = xpass_wide(d);
+    // stream-K scratch: the sorted-z / routed-hidden region, unused until the dispatch
+    a.sync = at<int32_t>(ws, L.sync);
+    a.sk_part = at<float>(ws, L.zp);
+    a.sk_bytes = L.eo - L.zp;
+    a.stream_k = stream_k_mode();
     ProfScope ps("xpass", st);
     LMOE_CUDA(umma_xpass(a, status, st), "x-pass (tcgen05)");
   }

@@ -62,19 +62,31 @@ constexpr uint64_t WAIT_CAP_NS = 2000000000ull;
 
 // XPASS_F32: the x-pass with fp32 z and shared gate / up pre-activations (no SiTU)
 // XPASS_WIDE, FINAL_WIDE, ROUTED1_WIDE: those GEMMs on 256 x 512 pair tiles (see Cfg)
+// XPASS_SK, XPASS_WIDE_SK: the x-pass under stream-K (their own instantiations,
+//   so that the stream-K code costs the plain x-pass no registers)
 enum Mode {
   XPASS = 0, FINAL = 1, ROUTED1 = 2, ROUTED2 = 3, XPASS_F32 = 4,
-  XPASS_WIDE = 5, FINAL_WIDE = 6, ROUTED1_WIDE = 7
+  XPASS_WIDE = 5, FINAL_WIDE = 6, ROUTED1_WIDE = 7, XPASS_SK = 8, XPASS_WIDE_SK = 9
 };
 template <int MODE>
-constexpr bool is_wide() { return MODE == XPASS_WIDE || MODE == FINAL_WIDE || MODE == ROUTED1_WIDE; }
+constexpr bool is_wide() {
+  return MODE == XPASS_WIDE || MODE == FINAL_WIDE || MODE == ROUTED1_WIDE || MODE == XPASS_WIDE_SK;
+}
 // the GEMM a mode computes (a wide mode computes its base mode's GEMM)
 template <int MODE>
 constexpr int base_of() {
-  return MODE == XPASS_WIDE ? XPASS : MODE == FINAL_WIDE ? FINAL : MODE == ROUTED1_WIDE ? ROUTED1 : MODE;
+  return MODE == XPASS_WIDE || MODE == XPASS_SK || MODE == XPASS_WIDE_SK ? XPASS
+         : MODE == FINAL_WIDE                                           ? FINAL
+         : MODE == ROUTED1_WIDE                                         ? ROUTED1
+                                                                        : MODE;
 }
 template <int MODE>
-constexpr bool is_xpass() { return MODE == XPASS || MODE == XPASS_F32 || MODE == XPASS_WIDE; }
+constexpr bool is_xpass() {
+  return MODE == XPASS || MODE == XPASS_F32 || MODE == XPASS_WIDE || MODE == XPASS_SK ||
+         MODE == XPASS_WIDE_SK;
+}
+template <int MODE>
+constexpr bool is_xpass_sk() { return MODE == XPASS_SK || MODE == XPASS_WIDE_SK; }
 
 // CG = 1: one CTA computes a 128-row tile and loads every B sub-tile.
 // CG = 2: a CTA pair (cluster of 2) computes a 256-row tile with
@@ -307,6 +319,25 @@ __device__ __forceinline__ void tc_ld32x2(uint32_t ta, float (&va)[32], uint32_t
     va[i] = __uint_as_float(r[i]);
     vb[i] = __uint_as_float(q[i]);
   }
+}
+// Two 32-column TMEM stores, then a wait for both (32 lanes x 32 columns each).
+__device__ __forceinline__ void tc_st32x2(uint32_t ta, const float (&va)[32], uint32_t tb,
+                                          const float (&vb)[32]) {
+#define LMOE_TC_ST32(ADDR, V)                                                                   \
+  asm volatile(                                                                                 \
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "                                           \
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"                                \
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"                       \
+      ::"r"(ADDR), "f"(V[0]), "f"(V[1]), "f"(V[2]), "f"(V[3]), "f"(V[4]), "f"(V[5]), "f"(V[6]), \
+      "f"(V[7]), "f"(V[8]), "f"(V[9]), "f"(V[10]), "f"(V[11]), "f"(V[12]), "f"(V[13]),          \
+      "f"(V[14]), "f"(V[15]), "f"(V[16]), "f"(V[17]), "f"(V[18]), "f"(V[19]), "f"(V[20]),       \
+      "f"(V[21]), "f"(V[22]), "f"(V[23]), "f"(V[24]), "f"(V[25]), "f"(V[26]), "f"(V[27]),       \
+      "f"(V[28]), "f"(V[29]), "f"(V[30]), "f"(V[31])                                            \
+      : "memory")
+  LMOE_TC_ST32(ta, va);
+  LMOE_TC_ST32(tb, vb);
+#undef LMOE_TC_ST32
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 // Two 16-column TMEM loads in flight before one wait.
 __device__ __forceinline__ void tc_ld16x2(uint32_t ta, float (&va)[16], uint32_t tb,
@@ -636,7 +667,7 @@ template <int MODE, int CG>
 __device__ __forceinline__ WorkIter work_begin(const Params& p, int unit, int n_units) {
   WorkIter it;
   it.nkb = k_blocks<MODE>(p);
-  it.sk = base_of<MODE>() == FINAL && p.stream_k;
+  it.sk = (base_of<MODE>() == FINAL || is_xpass_sk<MODE>()) && p.stream_k;
   const int64_t total = total_tiles<MODE, CG>(p);
   if (it.sk) {
     const int64_t q = total * it.nkb;
@@ -1011,10 +1042,77 @@ __device__ __forceinline__ void route_row32(const Params& p, const float (&lg)[3
   for (int slot = 0; slot < p.top_k; ++slot) probs[slot] = probs[slot] / den;
 }
 
+// x-pass stream-K share of one tile (see the epilogue).  Role 1: store the
+// raw accumulator (NB 64-column blocks of this warp's lane quarter, if any
+// of its rows exist) and count
+// the warp in sk_flags; returns false (no epilogue).  Role 2: wait for the
+// shares of units unit + 1 .. sk_last, add them into TMEM in unit order, and
+// meet the other epilogue warps at the fix-up barrier (capped), so that the
+// epilogue reads fixed columns only; returns whether all of that completed.
+template <int NB, int CG>
+__device__ __noinline__ bool xpass_sk_fixup(const Params& p, uint32_t tbase, int sk_role, int unit,
+                                            int sk_last, uint32_t rank, int ew, int h0,
+                                            bool has_rows, uint64_t* fixbar, uint32_t& fix_phase,
+                                            volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31;
+  auto part = [&](int u, int cb) {
+    return reinterpret_cast<float4*>(p.sk_part) +
+           ((((size_t)u * 2 + rank) * 4 + ew) * NB + cb) * 16 * 32 + lane;
+  };
+  bool waited = true;
+  if (sk_role == 2 && lane == 0)
+    for (int u2 = unit + 1; u2 <= sk_last && waited; ++u2)
+      waited = wait_count(p.sk_flags + u2, CG * EPI_WARPS, abort_flag, p.status);
+  waited = __shfl_sync(0xffffffffu, (int)waited, 0) != 0;
+  __syncwarp();
+  // a warp whose 32 rows lie past the tile's last row neither stores nor
+  // reads partials (they would never be stored)
+#pragma unroll 1
+  for (int cb = h0; has_rows && waited && cb < NB; cb += HS) {
+    float a[32], b[32];
+    tc_ld32x2(tbase + cb * 64, a, tbase + cb * 64 + 32, b);
+    if (sk_role == 1) {
+      float4* dst = part(unit, cb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        dst[j * 32] = make_float4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
+        dst[(8 + j) * 32] = make_float4(b[4 * j], b[4 * j + 1], b[4 * j + 2], b[4 * j + 3]);
+      }
+      continue;
+    }
+    for (int u2 = unit + 1; u2 <= sk_last; ++u2) {
+      const float4* src = part(u2, cb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 pa = __ldcg(src + j * 32), pb = __ldcg(src + (8 + j) * 32);
+        a[4 * j] += pa.x; a[4 * j + 1] += pa.y; a[4 * j + 2] += pa.z; a[4 * j + 3] += pa.w;
+        b[4 * j] += pb.x; b[4 * j + 1] += pb.y; b[4 * j + 2] += pb.z; b[4 * j + 3] += pb.w;
+      }
+    }
+    tc_st32x2(tbase + cb * 64, a, tbase + cb * 64 + 32, b);
+  }
+  if (sk_role == 1) {
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) atomicAdd(p.sk_flags + unit, 1);
+    return false;
+  }
+  // the other epilogue warps' columns are fixed too: an mbarrier with a
+  // capped wait (a warp that gave up earlier cannot hang the others)
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(fixbar));
+  const bool fixed = mbar_wait(smem_u32(fixbar), fix_phase, abort_flag, p.status);
+  fix_phase ^= 1u;
+  tc_fence_after();
+  return waited && fixed;
+}
+
 template <int MODE, int CG>
 __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint64_t* tempty,
-                                         uint32_t tmem, uint32_t stage, volatile int* abort_flag,
-                                         uint32_t rank, int unit, int n_units) {
+                                         uint64_t* fixbar, uint32_t tmem, uint32_t stage,
+                                         volatile int* abort_flag, uint32_t rank, int unit,
+                                         int n_units) {
   const int ew = (threadIdx.x >> 5) & 3;  // TMEM lane quarter this warp may access
   // first column block of this warp (then every HS-th)
   const int h0 = EPI_WARPS == 8 ? ((threadIdx.x >> 5) - 2) >> 2 : 0;
@@ -1045,6 +1143,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
   }
   int acc = 0;
   uint32_t acc_phase = 0;
+  uint32_t fix_phase = 0;  // x-pass stream-K: phase of the fix-up barrier
   const int nkb = k_blocks<MODE>(p);
   const int64_t q_sk = (int64_t)total_tiles<MODE, CG>(p) * nkb;  // stream-K iterations
   WorkIter wi = work_begin<MODE, CG>(p, unit, n_units);
@@ -1057,7 +1156,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
     // waits for the partials of the units after it that hold the rest, and
     // adds them in unit order before the epilogue: a fixed summation order.
     int sk_role = 0, sk_last = unit;
-    if (base_of<MODE>() == FINAL && p.stream_k) {
+    if ((base_of<MODE>() == FINAL || is_xpass_sk<MODE>()) && p.stream_k) {
       if (wk.kb0 > 0) {
         sk_role = 1;
       } else if (wk.kb1 < nkb) {
@@ -1070,8 +1169,18 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
     const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + acc * Cfg<MODE, CG>::ACC_STRIDE;
     const int rows = min(32, tl.rows - wrow);  // rows of this warp inside the tile
     const int64_t grow0 = (int64_t)tl.m0 + wrow;
-    if (rows <= 0) {
-      // nothing of this warp's rows exists in the tile
+    bool sk_skip = false;  // x-pass role 1: partial stored, no epilogue
+    if constexpr (is_xpass_sk<MODE>()) {
+      if (sk_role != 0) {
+        // x-pass stream-K: role 1 stores the raw accumulator and skips the
+        // epilogue; role 2 adds the other shares into TMEM first
+        sk_skip = !xpass_sk_fixup<Cfg<MODE, CG>::W * 4, CG>(p, tbase, sk_role, unit, sk_last,
+                                                           rank, ew, h0, rows > 0, fixbar,
+                                                           fix_phase, abort_flag);
+      }
+    }
+    if (rows <= 0 || sk_skip) {
+      // nothing of this warp's rows exists in the tile (or a stream-K share)
     } else if (tl.epi == EPI_SITU) {
       // columns [0,128) hold gate pre-activations, [128,256) the matching up ones;
       // this warp writes the blocks of 64 hidden units h0, h0 + HS, ...
@@ -1234,7 +1343,7 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
                         p.ld0, rows, cols);
       }
     }
-    if (sk_role == 1) {  // every warp counts, whether or not it had rows to store
+    if (base_of<MODE>() == FINAL && sk_role == 1) {  // every warp counts, rows or not
       __threadfence();
       __syncwarp();
       if (lane == 0) atomicAdd(p.sk_flags + unit, 1);
@@ -1258,7 +1367,8 @@ template <int MODE, int CG>
 __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
   using C = Cfg<MODE, CG>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[C::STAGES], empty[C::STAGES], tfull[2], tempty[2], drain;
+  __shared__ __align__(8) uint64_t full[C::STAGES], empty[C::STAGES], tfull[2], tempty[2], drain,
+      fixbar;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
   uint8_t* ring = reinterpret_cast<uint8_t*>(
@@ -1278,6 +1388,7 @@ __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_cons
       mbar_init(smem_u32(&tempty[a]), EPI_WARPS * CG);
     }
     mbar_init(smem_u32(&drain), 1);
+    mbar_init(smem_u32(&fixbar), EPI_WARPS);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1323,14 +1434,15 @@ __global__ void __launch_bounds__(THREADS, 1) umma_gemm_kernel(const __grid_cons
   } else {
     const uint32_t stage =
         smem_u32(ring) + C::STAGES * C::STAGE_BYTES + (warp - 2) * C::EPI_STAGE;
-    epilogue<MODE, CG>(p, tfull, tempty, tmem, stage, &abort_flag, rank, unit, n_units);
+    epilogue<MODE, CG>(p, tfull, tempty, &fixbar, tmem, stage, &abort_flag, rank, unit, n_units);
   }
 
   tc_fence_before();
   __syncthreads();
   if (CG == 2) cluster_sync();  // neither CTA frees TMEM or exits while its pair still works
   tc_fence_after();
-  if (base_of<MODE>() == FINAL && (p.fuse_combine || p.stream_k) && threadIdx.x == 0) {
+  if ((base_of<MODE>() == FINAL || is_xpass_sk<MODE>()) && (p.fuse_combine || p.stream_k) &&
+      threadIdx.x == 0) {
     // the last CTA to finish (every CTA is past its waits) zeroes the counts
     // and flags for the next launch
     __threadfence();
@@ -1553,8 +1665,25 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   const int total = (int)((a.N + 2 * BM - 1) / (2 * BM)) * p.n_tiles;
   const int units = a.max_units > 0 ? std::min(a.max_units, num_sms() / 2) : num_sms() / 2;
   if (f32) return launch<XPASS_F32, 2>(p, std::min(total, units), st);
-  return wide ? launch<XPASS_WIDE, 2>(p, std::min(total, units), st)
-              : launch<XPASS, 2>(p, std::min(total, units), st);
+  int grid = std::min(total, units);
+  // Stream-K by the final GEMM's rule (a decode step at the K3 width: 17 row x
+  // column tiles of 112 K blocks for 74 pairs)
+  const int64_t iters = (int64_t)total * p.kb0;
+  const int waves = (total + units - 1) / units;
+  const size_t part_bytes = (size_t)units * 2 * BM * (wide ? 4 : 2) * SUB * 4;
+  const bool sk_fits = a.sk_part != nullptr && a.sync != nullptr && part_bytes <= a.sk_bytes &&
+                       units <= kSyncWords - 1;
+  const bool sk_pays = (double)total < 0.9 * waves * units && iters >= 8LL * units;
+  if (sk_fits && (a.stream_k == 1 || (a.stream_k < 0 && sk_pays))) {
+    p.stream_k = 1;
+    p.sk_part = a.sk_part;
+    p.sk_flags = a.sync + (kSyncWords - 1 - units);
+    p.c_sync = a.sync;
+    grid = (int)std::min<int64_t>(units, iters);
+  }
+  if (p.stream_k)
+    return wide ? launch<XPASS_WIDE_SK, 2>(p, grid, st) : launch<XPASS_SK, 2>(p, grid, st);
+  return wide ? launch<XPASS_WIDE, 2>(p, grid, st) : launch<XPASS, 2>(p, grid, st);
 }
 
 cudaError_t umma_final(const FinalArgs& a, int32_t* status, cudaStream_t st) {

@@ -45,6 +45,13 @@ struct XpassArgs {
   // 1: 256 x 512 tiles (two N = 256 MMAs per K step, one TMEM accumulator);
   // 0: 256 x 256 tiles (double-buffered accumulator).  Ignored for z32.
   int wide;
+  // Stream-K as in FinalArgs (few row tiles, e.g. a decode step): a tile
+  // split between CTA pairs gets the others' fp32 partials added into its
+  // accumulator before the epilogue.  Not with z32.
+  float* sk_part;
+  size_t sk_bytes;
+  int32_t* sync;  // kSyncWords zeroed words (left zeroed)
+  int stream_k;   // -1 by the wave fill, 0 never, 1 whenever sk_part fits
 };
 
 // final: y [N, d] = sum_j hsh[:, jG:(j+1)G] W_o,sh_j^T + uhat W_up^T
