@@ -201,10 +201,10 @@ LMOE_API lmoe_status moe_router_losses(const lmoe_dims* dims, const float* logit
  * `stream`; no host synchronisation.  The router logits stay in the
  * workspace for moe_router_losses.  Results are bitwise repeatable for given
  * dims on a given GPU.  When whole output tiles would fill the SMs' last wave
- * below 90%, the final GEMM (bf16) splits the K loop of some tiles between
- * CTA pairs (stream-K) and adds the fp32 partials in a fixed order; the
- * environment variable LMOE_STREAM_K=0 turns that off, =1 uses it whenever
- * its scratch fits. */
+ * below 90%, the x-pass and the final GEMM (bf16) split the K loop of some
+ * tiles between CTA pairs (stream-K) and add the fp32 partials in a fixed
+ * order; the environment variable LMOE_STREAM_K=0 turns that off, =1 uses it
+ * whenever its scratch fits. */
 LMOE_API lmoe_status latent_moe_forward(const lmoe_dims* dims, const lmoe_weights* weights, const void* x,
                                void* y, int32_t* ids_out, float* probs_out, int32_t* counts_out,
                                void* ws, size_t ws_bytes, lmoe_stream stream);

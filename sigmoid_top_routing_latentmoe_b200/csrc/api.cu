@@ -211,8 +211,9 @@ static Layout layout(const lmoe_dims* d, bool host_copies) {
   L.tiles2 = take((size_t)L.max_tiles * sizeof(int4));
   L.zp = take((size_t)P * d->latent * es);
   L.h = take((size_t)P * d->ff_routed * es);
-  // The final GEMM's stream-K partials reuse [zp, eo), dead by then; this
-  // tops it up to one 256-row tile of fp32 per CTA pair (up to kSkMaxPairs).
+  // The stream-K partials of the x-pass (before the dispatch writes zp) and of
+  // the final GEMM (after the routed GEMMs) reuse [zp, eo); this tops it up
+  // to one 256-row tile of fp32 per CTA pair (up to kSkMaxPairs).
   if (d->dtype == LMOE_BF16) {
     const size_t bn_max = d->d >= 4096 ? 512 : 256;
     const size_t need = (size_t)kSkMaxPairs * 2 * 128 * bn_max * 4, have = off - L.zp;
@@ -288,20 +289,15 @@ static lmoe_status run_route(const lmoe_dims* d, const void* x, const void* w_r,
   return LMOE_OK;
 }
 
-// The bf16 routed GEMMs run on CTA pairs over 256-row tiles when experts get
-// 64 to 256 sorted pairs on average: one pair tile then covers an expert's
-// rows, so its weights stream once per output tile, half through each SM (at
-// the K3 width, 146 rows per expert: W_o GEMM 1093 -> 889 us).  With more rows
-// per expert (512 at the 0.5b shape, 2048 at the mid one) single CTAs over
-// 128-row tiles were faster (0.5b: 18 + 11 us against 27 + 17 us), and for
-// decode-like loads of a few rows a 256-row MMA would mostly multiply empty
-// rows.
-// Routed GEMMs on CTA pairs over <= 256-row tiles, or single CTAs over <= 128.
-// Pairs when experts average 64 to 256 pairs (one tile per expert: its weights
-// stream once per output tile); with more, GEMM1 stays on pairs only for a
+// The bf16 routed GEMMs run on CTA pairs over <= 256-row tiles, or on single
+// CTAs over <= 128.  Pairs when experts average 64 to 256 sorted pairs: one
+// pair tile then covers an expert's rows, so its weights stream once per
+// output tile, half through each SM (K3 width, 146 rows per expert: W_o GEMM
+// 1093 -> 889 us).  With more rows per expert GEMM1 stays on pairs only for a
 // long K (l >= 1024; mid shape, 2048 rows per expert: GEMM1 528 -> 469 us on
-// pairs, GEMM2 280 -> 418 us, so GEMM2 stays single; 0.5b shape, l = 384:
-// both slower on pairs, 14.7 -> 19.8 and 8.1 -> 10.8 us).
+// pairs, while GEMM2 went 280 -> 418 us, so GEMM2 stays single; 0.5b shape,
+// l = 384: both slower on pairs, 14.7 -> 19.8 and 8.1 -> 10.8 us).  For
+// decode-like loads of a few rows a 256-row MMA would mostly multiply empty rows.
 static bool routed_pairs(const lmoe_dims* d, int gemm) {
   const int64_t pairs = d->n_tokens * (int64_t)d->top_k, R = d->n_routed;
   if (d->dtype != LMOE_BF16 || pairs < 64 * R) return false;
@@ -406,8 +402,8 @@ static lmoe_status run_expert_ffn(const lmoe_dims* d, const void* z, const int32
   return LMOE_OK;
 }
 
-// Stream-K for the final GEMM: chosen by the wave fill unless LMOE_STREAM_K
-// is 0 (never) or 1 (whenever its scratch fits).
+// Stream-K for the x-pass and the final GEMM: chosen by the wave fill unless
+// LMOE_STREAM_K is 0 (never) or 1 (whenever its scratch fits).
 static int stream_k_mode() {
   if (const char* v = getenv("LMOE_STREAM_K")) {
     if (v[0] == '0') return 0;
