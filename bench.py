@@ -266,6 +266,41 @@ def run_reference(args, wl):
     return 0
 
 
+def run_library_gemm_shapes(args, wl):
+    """Context for the roofline: cuBLAS (torch.matmul, bf16, fp32 accumulation)
+    on plain GEMMs of the layer's two dense shapes -- the x-pass [N, d] x
+    [d, l + R + 2 S G] and the final GEMM [N, S G + l] x [S G + l, d] -- and
+    on an 8192^3 square, timed like the forward (CUDA events, L2 flushed
+    before each call).  None of this is on the product path."""
+    import torch
+    dev = torch.device("cuda", 0)
+    N, d, L, R, S, G = wl.n_tokens, wl.d, wl.latent, wl.n_routed, wl.n_shared, wl.ff_shared
+    shapes = {"xpass": (N, d, L + R + 2 * S * G), "final": (N, S * G + L, d),
+              "square": (8192, 8192, 8192)}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = {"workload": wl.name, "what": "cuBLAS bf16 plain GEMM [M,K] x [K,N], us and TFLOP/s"}
+    for name, (M, K, Nn) in shapes.items():
+        a = torch.randn(M, K, device=dev, dtype=torch.bfloat16)
+        b = torch.randn(Nn, K, device=dev, dtype=torch.bfloat16)
+        for _ in range(max(3, args.warmup)):
+            a @ b.t()
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            a @ b.t()
+            e1.record()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        us = total / args.steps * 1e3
+        out[name] = {"M": M, "K": K, "N": Nn, "us": round(us, 2),
+                     "tflops": round(2.0 * M * K * Nn / (us * 1e-6) / 1e12, 1)}
+    print(json.dumps(out))
+    return 0
+
+
 def run_memory_kernels(args, wl):
     """Routing, dispatch and combine called on their own through the C ABI at the
     workload's shapes (synthetic activations; no expert weights), each timed with
@@ -431,6 +466,8 @@ def main():
                     help="time moe_route / moe_dispatch / moe_combine on their own instead")
     ap.add_argument("--backward", action="store_true",
                     help="time latent_moe_backward instead of the forward")
+    ap.add_argument("--library-gemm-shapes", action="store_true",
+                    help="time cuBLAS on plain GEMMs of the layer's dense shapes (context only)")
     ap.add_argument("--sustained-seconds", type=float, default=1.0,
                     help="length of the back-to-back replay pass whose clocks are reported as "
                          "clocks_sustained (0: no such pass, e.g. under a profiler)")
@@ -438,6 +475,8 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     if args.memory_kernels:
         return run_memory_kernels(args, wl)
+    if args.library_gemm_shapes:
+        return run_library_gemm_shapes(args, wl)
     if args.backward:
         return run_backward_bench(args, wl)
     if args.impl == "reference":
