@@ -497,6 +497,27 @@ def test_routed_gemms_on_different_tile_heights():
     assert rel_err(host(eo)[rows], exp_eo) <= 2e-2
 
 
+@pytest.mark.parametrize("name,n,colscan", [("halfb_uniform", 4096, False), ("mid", 2200, False),
+                                            ("k3_width", 320, True)])
+def test_forward_launches_follow_the_plan(name, n, colscan):
+    """The launches of one forward are the ones lmoe_forward_plan reports: the
+    x-pass, top-k for R > 32, histogram (+ column scan for a large count
+    matrix) + scatter, GEMM2's own tile list when the two routed GEMMs use
+    different tile heights, the gather unless the scatter copies the rows, the
+    two routed GEMMs, the combine unless it is fused, and the final GEMM."""
+    wl = W[name].with_tokens(n)
+    plan = lm.forward_plan(ldims(wl))
+    expected = (1 + (wl.n_routed > 32) + 2 + colscan
+                + (plan["gemm1_pairs"] != plan["gemm2_pairs"]) + (not plan["rows_in_scatter"])
+                + 2 + (not plan["combine_fused"]) + 1)
+    inp = prepare(wl)
+    dev = device_inputs(inp)
+    _run_forward(wl, dev)          # first call: one-time setup outside the count
+    lm.launch_count(reset=True)
+    _run_forward(wl, dev)
+    assert lm.launch_count() == expected, (plan, expected)
+
+
 def test_wide_routed_gemm_parity():
     """Routed experts at the K3 latent width (l = 3584) with 64..256 rows per
     expert: CTA pairs and 256 x 512 tiles of 256 hidden units for GEMM1.
