@@ -270,7 +270,8 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
  *   GEMM1_PAIRS / GEMM2_PAIRS  routed GEMM1 / GEMM2 on CTA pairs (256-row tiles);
  *   GEMM1_WIDE        routed GEMM1 on 256 x 512 tiles;
  *   ROWS_IN_SCATTER   the dispatch's scatter writes the sorted copy of z
- *                     (else a gather kernel does).
+ *                     (at most 16 MiB and at least 4096 pairs; else a gather
+ *                     kernel does).
  * The final GEMM's stream-K choice is made at launch and not reported here.
  * EINVAL on bad dims or flags == NULL. */
 enum {

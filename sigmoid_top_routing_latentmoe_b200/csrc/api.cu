@@ -419,6 +419,16 @@ static int xpass_wide(const lmoe_dims* d) {
   return d->d >= 2048 ? 1 : 0;
 }
 
+// The scatter also writes the sorted copy of z when it is at most 16 MiB and
+// there are at least 4096 pairs (enough chunks to spread the copy over many
+// CTAs); otherwise the gather kernel does (decode step, 1024 pairs: dispatch +
+// copy 26 -> 17 us).
+static bool rows_in_scatter(const lmoe_dims* d) {
+  const size_t es = d->dtype == LMOE_BF16 ? 2 : 4;
+  const int64_t P = d->n_tokens * (int64_t)d->top_k;
+  return (uint64_t)P * d->latent * es <= (16u << 20) && P >= 4096;
+}
+
 // The combine inside the final GEMM (bf16, l <= 1024, <= 64 MB of expert outputs).
 static bool combine_fused(const lmoe_dims* d) {
   return d->dtype == LMOE_BF16 && d->latent <= 1024 &&
@@ -479,9 +489,9 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
               "route_topk");
   }
   // step 3: dispatch, routed experts, combine + RMSNorm
-  // Small sorted copies of z (up to 16 MiB) are made by the scatter itself, saving a
-  // launch; larger ones by the gather kernel, which has more memory parallelism.
-  const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * sizeof(T) <= (16u << 20);
+  // Mid-sized sorted copies of z are made by the scatter itself, saving a
+  // launch; others by the gather kernel (rows_in_scatter).
+  const bool fuse_rows = rows_in_scatter(d);
   LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
   LMOE_TRY(run_expert_ffn<T>(d, z, perm, offsets, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
   // For l <= 1024 and up to 64 MB of expert outputs the combine runs inside
@@ -560,9 +570,9 @@ static lmoe_status run_forward(const lmoe_dims* d, const lmoe_weights* w, const 
   // step 2: routing
   LMOE_TRY(run_route<T>(d, x, w->w_router, w->expert_bias, ids, probs, ws, st));
   // step 3: dispatch, routed experts, combine + RMSNorm
-  // Small sorted copies of z (up to 16 MiB) are made by the scatter itself, saving a
-  // launch; larger ones by the gather kernel, which has more memory parallelism.
-  const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * sizeof(T) <= (16u << 20);
+  // Mid-sized sorted copies of z are made by the scatter itself, saving a
+  // launch; others by the gather kernel (rows_in_scatter).
+  const bool fuse_rows = rows_in_scatter(d);
   LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
   LMOE_TRY(run_expert_ffn<T>(d, z, perm, offsets, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
   {
@@ -1023,8 +1033,7 @@ lmoe_status lmoe_forward_plan(const lmoe_dims* dims, int32_t* flags) {
   if (flags == nullptr) return fail(LMOE_EINVAL, "flags is NULL");
   const lmoe_dims* d = dims;
   const bool bf16 = d->dtype == LMOE_BF16;
-  const size_t es = bf16 ? 2 : 4;
-  const bool fuse_rows = (uint64_t)d->n_tokens * d->top_k * d->latent * es <= (16u << 20);
+  const bool fuse_rows = rows_in_scatter(d);
   int32_t f = 0;
   if (bf16 && combine_fused(d)) f |= LMOE_PLAN_COMBINE_FUSED;
   if (bf16 && xpass_wide(d)) f |= LMOE_PLAN_XPASS_WIDE;

@@ -87,8 +87,10 @@ def test_forward_plan(lm):
     assert on(halfb) == {"combine_fused", "rows_in_scatter"}
     assert on(mid) == {"xpass_wide", "gemm1_pairs"}     # GEMM2 on single CTAs
     assert on(k3) == {"xpass_wide", "gemm1_pairs", "gemm2_pairs", "gemm1_wide"}
-    assert on(lm.make_dims(128, 256, 128, 16, 2, 2, 256, 512, dtype=torch.float32)) \
-        == {"rows_in_scatter"}
+    # the scatter copies the sorted z rows only from 4096 pairs on (and up to 16 MiB)
+    assert on(lm.make_dims(128, 256, 128, 16, 2, 2, 256, 512, dtype=torch.float32)) == set()
+    assert "rows_in_scatter" in on(lm.make_dims(2048, 768, 384, 16, 2, 2, 768, 1536))
+    assert "rows_in_scatter" not in on(lm.make_dims(2047, 768, 384, 16, 2, 2, 768, 1536))
     flags = ctypes.c_int32(0)
     assert lm._lib.lmoe_forward_plan(ctypes.byref(halfb), None) == lm.EINVAL
     bad = lm.make_dims(4096, 770, 384, 16, 2, 2, 768, 1536)
