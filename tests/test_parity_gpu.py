@@ -344,6 +344,32 @@ def test_host_entry_point_matches_device():
     assert torch.equal(y_h, y.cpu())
 
 
+@pytest.mark.parametrize("name,n,chunks", [("halfb_uniform", 1000, "3"), ("mid", 700, "2"),
+                                           ("halfb_skewed", 4096, "8")])
+def test_host_entry_point_in_chunks(name, n, chunks, monkeypatch):
+    """latent_moe_forward_host pipelining the tokens in several chunks (x in on
+    one copy stream, each chunk's forward, y out on another, uneven last
+    chunk): y against the oracle on sampled rows and against one device-side
+    forward over all tokens (the chunks may tile the GEMMs differently, so
+    within rounding)."""
+    monkeypatch.setenv("LMOE_HOST_CHUNKS", chunks)
+    wl = W[name].with_tokens(n)
+    inp = prepare(wl)
+    dev = device_inputs(inp)
+    y, ids, probs, _, _ = _run_forward(wl, dev)
+    dims = ldims(wl)
+    ws = lm.alloc_workspace(dims, host=True)
+    x_h = dev["x"].cpu().pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    lm.latent_moe_forward_host(dims, dev, x_h, y_h, ws)
+    assert lm.get_device_status(ws) == lm.OK
+    assert rel_err(host(y_h), host(y)) <= 1e-2
+    rows = np.arange(0, n, max(1, n // 64))
+    ref = oracle.forward(odims(wl, len(rows)), oracle_weights(inp),
+                         synth.to_f32(inp["x"])[rows])
+    assert rel_err(host(y_h)[rows], ref["y"]) <= y_tol(wl)
+
+
 def test_capped_wait_reports_timeout():
     dims = lm.make_dims(8, 64, 32, 4, 2, 1, 64, 64)
     ws = lm.alloc_workspace(dims)
