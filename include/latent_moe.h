@@ -266,7 +266,8 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
 /* The launch plan latent_moe_forward takes for these dims (host only,
  * nothing is launched), as LMOE_PLAN_* bits in *flags:
  *   COMBINE_FUSED     the combine + RMSNorm runs in the final GEMM's epilogue;
- *   XPASS_WIDE        x-pass on 256 x 512 tiles;
+ *   XPASS_WIDE        x-pass on 256 x 512 tiles (not taken by the current
+ *                     rule: 256 x 256 tiles measured faster at every shape);
  *   GEMM1_PAIRS / GEMM2_PAIRS  routed GEMM1 / GEMM2 on CTA pairs (256-row tiles);
  *   GEMM1_WIDE        routed GEMM1 on 256 x 512 tiles;
  *   ROWS_IN_SCATTER   the dispatch's scatter writes the sorted copy of z

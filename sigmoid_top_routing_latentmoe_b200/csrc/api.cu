@@ -412,12 +412,14 @@ static int stream_k_mode() {
   return -1;
 }
 
-// The x-pass uses 256 x 512 tiles (no accumulator double-buffering, 1.33x the
-// FLOPs per streamed byte) when K = d is long enough for the main loop to hide
-// the epilogue: d >= 2048 (mid shape -8 %, K3 width -17 %; +3 % at d = 768).
-static int xpass_wide(const lmoe_dims* d) {
-  return d->d >= 2048 ? 1 : 0;
-}
+// The forward's x-pass runs on 256 x 256 tiles with a double-buffered
+// accumulator.  The engine's 256 x 512 x-pass tiles (1.33x the FLOPs per
+// streamed byte, one accumulator, the SiTU epilogue exposed once per tile) won
+// at d >= 2048 only while the tiles went rows-fastest over all row tiles;
+// with the grouped tile order the 256 x 256 tiles measured faster at every
+// shape (mid: x-pass 470 -> 420 us; K3 width 708 -> 688 us; decode step
+// 76 -> 59 us), so the wide x-pass is not chosen (XpassArgs.wide still works).
+static int xpass_wide(const lmoe_dims*) { return 0; }
 
 // The scatter also writes the sorted copy of z when it is at most 16 MiB and
 // there are at least 4096 pairs (enough chunks to spread the copy over many
