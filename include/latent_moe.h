@@ -272,7 +272,14 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
  *   GEMM1_WIDE        routed GEMM1 on 256 x 512 tiles;
  *   ROWS_IN_SCATTER   the dispatch's scatter writes the sorted copy of z
  *                     (at most 16 MiB and at least 4096 pairs; else a gather
- *                     kernel does).
+ *                     kernel does);
+ *   COUNTS_IN_XPASS   the x-pass's routing epilogue (bf16, R <= 32) also
+ *                     counts each 32 tokens' pairs per expert and the
+ *                     dispatch starts from those counts, with no histogram
+ *                     kernel (k dividing the counting sort's chunks and
+ *                     ceil(N / 32) * R <= 8192; the environment variable
+ *                     LMOE_XPASS_COUNTS=0 turns it off).  The permutation is
+ *                     the same either way.
  * The final GEMM's stream-K choice is made at launch and not reported here.
  * EINVAL on bad dims or flags == NULL. */
 enum {
@@ -281,7 +288,8 @@ enum {
   LMOE_PLAN_GEMM1_PAIRS = 4,
   LMOE_PLAN_GEMM2_PAIRS = 8,
   LMOE_PLAN_GEMM1_WIDE = 16,
-  LMOE_PLAN_ROWS_IN_SCATTER = 32
+  LMOE_PLAN_ROWS_IN_SCATTER = 32,
+  LMOE_PLAN_COUNTS_IN_XPASS = 64
 };
 LMOE_API lmoe_status lmoe_forward_plan(const lmoe_dims* dims, int32_t* flags);
 

@@ -173,7 +173,7 @@ def workspace_views(dims: Dims, ws: torch.Tensor) -> dict:
 
 
 PLAN_BITS = {"combine_fused": 1, "xpass_wide": 2, "gemm1_pairs": 4, "gemm2_pairs": 8,
-             "gemm1_wide": 16, "rows_in_scatter": 32}
+             "gemm1_wide": 16, "rows_in_scatter": 32, "counts_in_xpass": 64}
 
 
 def forward_plan(dims: Dims) -> dict:

@@ -206,7 +206,7 @@ static Layout layout(const lmoe_dims* d, bool host_copies) {
   L.offsets = take((size_t)(R + 1) * 4);
   L.perm = take((size_t)P * 4);
   L.inv = take((size_t)P * 4);
-  L.block_counts = take((size_t)dispatch_blocks(P) * R * 4);
+  L.block_counts = take((size_t)dispatch_count_rows(N, d->top_k) * R * 4);
   L.tiles = take((size_t)L.max_tiles * sizeof(int4));
   L.tiles2 = take((size_t)L.max_tiles * sizeof(int4));
   L.zp = take((size_t)P * d->latent * es);
@@ -310,9 +310,12 @@ static int routed_tile_m(const lmoe_dims* d, int gemm = 1) {
 
 // z != nullptr: the scatter also writes the sorted rows of z to the workspace
 // (the A operand of the routed GEMMs).
+// row_counts: the x-pass wrote the expert counts of every 32 tokens to the
+// dispatch's count scratch (counts_in_xpass), so no histogram is launched.
 static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t* counts,
                                 int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
-                                cudaStream_t st, const void* z = nullptr) {
+                                cudaStream_t st, const void* z = nullptr,
+                                bool row_counts = false) {
   const Layout L = layout(d, false);
   DispatchScratch s;
   s.block_counts = at<int32_t>(ws, L.block_counts);
@@ -323,7 +326,7 @@ static lmoe_status run_dispatch(const lmoe_dims* d, const int32_t* ids, int32_t*
   const int es = d->dtype == LMOE_BF16 ? 2 : 4;
   LMOE_CUDA(launch_dispatch(ids, d->n_tokens, d->top_k, d->n_routed, counts, offsets, perm, inv,
                             s, st, z, z != nullptr ? at<char>(ws, L.zp) : nullptr,
-                            d->latent * es, routed_tile_m(d)),
+                            d->latent * es, routed_tile_m(d), row_counts),
             "dispatch");
   return LMOE_OK;
 }
@@ -431,6 +434,17 @@ static bool rows_in_scatter(const lmoe_dims* d) {
   return (uint64_t)P * d->latent * es <= (16u << 20) && P >= 4096;
 }
 
+// With routing in the x-pass's epilogue (R <= 32) the epilogue also counts
+// each 32 tokens' pairs per expert, and the dispatch starts from those counts
+// instead of launching its histogram kernel (0.5b shape: one launch fewer).
+// LMOE_XPASS_COUNTS=0 keeps the histogram kernel.
+static bool counts_in_xpass(const lmoe_dims* d) {
+  if (const char* v = getenv("LMOE_XPASS_COUNTS"))
+    if (v[0] == '0') return false;
+  return d->dtype == LMOE_BF16 && d->n_routed <= 32 &&
+         dispatch_takes_row_counts(d->n_tokens, d->top_k, d->n_routed);
+}
+
 // The combine inside the final GEMM (bf16, l <= 1024, <= 64 MB of expert outputs).
 static bool combine_fused(const lmoe_dims* d) {
   return d->dtype == LMOE_BF16 && d->latent <= 1024 &&
@@ -465,6 +479,7 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
     LMOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * R, st), "memset");
     return LMOE_OK;
   }
+  const bool row_counts = counts_in_xpass(d);
   // steps 1, 2 and 4 in one pass over x (routing in the epilogue when R <= 32)
   {
     XpassArgs a{};
@@ -475,6 +490,7 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
     a.z = z; a.logits = logits; a.logits_ld = L.logits_ld;
     a.hsh = hsh; a.beta1 = d->beta1; a.beta2 = d->beta2;
     a.bias = w->expert_bias; a.ids = ids; a.probs = probs; a.top_k = k; a.router = d->router;
+    if (row_counts) a.row_counts = at<int32_t>(ws, L.block_counts);
     a.wide = xpass_wide(d);
     // stream-K scratch: the sorted-z / routed-hidden region, unused until the dispatch
     a.sync = at<int32_t>(ws, L.sync);
@@ -494,7 +510,8 @@ static lmoe_status run_forward_tc(const lmoe_dims* d, const lmoe_weights* w, con
   // Mid-sized sorted copies of z are made by the scatter itself, saving a
   // launch; others by the gather kernel (rows_in_scatter).
   const bool fuse_rows = rows_in_scatter(d);
-  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr));
+  LMOE_TRY(run_dispatch(d, ids, counts, offsets, perm, inv, ws, st, fuse_rows ? z : nullptr,
+                        row_counts));
   LMOE_TRY(run_expert_ffn<T>(d, z, perm, offsets, w->w_g, w->w_u, w->w_o, eo, ws, st, fuse_rows));
   // For l <= 1024 and up to 64 MB of expert outputs the combine runs inside
   // the final GEMM (its epilogue warps write RMSNorm(u) while the K loop goes
@@ -1043,6 +1060,7 @@ lmoe_status lmoe_forward_plan(const lmoe_dims* dims, int32_t* flags) {
   if (routed_pairs(d, 2)) f |= LMOE_PLAN_GEMM2_PAIRS;
   if (routed_pairs(d, 1) && d->latent >= 2048) f |= LMOE_PLAN_GEMM1_WIDE;
   if (fuse_rows) f |= LMOE_PLAN_ROWS_IN_SCATTER;
+  if (counts_in_xpass(d)) f |= LMOE_PLAN_COUNTS_IN_XPASS;
   *flags = f;
   return LMOE_OK;
 }

@@ -2,7 +2,9 @@
 // sparse dispatch, step 1): the N*k (token, expert) pairs, flattened
 // token-major, are stably sorted by expert id -- the pages' argsort(stable) +
 // bincount + cumsum -- as a deterministic counting sort over chunks of pairs:
-//   1. hist:    one CTA per chunk counts its pairs per expert,
+//   1. hist:    one CTA per chunk counts its pairs per expert (skipped when
+//               the x-pass's routing epilogue already wrote the expert
+//               counts of every 32 tokens: R <= 32),
 //   2. colscan: (large count matrices only) one CTA per 32 experts turns
 //               each expert's column of chunk counts into exclusive prefixes
 //               and the expert's total,
@@ -154,8 +156,10 @@ __global__ void empty_scan_kernel(int R, int32_t* __restrict__ counts, int32_t* 
 // Ranks each chunk's pairs inside their expert in pair order and scatters.
 // Prologue: every CTA derives, for each expert, its chunk's first sorted slot
 // -- offsets[e] (an exclusive scan of the per-expert totals) plus the pairs of
-// expert e in earlier chunks -- from the chunk counts: summed here when
-// `prefixed` is 0, or read as the column scan left them.  CTA 0 also writes
+// expert e in earlier chunks -- from the count rows: summed here when
+// `prefixed` is 0, or read as the column scan left them.  The count rows are
+// the histogram's (one per chunk, sub_rows = 1) or the x-pass's (one per 32
+// tokens, sub_rows of them per chunk); crows rows in all.  CTA 0 also writes
 // counts (unless prefixed), offsets and the routed row-tile list.
 // With z != nullptr each chunk has `subs` CTAs: all of them rank the chunk's
 // pairs (cheap), sub-CTA 0 writes perm_token / inv_pair, and sub-CTA s copies
@@ -163,8 +167,9 @@ __global__ void empty_scan_kernel(int R, int32_t* __restrict__ counts, int32_t* 
 // zp (row_vecs 16-byte vectors per row), a warp's rows copied together so that
 // many loads are in flight.
 __global__ void __launch_bounds__(kThreads) scatter_kernel(
-    const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int k, int R, int C,
-    const int32_t* __restrict__ chunk_counts, int prefixed, int32_t* __restrict__ counts,
+    const int32_t* __restrict__ ids, int64_t n_pairs, int64_t chunk, int k, int R, int crows,
+    int sub_rows, const int32_t* __restrict__ chunk_counts, int prefixed,
+    int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ n_mtiles, int4* __restrict__ tiles,
     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_pair, int subs,
     const uint4* __restrict__ z, uint4* __restrict__ zp, int row_vecs, int tile_m) {
@@ -181,6 +186,31 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
   const int cb = blockIdx.x / subs, sub = blockIdx.x - cb * subs;
   for (int i = threadIdx.x; i < kWarps * R; i += kThreads) wcnt[i] = 0;
   if (threadIdx.x == 0) carry[0] = carry[1] = 0;
+  const int lim = cb * sub_rows;  // count rows before this chunk
+  // R <= 32: warp w sums rows w, w + 8, ... (lane = expert), then the warps'
+  // partial sums are added per expert
+  __shared__ int32_t part[2][kWarps][32];
+  const bool by_warps = !prefixed && R <= 32;
+  if (by_warps) {
+    int32_t f = 0, t = 0;
+    if (lane < R) {
+      for (int c0 = warp; c0 < crows; c0 += kWarps * 16) {  // 16 loads in flight
+        int32_t v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int c = c0 + u * kWarps;
+          v[u] = c < crows ? chunk_counts[(int64_t)c * R + lane] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          f += c0 + u * kWarps < lim ? v[u] : 0;
+          t += v[u];
+        }
+      }
+    }
+    part[0][warp][lane] = f;
+    part[1][warp][lane] = t;
+  }
   __syncthreads();
   for (int e0 = 0; e0 < R; e0 += kThreads) {
     const int e = e0 + threadIdx.x;
@@ -189,15 +219,21 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(
       if (prefixed) {
         first = chunk_counts[(int64_t)cb * R + e];
         tot = counts[e];
+      } else if (by_warps) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          first += part[0][w][e];
+          tot += part[1][w][e];
+        }
       } else {
-        for (int c0 = 0; c0 < C; c0 += 32) {  // up to 32 loads in flight
+        for (int c0 = 0; c0 < crows; c0 += 32) {  // up to 32 loads in flight
           int32_t v[32];
 #pragma unroll
           for (int u = 0; u < 32; ++u)
-            v[u] = c0 + u < C ? chunk_counts[(int64_t)(c0 + u) * R + e] : 0;
+            v[u] = c0 + u < crows ? chunk_counts[(int64_t)(c0 + u) * R + e] : 0;
 #pragma unroll
           for (int u = 0; u < 32; ++u) {
-            first += c0 + u < cb ? v[u] : 0;
+            first += c0 + u < lim ? v[u] : 0;
             tot += v[u];
           }
         }
@@ -426,10 +462,21 @@ int dispatch_blocks(int64_t n_pairs) {
   return (int)((n_pairs + chunk - 1) / chunk);
 }
 
+bool dispatch_takes_row_counts(int64_t n, int k, int R) {
+  const int64_t n_pairs = n * k;
+  if (n_pairs == 0 || R > 32) return false;
+  const int64_t rows = (n + kCountRowTokens - 1) / kCountRowTokens;
+  return chunk_pairs(n_pairs) % ((int64_t)kCountRowTokens * k) == 0 && rows * R <= kSmallScan;
+}
+
+int64_t dispatch_count_rows(int64_t n, int k) {
+  return std::max<int64_t>(dispatch_blocks(n * k), (n + kCountRowTokens - 1) / kCountRowTokens);
+}
+
 cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
                             const DispatchScratch& s, cudaStream_t st, const void* z, void* zp,
-                            int row_bytes, int tile_m) {
+                            int row_bytes, int tile_m, bool row_counts) {
   const int64_t n_pairs = n * k;
   const int64_t chunk = chunk_pairs(n_pairs);
   const int nb = dispatch_blocks(n_pairs);
@@ -438,13 +485,21 @@ cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t
     return launch_pdl(empty_scan_kernel, dim3(1), dim3(32), 0, st, 1, R, counts, offsets,
                       s.n_mtiles);
   }
-  cudaError_t e = set_smem(hist_kernel, R * sizeof(int32_t));
-  if (e != cudaSuccess) return e;
-  count_launch();
-  e = launch_pdl(hist_kernel, dim3(nb), dim3(kThreads), R * sizeof(int32_t), st, 1, ids, n_pairs,
-                 chunk, R, s.block_counts, s.status);
-  if (e != cudaSuccess) return e;
-  const int prefixed = (int64_t)nb * R > kSmallScan ? 1 : 0;
+  if (row_counts && !dispatch_takes_row_counts(n, k, R)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaSuccess;
+  int crows = nb, sub_rows = 1;
+  if (row_counts) {
+    crows = (int)((n + kCountRowTokens - 1) / kCountRowTokens);
+    sub_rows = (int)(chunk / ((int64_t)kCountRowTokens * k));
+  } else {
+    e = set_smem(hist_kernel, R * sizeof(int32_t));
+    if (e != cudaSuccess) return e;
+    count_launch();
+    e = launch_pdl(hist_kernel, dim3(nb), dim3(kThreads), R * sizeof(int32_t), st, 1, ids,
+                   n_pairs, chunk, R, s.block_counts, s.status);
+    if (e != cudaSuccess) return e;
+  }
+  const int prefixed = !row_counts && (int64_t)nb * R > kSmallScan ? 1 : 0;
   if (prefixed) {
     count_launch();
     e = launch_pdl(colscan_kernel, dim3((R + 31) / 32), dim3(kThreads), 0, st, 1, s.block_counts,
@@ -458,7 +513,8 @@ cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t
   const int subs = z != nullptr ? std::max(1, std::min(16, (2 * 148 + nb - 1) / nb)) : 1;
   count_launch();
   e = launch_pdl(scatter_kernel, dim3((unsigned)(nb * subs)), dim3(kThreads), smem, st, 1, ids,
-                 n_pairs, chunk, k, R, nb, (const int32_t*)s.block_counts, prefixed, counts,
+                 n_pairs, chunk, k, R, crows, sub_rows, (const int32_t*)s.block_counts, prefixed,
+                 counts,
                  offsets, s.n_mtiles, s.tiles, perm_token, inv_pair, subs,
                  static_cast<const uint4*>(z), static_cast<uint4*>(zp), row_bytes / 16, tile_m);
   if (e != cudaSuccess) return e;

@@ -30,20 +30,35 @@ cudaError_t launch_router_losses(const float* logits, int64_t ld, const int32_t*
                                  int32_t* status, float* out, cudaStream_t st);
 
 // ----------------------------------------------------------- permutation
+// Tokens per row of the expert counts the x-pass's routing epilogue writes
+// (one warp's rows): row j holds, for each expert, the pairs of tokens
+// [32 j, 32 j + 32) routed to it.
+constexpr int kCountRowTokens = 32;
+
 struct DispatchScratch {
-  int32_t* block_counts;  // [n_blocks, R]
+  int32_t* block_counts;  // [dispatch_count_rows, R]: chunk counts or the x-pass's row counts
   int32_t* status;        // workspace status word
   int32_t* n_mtiles;      // out: number of routed row tiles
   int4* tiles;            // out: [max_tiles] (expert, row0, rows, 0)
 };
 int dispatch_blocks(int64_t n_pairs);
+// Rows of block_counts the dispatch needs (either kind of count row).
+int64_t dispatch_count_rows(int64_t n, int k);
+// Whether the dispatch can start from per-32-token expert counts (R <= 32,
+// each chunk of the counting sort a whole number of count rows, and the rows
+// few enough to be summed inside the scatter).
+bool dispatch_takes_row_counts(int64_t n, int k, int R);
 // With z != nullptr the scatter also copies each pair's z row (row_bytes, a
 // multiple of 16) to its sorted slot in zp.  The routed tile list holds tiles
-// of at most tile_m rows of one expert (kTileM or kRoutedPairTileM).
+// of at most tile_m rows of one expert (kTileM or kRoutedPairTileM).  With
+// row_counts, block_counts already holds the x-pass's count rows for these
+// ids and the histogram kernel is not launched (cudaErrorInvalidValue when
+// dispatch_takes_row_counts is false).
 cudaError_t launch_dispatch(const int32_t* ids, int64_t n, int k, int R, int32_t* counts,
                             int32_t* offsets, int32_t* perm_token, int32_t* inv_pair,
                             const DispatchScratch& s, cudaStream_t st, const void* z = nullptr,
-                            void* zp = nullptr, int row_bytes = 0, int tile_m = 128);
+                            void* zp = nullptr, int row_bytes = 0, int tile_m = 128,
+                            bool row_counts = false);
 cudaError_t launch_build_tiles(const int32_t* offsets, int R, int32_t* n_mtiles, int4* tiles,
                                cudaStream_t st, int tile_m = 128);
 // Consistency check of a permutation (bitmap: (N k + 31) / 32 words of scratch).

@@ -134,6 +134,7 @@ struct Params {
   const float* bias;
   int32_t* ids;
   float* probs;
+  int32_t* row_counts;                 // XPASS with fuse_topk: per 32 rows, pairs per expert
   void* out0;
   void* out1;
   void* out2;
@@ -1054,6 +1055,30 @@ __device__ __forceinline__ void route_row32(const Params& p, const float (&lg)[3
   for (int slot = 0; slot < p.top_k; ++slot) probs[slot] = probs[slot] / den;
 }
 
+// Pairs per expert among one warp's 32 rows of a routed x-pass tile (the
+// dispatch's count row grow0 / 32): lane e counts the ids equal to e, matching
+// the five bits of each id by ballots.  The warp's own ids were just written
+// by its lanes, each lane reading its own row.  Kept out of line so that the
+// epilogue's registers stay as they are.
+__device__ __noinline__ void count_row_experts(const int32_t* ids, int top_k, int R,
+                                               int32_t* row_counts, int64_t grow0, int rows) {
+  const int lane = threadIdx.x & 31;
+  const unsigned have = __ballot_sync(0xffffffffu, lane < rows);
+  int32_t cnt = 0;
+#pragma unroll 1
+  for (int j = 0; j < top_k; ++j) {
+    const int e = lane < rows ? ids[(grow0 + lane) * top_k + j] : 0;
+    unsigned m = have;
+#pragma unroll
+    for (int bit = 0; bit < 5; ++bit) {
+      const unsigned set = __ballot_sync(0xffffffffu, (e >> bit) & 1);
+      m &= ((lane >> bit) & 1) ? set : ~set;
+    }
+    cnt += __popc(m);
+  }
+  if (lane < R) row_counts[(grow0 >> 5) * R + lane] = cnt;
+}
+
 // x-pass stream-K share of one tile (see the epilogue).  Role 1: store the
 // raw accumulator (NB 64-column blocks of this warp's lane quarter, if any
 // of its rows exist) and count
@@ -1268,6 +1293,8 @@ __device__ __forceinline__ void epilogue(const Params& p, uint64_t* tfull, uint6
                         make_float4(lg[g4 * 4], lg[g4 * 4 + 1], lg[g4 * 4 + 2], lg[g4 * 4 + 3]);
                 route_row32(p, lg, grow0 + lane);
               }
+              if (p.row_counts != nullptr && rows > 0)
+                count_row_experts(p.ids, p.top_k, p.R, p.row_counts, grow0, rows);
             }
             continue;
           }
@@ -1674,6 +1701,7 @@ cudaError_t umma_xpass(const XpassArgs& a, int32_t* status, cudaStream_t st) {
   p.bias = a.bias;
   p.ids = a.ids;
   p.probs = a.probs;
+  p.row_counts = p.fuse_topk ? a.row_counts : nullptr;
   const int total = (int)((a.N + 2 * BM - 1) / (2 * BM)) * p.n_tiles;
   const int units = a.max_units > 0 ? std::min(a.max_units, num_sms() / 2) : num_sms() / 2;
   if (f32) return launch<XPASS_F32, 2>(p, std::min(total, units), st);

@@ -41,6 +41,10 @@ struct XpassArgs {
   int32_t* ids;
   float* probs;
   int top_k;
+  // With routing in the epilogue and row_counts != nullptr: row j of
+  // row_counts [ceil(N / 32), R] gets, for each expert, the number of pairs of
+  // tokens [32 j, 32 j + 32) routed to it (the dispatch's count rows).
+  int32_t* row_counts;
   int max_units;  // at most this many CTA pairs (0: one per pair of SMs)
   // 1: 256 x 512 tiles (two N = 256 MMAs per K step, one TMEM accumulator);
   // 0: 256 x 256 tiles (double-buffered accumulator).  Ignored for z32.

@@ -84,9 +84,16 @@ def test_forward_plan(lm):
     halfb = lm.make_dims(4096, 768, 384, 16, 2, 2, 768, 1536)
     mid = lm.make_dims(16384, 2048, 1024, 64, 8, 1, 1024, 4096)
     k3 = lm.make_dims(8192, 7168, 3584, 896, 16, 1, 512, 2048)
-    assert on(halfb) == {"combine_fused", "rows_in_scatter"}
+    assert on(halfb) == {"combine_fused", "rows_in_scatter", "counts_in_xpass"}
     assert on(mid) == {"gemm1_pairs"}     # GEMM2 on single CTAs
     assert on(k3) == {"gemm1_pairs", "gemm2_pairs", "gemm1_wide"}
+    # the x-pass counts the pairs per expert for R <= 32 when each chunk of the
+    # counting sort is whole rows of 32 tokens and the rows are few enough
+    assert "counts_in_xpass" in on(lm.make_dims(16384, 768, 384, 16, 2, 2, 768, 1536))
+    assert "counts_in_xpass" not in on(lm.make_dims(16416, 768, 384, 16, 2, 2, 768, 1536))
+    assert "counts_in_xpass" not in on(lm.make_dims(4096, 768, 384, 16, 3, 2, 768, 1536))
+    assert "counts_in_xpass" in on(lm.make_dims(4096, 768, 384, 32, 8, 2, 768, 1536))
+    assert "counts_in_xpass" not in on(lm.make_dims(4096, 768, 384, 33, 2, 2, 768, 1536))
     # the scatter copies the sorted z rows only from 4096 pairs on (and up to 16 MiB)
     assert on(lm.make_dims(128, 256, 128, 16, 2, 2, 256, 512, dtype=torch.float32)) == set()
     assert "rows_in_scatter" in on(lm.make_dims(2048, 768, 384, 16, 2, 2, 768, 1536))

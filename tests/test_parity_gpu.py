@@ -527,13 +527,15 @@ def test_routed_gemms_on_different_tile_heights():
                                             ("k3_width", 320, True)])
 def test_forward_launches_follow_the_plan(name, n, colscan):
     """The launches of one forward are the ones lmoe_forward_plan reports: the
-    x-pass, top-k for R > 32, histogram (+ column scan for a large count
-    matrix) + scatter, GEMM2's own tile list when the two routed GEMMs use
-    different tile heights, the gather unless the scatter copies the rows, the
-    two routed GEMMs, the combine unless it is fused, and the final GEMM."""
+    x-pass, top-k for R > 32, histogram unless the x-pass counted the pairs (+
+    column scan for a large count matrix) + scatter, GEMM2's own tile list
+    when the two routed GEMMs use different tile heights, the gather unless the
+    scatter copies the rows, the two routed GEMMs, the combine unless it is
+    fused, and the final GEMM."""
     wl = W[name].with_tokens(n)
     plan = lm.forward_plan(ldims(wl))
-    expected = (1 + (wl.n_routed > 32) + 2 + colscan
+    assert plan["counts_in_xpass"] == (name == "halfb_uniform")
+    expected = (1 + (wl.n_routed > 32) + (not plan["counts_in_xpass"]) + 1 + colscan
                 + (plan["gemm1_pairs"] != plan["gemm2_pairs"]) + (not plan["rows_in_scatter"])
                 + 2 + (not plan["combine_fused"]) + 1)
     inp = prepare(wl)
@@ -570,3 +572,37 @@ def test_wide_routed_gemm_parity():
     exp_eo = np.stack([oracle.situ(ow["w_g"][e], ow["w_u"][e], ow["w_o"][e], z[perm[r]],
                                    wl.beta1, wl.beta2)[0] for r, e in zip(rows, expert)])
     assert rel_err(host(eo)[rows], exp_eo) <= 2e-2
+
+
+@pytest.mark.parametrize("n,over", [(4096, {}), (1000, {}), (1, {}),
+                                    (777, dict(top_k=8, n_routed=32)),
+                                    (5000, dict(top_k=1)),
+                                    (16384, dict(top_k=4, n_routed=8))])
+def test_counts_in_xpass_match_the_histogram(n, over, monkeypatch):
+    """Routing in the x-pass's epilogue (R <= 32): the expert counts of every 32
+    tokens written there replace the dispatch's histogram kernel.  The forward
+    is bit-identical with the histogram kernel (LMOE_XPASS_COUNTS=0): ids,
+    counts, the permutation and y; ragged token counts (partial 32-token rows,
+    a partial last chunk), k = 1, 2, 4, 8 (1, 4, 8 or 32 count rows per chunk
+    of the counting sort)."""
+    wl = W["halfb_uniform"].with_tokens(n).replace(**over)
+    dims = ldims(wl)
+    assert lm.forward_plan(dims)["counts_in_xpass"]
+    inp = prepare(wl)
+    dev = device_inputs(inp)
+    monkeypatch.delenv("LMOE_XPASS_COUNTS", raising=False)
+    y, ids, probs, counts, ws = _run_forward(wl, dev)
+    v = lm.workspace_views(dims, ws)
+    got = [host(v[k]).copy() for k in ("offsets", "perm", "inv")]
+    monkeypatch.setenv("LMOE_XPASS_COUNTS", "0")
+    assert not lm.forward_plan(dims)["counts_in_xpass"]
+    y0, ids0, probs0, counts0, ws0 = _run_forward(wl, dev)
+    v0 = lm.workspace_views(dims, ws0)
+    assert torch.equal(ids, ids0) and torch.equal(counts, counts0)
+    for a, b in zip(got, [host(v0[k]) for k in ("offsets", "perm", "inv")]):
+        np.testing.assert_array_equal(a, b)
+    assert torch.equal(y, y0)
+    h_ids = host(ids)
+    check_permutation_properties(h_ids, host(counts), got[0], got[1], got[2], wl.n_routed)
+    rows = np.unique(np.linspace(0, n - 1, min(n, 64)).astype(np.int64))
+    _compare_forward(wl, inp, y, ids, probs, rows)
