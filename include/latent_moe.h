@@ -276,7 +276,8 @@ LMOE_API lmoe_status latent_moe_forward_host(const lmoe_dims* dims, const lmoe_w
  *   COUNTS_IN_XPASS   the x-pass's routing epilogue (bf16, R <= 32) also
  *                     counts each 32 tokens' pairs per expert and the
  *                     dispatch starts from those counts, with no histogram
- *                     kernel (k dividing the counting sort's chunks and
+ *                     kernel (each chunk of pairs the counting sort takes is
+ *                     whole 32-token rows, always so for k = 1, 2, 4, 8, and
  *                     ceil(N / 32) * R <= 8192; the environment variable
  *                     LMOE_XPASS_COUNTS=0 turns it off).  The permutation is
  *                     the same either way.
